@@ -1,0 +1,249 @@
+/*
+ * mk.h - C ABI of the decode-step megakernel library (libmk.so).
+ *
+ * One low-batch decode step of a Qwen3-style decoder runs as ONE persistent
+ * kernel launch on one GPU: an SM-level task graph (tGraph) is built on the
+ * host once, and a worker kernel with one CTA per SM executes it with event
+ * counters and per-SM task queues, with no further launches inside the step.
+ *
+ * Where the operations come from:
+ *   - "MPK: A Compiler and Runtime for Mega-Kernelizing Tensor Programs",
+ *     Abstract: an SM-level graph captures data dependencies per SM-sized
+ *     task; an in-kernel runtime executes the tasks inside one persistent
+ *     kernel with decentralized scheduling across SMs.
+ *   - MPK review (zhaifeiyue), section 2.4: event fusion, normalisation so
+ *     that every task has at most one dependency event and one trigger event,
+ *     BFS linearisation so that an event's fan-out is a [first, last] task
+ *     range, scheduling with only atomicAdd and local state.
+ *   - "Mirage Persistent Kernel (MPK)" page, section 5.1 (worker kernel with
+ *     one resident CTA per worker, dispatch-only scheduler beside it) and
+ *     section 5.3 (one call runs the decode; the baseline launches one kernel
+ *     per operator and takes the argmax of the logits).
+ *
+ * Conventions for every call:
+ *   - Every function returns mk_status (MK_OK = 0 on success); nothing throws
+ *     across the ABI.  mk_last_error(h) gives a text for the last failure on h.
+ *   - Pointers named d_* are device pointers on the handle's device; other
+ *     pointers are host pointers.  Streams are cudaStream_t passed as void*
+ *     (NULL = the legacy default stream).
+ *   - bf16 data is IEEE bfloat16 bit patterns (uint16_t); matrices are
+ *     row-major [out_features][in_features], the nn.Linear layout.
+ *   - Calls on one handle are not thread-safe; use one handle per thread.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mk_handle mk_handle;
+
+typedef enum {
+  MK_OK = 0,
+  MK_ERR_ARG = -1,        /* bad argument or unsupported shape */
+  MK_ERR_CUDA = -2,       /* a CUDA runtime call failed */
+  MK_ERR_OOM = -3,        /* device or host allocation failed */
+  MK_ERR_GRAPH = -4,      /* graph construction found an inconsistency (a cycle) */
+  MK_ERR_NOT_LOADED = -5, /* mk_decode_step before mk_load_weights */
+  MK_ERR_TIMEOUT = -6,    /* a device-side event wait ran out of time */
+  MK_ERR_DEVICE = -7      /* device-side check failed (kv_len or token range) */
+} mk_status;
+
+/* Task types as stored in the task table (mk_graph_view.task_type). */
+enum {
+  MK_TASK_GENERIC = 0, /* task of a graph built by mk_graph_from_edges */
+  MK_TASK_EMBED = 1,   /* x0[b] = float(E[token_b])                                  */
+  MK_TASK_QKV = 2,     /* RMSNorm prologue, q/k/v rows of one kv-group-aligned tile    */
+  MK_TASK_ATTN = 3,    /* one (sequence, kv head, KV split) of decode attention        */
+  MK_TASK_MERGE = 4,   /* online-softmax merge of the splits of one (sequence, kv head) */
+  MK_TASK_OPROJ = 5,   /* O projection tile, residual add epilogue                     */
+  MK_TASK_GATEUP = 6,  /* RMSNorm prologue, gate/up tile, SiLU(g)*u epilogue           */
+  MK_TASK_DOWN = 7,    /* down projection tile, residual add epilogue                  */
+  MK_TASK_LMHEAD = 8,  /* final RMSNorm prologue, LM-head tile, partial argmax epilogue */
+  MK_TASK_ARGMAX = 9,  /* argmax over the partials, token write, kv_len += 1           */
+  MK_TASK_EMPTY = 10   /* normalisation task: waits on one event, triggers another     */
+};
+
+/* Shape of the decoder and of the batch state one handle serves. */
+typedef struct {
+  int n_layers;        /* decoder layers (Ly) */
+  int hidden;          /* H, multiple of 256 */
+  int n_q_heads;       /* Hq */
+  int n_kv_heads;      /* Hkv, divides Hq */
+  int head_dim;        /* D: 64 or 128 */
+  int ffn;             /* F, multiple of 256 */
+  int vocab;           /* V */
+  int tied_embeddings; /* 1: the LM head is the embedding matrix */
+  float rms_eps;       /* epsilon of every RMSNorm */
+  double rope_theta;   /* RoPE base */
+  int batch;           /* B sequences advanced per step, 1..16 */
+  int kv_capacity;     /* cache rows per (layer, sequence, kv head) */
+} mk_model_config;
+
+/* Tuning knobs; pass NULL for defaults.  A zero field also means "default". */
+typedef struct {
+  int num_workers;           /* worker CTAs W; 0 = one per SM of the device */
+  int col_align;             /* rows per GEMV task rounded up to this (16) */
+  int attn_tasks_per_worker; /* target attention tasks per worker (4) */
+  int attn_min_chunk;        /* smallest KV positions per attention task (64) */
+  int use_mma;               /* reserved: tensor-core projections for batch >= 2 */
+  int ring_stages;           /* shared-memory weight ring depth (4) */
+  int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
+  int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring (0 = off) */
+  unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
+} mk_tuning;
+
+/* Weights: device pointers, bf16, row-major [out][in].  Per-layer arrays are
+ * host arrays of n_layers device pointers.  lm_head must be NULL iff tied. */
+typedef struct {
+  const void *embed;      /* [vocab][hidden] */
+  const void *final_norm; /* [hidden] */
+  const void *lm_head;    /* [vocab][hidden] or NULL when tied */
+  const void *const *attn_norm; /* [hidden] */
+  const void *const *wq;        /* [n_q_heads*head_dim][hidden] */
+  const void *const *wk;        /* [n_kv_heads*head_dim][hidden] */
+  const void *const *wv;        /* [n_kv_heads*head_dim][hidden] */
+  const void *const *q_norm;    /* [head_dim], shared by all q heads */
+  const void *const *k_norm;    /* [head_dim], shared by all kv heads */
+  const void *const *wo;        /* [hidden][n_q_heads*head_dim] */
+  const void *const *mlp_norm;  /* [hidden] */
+  const void *const *w_gate;    /* [ffn][hidden] */
+  const void *const *w_up;      /* [ffn][hidden] */
+  const void *const *w_down;    /* [hidden][ffn] */
+} mk_weights;
+
+/* Host copies of the graph tables (owned by the handle, valid until
+ * mk_destroy).  Tasks are in linear (BFS) order; task i runs on worker
+ * i mod num_workers; worker w runs its tasks in increasing order. */
+typedef struct {
+  int32_t n_tasks, n_events, n_edges, num_workers;
+  const int32_t *task_type, *task_op, *task_layer, *task_idx, *task_dep, *task_trig;
+  const int32_t *event_count, *event_first, *event_last;
+  const int32_t *edge_src, *edge_dst; /* raw data dependencies, final task ids */
+  /* tiling chosen for the decode graph (0 for generic graphs) */
+  int32_t qkv_rows, o_rows, gu_rows, down_rows, lm_rows, attn_splits, attn_chunk;
+} mk_graph_view;
+
+/* Sizes and roofline inputs of a built handle. */
+typedef struct {
+  int32_t device, num_workers, n_tasks, n_events, n_ops;
+  int32_t smem_bytes, ring_stages, ring_stage_bytes;
+  int64_t weight_bytes;  /* bytes of the weight arena (every weight once) */
+  int64_t act_bytes;     /* bytes of the library-owned activation buffers */
+} mk_info;
+
+/*
+ * mk_plan_graph - build the task graph of one decode step on the host only
+ * (no CUDA call).  Tiling, raw events from region overlaps, fusion, reduction,
+ * normalisation and BFS linearisation follow the MPK review (zhaifeiyue),
+ * section 2.4.  num_workers must be >= 1.  The handle can be inspected with
+ * mk_graph_export and must be released with mk_destroy; it cannot run steps.
+ * Errors: MK_ERR_ARG (shape unsupported), MK_ERR_GRAPH, MK_ERR_OOM.
+ */
+mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int num_workers,
+                        mk_handle **out);
+
+/*
+ * mk_graph_from_edges - the same fusion/normalisation/linearisation pipeline
+ * on an arbitrary op-ordered task DAG (for property tests).  Task i has key
+ * (task_op[i], task_idx[i]) (keys unique); every edge src -> dst must go from
+ * an earlier op to a later one.  Host only.  Errors: MK_ERR_ARG, MK_ERR_GRAPH.
+ */
+mk_status mk_graph_from_edges(int n_tasks, const int32_t *task_op, const int32_t *task_idx,
+                              int n_edges, const int32_t *edge_src, const int32_t *edge_dst,
+                              mk_handle **out);
+
+/*
+ * mk_build_graph - plan the graph for `device` (W = its SM count unless
+ * tuning->num_workers is set), upload the task/event tables, and allocate the
+ * event counters, the step epoch, the status word and the activation buffers
+ * (all owned by the handle).  Errors: MK_ERR_ARG, MK_ERR_CUDA, MK_ERR_OOM.
+ */
+mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, int device,
+                         mk_handle **out);
+
+/*
+ * mk_load_weights - copy the caller's weights into a library-owned arena laid
+ * out in task-stream order: QKV rows group-major (per kv head: its q heads,
+ * then k, then v), gate and up rows interleaved, every task's weight tile one
+ * contiguous range.  Copies are ordered on `stream`; the caller may free its
+ * tensors once the stream has passed this call.  May be called again to
+ * replace the weights.  Errors: MK_ERR_ARG, MK_ERR_OOM, MK_ERR_CUDA.
+ */
+mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream);
+
+/*
+ * mk_decode_step - advance every sequence b by one token with ONE persistent
+ * kernel launch on `stream` (asynchronous, stream ordered):
+ *   reads d_tokens_in[b]; appends K/V at row d_kv_len[b] of every layer's
+ *   cache; attends over d_kv_len[b] + 1 rows at RoPE position d_kv_len[b];
+ *   writes d_tokens_out[b] (greedy argmax, lowest index on ties); increments
+ *   d_kv_len[b].
+ * Buffers (caller owned, device): d_tokens_in/out int32 [batch] (may be the
+ * same buffer); d_kv_len int32 [batch]; d_k_cache, d_v_cache bf16
+ * [n_layers][batch][n_kv_heads][kv_capacity][head_dim]; d_logits fp32
+ * [batch][vocab] or NULL (then logits are not stored).
+ * Device-side failures (kv_len[b] + 1 > kv_capacity or a token out of range:
+ * the step writes nothing; an event wait that times out) are recorded in the
+ * handle's status word, make later steps no-ops, and are returned by
+ * mk_sync_status.  Errors returned here: MK_ERR_NOT_LOADED, MK_ERR_ARG,
+ * MK_ERR_CUDA (for instance when the workers cannot all be co-resident).
+ */
+mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
+                         int32_t *d_kv_len, void *d_k_cache, void *d_v_cache, float *d_logits,
+                         void *stream);
+
+/*
+ * mk_decode_step_perop - the comparison path: the same task bodies, launched
+ * one grid per operator (one CTA per task, no event waits; kernel boundaries
+ * order the operators), as in the kernel-per-operator baseline of the MPK
+ * page, section 5.3.  Same arguments and results as mk_decode_step; the call
+ * only launches kernels, so it can be captured into a CUDA Graph.
+ */
+mk_status mk_decode_step_perop(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
+                               int32_t *d_kv_len, void *d_k_cache, void *d_v_cache,
+                               float *d_logits, void *stream);
+
+/* mk_sync_status - synchronize `stream`, then return the device status word
+ * (MK_OK, MK_ERR_TIMEOUT or MK_ERR_DEVICE).  detail (nullable, 4 ints):
+ * {status, task id, event id, block}.  The word stays set until mk_reset. */
+mk_status mk_sync_status(mk_handle *h, void *stream, int32_t *detail);
+
+/* mk_reset - stream-ordered: zero the event counters, the step epoch and the
+ * status word (needed after a device-side failure). */
+mk_status mk_reset(mk_handle *h, void *stream);
+
+/* mk_graph_export - fill *out with host views of the tables (see mk_graph_view). */
+mk_status mk_graph_export(const mk_handle *h, mk_graph_view *out);
+
+/* mk_get_info - sizes of a handle built with mk_build_graph. */
+mk_status mk_get_info(const mk_handle *h, mk_info *out);
+
+/* mk_final_hidden - device pointer to the fp32 [batch][hidden] residual
+ * stream after the last layer (before the final norm) of the latest step. */
+mk_status mk_final_hidden(const mk_handle *h, const float **d_ptr);
+
+/* mk_debug_set_event_count - test hook: overwrite one event's trigger count in
+ * the device table (stream ordered).  Raising it by one makes every waiter of
+ * that event time out, which exercises the bounded-wait error path. */
+mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *stream);
+
+/* mk_set_timeout_us - change the device-side bound on one event wait. */
+mk_status mk_set_timeout_us(mk_handle *h, unsigned timeout_us);
+
+/* mk_last_error - text of the last failure on h (or of the last failed
+ * constructor call when h is NULL).  Never NULL. */
+const char *mk_last_error(const mk_handle *h);
+
+/* mk_destroy - free everything the handle owns.  NULL is allowed. */
+void mk_destroy(mk_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MK_H */

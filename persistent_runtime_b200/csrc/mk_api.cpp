@@ -1,0 +1,647 @@
+// C ABI of the decode-step megakernel library (see include/mk.h).
+#include "mk.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "runtime.cuh"
+#include "tgraph.hpp"
+
+namespace mk {
+size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim);
+cudaError_t worker_configure(size_t smem);
+cudaError_t worker_max_blocks(int *blocks, size_t smem);
+cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream);
+cudaError_t launch_tasks(const Params &p, int n_ctas, size_t smem, cudaStream_t stream);
+}  // namespace mk
+
+using mk::Params;
+
+struct mk_handle {
+  mk_model_config cfg{};
+  mk_tuning tune{};
+  mk::TaskGraph graph;
+  bool host_only = true;
+  int device = -1;
+  std::string err;
+  // device state
+  void *dev_block = nullptr;  // graph tables, counters, activations, rope table
+  size_t dev_block_bytes = 0;
+  void *arena = nullptr;      // weights
+  size_t arena_bytes = 0;
+  bool loaded = false;
+  mk::DevLayer *d_layers = nullptr;
+  std::vector<mk::DevLayer> layers;
+  std::vector<int32_t> op_offset;  // into d_op_tasks
+  int32_t *d_op_tasks = nullptr;
+  Params base{};
+  size_t smem = 0;
+  int64_t act_bytes = 0;
+  int64_t weight_bytes = 0;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+mk_status fail(mk_handle *h, mk_status s, const std::string &msg) {
+  if (h)
+    h->err = msg;
+  else
+    g_last_error = msg;
+  return s;
+}
+
+mk_status cuda_fail(mk_handle *h, cudaError_t e, const char *what) {
+  return fail(h, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+mk_tuning fill_defaults(const mk_tuning *t) {
+  mk_tuning d{};
+  if (t) d = *t;
+  if (d.col_align <= 0) d.col_align = 16;
+  if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 4;
+  if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
+  if (d.ring_stages <= 0) d.ring_stages = 4;
+  if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
+  if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
+  if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
+  return d;
+}
+
+std::string check_shape(const mk_model_config &c) {
+  if (c.n_layers < 1 || c.hidden < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.ffn < 1 ||
+      c.vocab < 1 || c.batch < 1 || c.kv_capacity < 1 || c.head_dim < 2)
+    return "model dimensions must be positive";
+  if (c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
+  if (!(c.rms_eps >= 0.0f)) return "rms_eps must be >= 0";
+  return "";
+}
+
+std::string check_gpu_shape(const mk_model_config &c) {
+  std::string e = check_shape(c);
+  if (!e.empty()) return e;
+  const int rep = c.n_q_heads / c.n_kv_heads;
+  const int qd = c.n_q_heads * c.head_dim;
+  if (c.head_dim != 64 && c.head_dim != 128) return "head_dim must be 64 or 128";
+  if (rep > mk::kMaxRep) return "at most 8 q heads per kv head";
+  if (c.hidden % 256 || c.ffn % 256 || qd % 256)
+    return "hidden, ffn and n_q_heads*head_dim must be multiples of 256";
+  if (std::max(std::max(c.hidden, c.ffn), qd) > mk::kMaxChunks * 8 * mk::kComputeThreads)
+    return "projection input width above 16384";
+  if (c.batch > 1)
+    return "batch > 1 needs the tensor-core projection path, which this build does not have";
+  if (c.batch > mk::kMaxBatch) return "batch above 16";
+  return "";
+}
+
+mk::ModelShape shape_of(const mk_model_config &c) {
+  return mk::ModelShape{c.n_layers, c.hidden, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                        c.ffn,      c.vocab,  c.batch,     c.kv_capacity};
+}
+
+mk_status plan(const mk_model_config *cfg, const mk_tuning &t, int workers, mk_handle *h) {
+  mk::GraphTuning gt;
+  gt.num_workers = workers;
+  gt.col_align = t.col_align;
+  gt.attn_tasks_per_worker = t.attn_tasks_per_worker;
+  gt.attn_min_chunk = t.attn_min_chunk;
+  int st = 0;
+  std::string e = mk::plan_decode_graph(shape_of(*cfg), gt, &h->graph, &st);
+  if (!e.empty()) return fail(h, st == -4 ? MK_ERR_GRAPH : MK_ERR_ARG, e);
+  return MK_OK;
+}
+
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int num_workers,
+                        mk_handle **out) {
+  if (!cfg || !out) return fail(nullptr, MK_ERR_ARG, "null argument");
+  *out = nullptr;
+  std::string e = check_shape(*cfg);
+  if (!e.empty()) return fail(nullptr, MK_ERR_ARG, e);
+  if (num_workers < 1) return fail(nullptr, MK_ERR_ARG, "num_workers must be >= 1");
+  mk_handle *h = new (std::nothrow) mk_handle();
+  if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
+  h->cfg = *cfg;
+  h->tune = fill_defaults(tuning);
+  h->tune.num_workers = num_workers;
+  mk_status s = plan(cfg, h->tune, num_workers, h);
+  if (s != MK_OK) {
+    g_last_error = h->err;
+    delete h;
+    return s;
+  }
+  *out = h;
+  return MK_OK;
+}
+
+mk_status mk_graph_from_edges(int n_tasks, const int32_t *task_op, const int32_t *task_idx,
+                              int n_edges, const int32_t *edge_src, const int32_t *edge_dst,
+                              mk_handle **out) {
+  if (!out || n_tasks < 0 || n_edges < 0 || (n_tasks && (!task_op || !task_idx)) ||
+      (n_edges && (!edge_src || !edge_dst)))
+    return fail(nullptr, MK_ERR_ARG, "bad argument");
+  *out = nullptr;
+  mk_handle *h = new (std::nothrow) mk_handle();
+  if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
+  int st = 0;
+  std::string e =
+      mk::plan_generic_graph(n_tasks, task_op, task_idx, n_edges, edge_src, edge_dst, &h->graph,
+                             &st);
+  if (!e.empty()) {
+    delete h;
+    return fail(nullptr, st == -4 ? MK_ERR_GRAPH : MK_ERR_ARG, e);
+  }
+  *out = h;
+  return MK_OK;
+}
+
+mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, int device,
+                         mk_handle **out) {
+  if (!cfg || !out) return fail(nullptr, MK_ERR_ARG, "null argument");
+  *out = nullptr;
+  std::string e = check_gpu_shape(*cfg);
+  if (!e.empty()) return fail(nullptr, MK_ERR_ARG, e);
+  cudaError_t ce = cudaSetDevice(device);
+  if (ce != cudaSuccess) return cuda_fail(nullptr, ce, "cudaSetDevice");
+  int sms = 0, coop = 0, smem_optin = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
+  cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (!coop) return fail(nullptr, MK_ERR_CUDA, "device does not support cooperative launch");
+
+  mk_handle *h = new (std::nothrow) mk_handle();
+  if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
+  h->host_only = false;
+  h->device = device;
+  h->cfg = *cfg;
+  h->tune = fill_defaults(tuning);
+  mk_tuning &t = h->tune;
+  const mk_model_config &c = *cfg;
+  const int D = c.head_dim;
+  if (t.ring_stage_bytes % 1024) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "ring_stage_bytes must be a multiple of 1024");
+  }
+  // shared memory: shrink the stage size until the CTA fits
+  size_t smem = 0;
+  for (;;) {
+    const int pps = t.ring_stage_bytes / (4 * D);
+    smem = mk::worker_smem_bytes(t.ring_stages, t.ring_stage_bytes, pps, D);
+    if ((int)smem <= smem_optin) break;
+    t.ring_stage_bytes -= 1024;
+    if (t.ring_stage_bytes < 2 * std::max(std::max(c.hidden, c.ffn), c.n_q_heads * D)) {
+      delete h;
+      return fail(nullptr, MK_ERR_ARG, "ring does not fit in shared memory");
+    }
+  }
+  h->smem = smem;
+  ce = mk::worker_configure(smem);
+  if (ce != cudaSuccess) {
+    mk_status s = cuda_fail(nullptr, ce, "cudaFuncSetAttribute");
+    delete h;
+    return s;
+  }
+  int per_sm = 0;
+  mk::worker_max_blocks(&per_sm, smem);
+  if (per_sm < 1) {
+    delete h;
+    return fail(nullptr, MK_ERR_CUDA, "worker kernel cannot be resident");
+  }
+  const int W = t.num_workers > 0 ? t.num_workers : sms;
+  if (W > sms * per_sm) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "more workers than co-resident CTAs");
+  }
+  t.num_workers = W;
+  mk_status s = plan(cfg, t, W, h);
+  if (s != MK_OK) {
+    g_last_error = h->err;
+    delete h;
+    return s;
+  }
+  const mk::TaskGraph &G = h->graph;
+  const mk::Tiling &T = G.tiling;
+
+  // sizes
+  const int B = c.batch, H = c.hidden, F = c.ffn, Ly = c.n_layers, V = c.vocab;
+  const int rep = c.n_q_heads / c.n_kv_heads, grp = (rep + 2) * D, n_qkv = c.n_kv_heads * grp;
+  const int qd = c.n_q_heads * D, S = T.attn_splits;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = up256(off + bytes);
+    return o;
+  };
+  const size_t o_tasks = take(sizeof(mk::DevTask) * G.type.size());
+  const size_t o_events = take(sizeof(mk::DevEvent) * std::max<size_t>(1, G.ev_count.size()));
+  const size_t o_counters = take(4 * std::max<size_t>(1, G.ev_count.size()));
+  const size_t o_epoch = take(4);
+  const size_t o_status = take(16);
+  const size_t o_layers = take(sizeof(mk::DevLayer) * Ly);
+  const size_t o_optasks = take(4 * G.type.size());
+  const size_t o_rope = take(4 * (size_t)c.kv_capacity * D);
+  const size_t o_lmv = take(4 * (size_t)B * T.n_lm);
+  const size_t o_lmi = take(4 * (size_t)B * T.n_lm);
+  const size_t act0 = off;
+  const size_t o_x = take(4 * (size_t)(Ly + 1) * B * H);
+  std::vector<size_t> o_qkv(Ly), o_part(Ly), o_att(Ly), o_xm(Ly), o_h(Ly);
+  for (int l = 0; l < Ly; ++l) {
+    o_qkv[l] = take(4 * (size_t)B * n_qkv);
+    o_part[l] = S > 1 ? take(4 * (size_t)B * c.n_q_heads * S * (D + 2)) : 0;
+    o_att[l] = take(4 * (size_t)B * qd);
+    o_xm[l] = take(4 * (size_t)B * H);
+    o_h[l] = take(4 * (size_t)B * F);
+  }
+  h->act_bytes = (int64_t)(off - act0);
+  h->dev_block_bytes = off;
+  ce = cudaMalloc(&h->dev_block, off);
+  if (ce != cudaSuccess) {
+    delete h;
+    return fail(nullptr, MK_ERR_OOM, "cudaMalloc of graph and activation buffers failed");
+  }
+  char *base = static_cast<char *>(h->dev_block);
+  cudaMemset(base, 0, off);
+
+  // tables
+  std::vector<mk::DevTask> tasks(G.type.size());
+  for (size_t i = 0; i < tasks.size(); ++i) {
+    tasks[i].type = (uint8_t)G.type[i];
+    tasks[i].pad = 0;
+    tasks[i].layer = (uint16_t)(G.layer[i] < 0 ? 0xFFFF : G.layer[i]);
+    tasks[i].idx = (uint32_t)G.idx[i];
+    tasks[i].dep = G.dep[i];
+    tasks[i].trig = G.trig[i];
+  }
+  std::vector<mk::DevEvent> events(G.ev_count.size());
+  for (size_t e = 0; e < events.size(); ++e)
+    events[e] = mk::DevEvent{(uint32_t)G.ev_count[e], G.ev_first[e], G.ev_last[e], 0u};
+  std::vector<int32_t> op_list;
+  h->op_offset.assign(G.n_ops + 1, 0);
+  for (int o = 0; o < G.n_ops; ++o) {
+    h->op_offset[o] = (int32_t)op_list.size();
+    op_list.insert(op_list.end(), G.op_tasks[o].begin(), G.op_tasks[o].end());
+  }
+  h->op_offset[G.n_ops] = (int32_t)op_list.size();
+  std::vector<float> rope((size_t)c.kv_capacity * D);
+  for (int pos = 0; pos < c.kv_capacity; ++pos)
+    for (int i = 0; i < D / 2; ++i) {
+      const double inv_freq = std::pow(c.rope_theta, -(2.0 * i) / (double)D);
+      const double ang = (double)pos * inv_freq;
+      rope[(size_t)pos * D + 2 * i] = (float)std::cos(ang);
+      rope[(size_t)pos * D + 2 * i + 1] = (float)std::sin(ang);
+    }
+  h->layers.resize(Ly);
+  for (int l = 0; l < Ly; ++l) {
+    mk::DevLayer &L = h->layers[l];
+    std::memset(&L, 0, sizeof(L));
+    L.qkv = reinterpret_cast<float *>(base + o_qkv[l]);
+    L.part = S > 1 ? reinterpret_cast<float *>(base + o_part[l]) : nullptr;
+    L.att = reinterpret_cast<float *>(base + o_att[l]);
+    L.xm = reinterpret_cast<float *>(base + o_xm[l]);
+    L.h = reinterpret_cast<float *>(base + o_h[l]);
+    L.x_in = reinterpret_cast<float *>(base + o_x) + (size_t)l * B * H;
+    L.x_out = reinterpret_cast<float *>(base + o_x) + (size_t)(l + 1) * B * H;
+  }
+  ce = cudaMemcpy(base + o_tasks, tasks.data(), sizeof(mk::DevTask) * tasks.size(),
+                  cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess && !events.empty())
+    ce = cudaMemcpy(base + o_events, events.data(), sizeof(mk::DevEvent) * events.size(),
+                    cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(base + o_optasks, op_list.data(), 4 * op_list.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(base + o_rope, rope.data(), 4 * rope.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(base + o_layers, h->layers.data(), sizeof(mk::DevLayer) * Ly,
+                    cudaMemcpyHostToDevice);
+  if (ce != cudaSuccess) {
+    mk_status st = cuda_fail(nullptr, ce, "upload of graph tables");
+    mk_destroy(h);
+    return st;
+  }
+  h->d_layers = reinterpret_cast<mk::DevLayer *>(base + o_layers);
+  h->d_op_tasks = reinterpret_cast<int32_t *>(base + o_optasks);
+
+  Params &p = h->base;
+  std::memset(&p, 0, sizeof(p));
+  p.tasks = reinterpret_cast<const mk::DevTask *>(base + o_tasks);
+  p.events = reinterpret_cast<const mk::DevEvent *>(base + o_events);
+  p.counters = reinterpret_cast<uint32_t *>(base + o_counters);
+  p.epoch = reinterpret_cast<uint32_t *>(base + o_epoch);
+  p.status = reinterpret_cast<int32_t *>(base + o_status);
+  p.n_tasks = (int)tasks.size();
+  p.layers = h->d_layers;
+  p.x0 = reinterpret_cast<float *>(base + o_x);
+  p.x_final = reinterpret_cast<float *>(base + o_x) + (size_t)Ly * B * H;
+  p.lm_val = reinterpret_cast<float *>(base + o_lmv);
+  p.lm_idx = reinterpret_cast<int32_t *>(base + o_lmi);
+  p.rope = reinterpret_cast<const float *>(base + o_rope);
+  p.B = B; p.H = H; p.Hq = c.n_q_heads; p.Hkv = c.n_kv_heads; p.D = D; p.F = F; p.V = V;
+  p.Ly = Ly; p.Lcap = c.kv_capacity; p.rep = rep; p.grp = grp; p.n_qkv = n_qkv; p.qdim = qd;
+  p.eps = c.rms_eps;
+  p.attn_scale = (float)(1.0 / std::sqrt((double)D));
+  p.qkv_rows = T.qkv_rows; p.o_rows = T.o_rows; p.gu_rows = T.gu_rows;
+  p.down_rows = T.down_rows; p.lm_rows = T.lm_rows; p.S = S; p.chunk = T.attn_chunk;
+  p.n_lm = T.n_lm;
+  auto rps = [&](int K) { return std::max(1, std::min(mk::kMaxRowsPerStage, t.ring_stage_bytes / (2 * K))); };
+  p.rps_qkv = rps(H);
+  p.rps_o = rps(qd);
+  p.rps_gu = std::max(2, rps(H) & ~1);
+  p.rps_down = rps(F);
+  p.rps_lm = rps(H);
+  p.pps = t.ring_stage_bytes / (4 * D);
+  p.ring_stages = t.ring_stages;
+  p.stage_bytes = t.ring_stage_bytes;
+  p.l2_prefetch_bytes = t.l2_prefetch_bytes;
+  p.timeout_ns = (unsigned long long)t.wait_timeout_us * 1000ull;
+  *out = h;
+  return MK_OK;
+}
+
+mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
+  if (!h) return fail(nullptr, MK_ERR_ARG, "null handle");
+  if (h->host_only) return fail(h, MK_ERR_ARG, "handle was made by mk_plan_graph");
+  if (!w || !w->embed || !w->final_norm || !w->attn_norm || !w->wq || !w->wk || !w->wv ||
+      !w->q_norm || !w->k_norm || !w->wo || !w->mlp_norm || !w->w_gate || !w->w_up ||
+      !w->w_down)
+    return fail(h, MK_ERR_ARG, "missing weight pointer");
+  const mk_model_config &c = h->cfg;
+  if ((w->lm_head == nullptr) != (c.tied_embeddings != 0))
+    return fail(h, MK_ERR_ARG, "lm_head must be NULL exactly when embeddings are tied");
+  cudaSetDevice(h->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = c.hidden, F = c.ffn, D = c.head_dim, Ly = c.n_layers, V = c.vocab;
+  const int rep = c.n_q_heads / c.n_kv_heads, grp = (rep + 2) * D;
+  const size_t n_qkv = (size_t)c.n_kv_heads * grp, qd = (size_t)c.n_q_heads * D;
+  // arena layout
+  size_t off = 0;
+  auto take = [&](size_t elems) {
+    size_t o = off;
+    off = up256(off + 2 * elems);
+    return o;
+  };
+  std::vector<size_t> o_qkv(Ly), o_o(Ly), o_gu(Ly), o_dn(Ly), o_an(Ly), o_qn(Ly), o_kn(Ly),
+      o_mn(Ly);
+  for (int l = 0; l < Ly; ++l) {
+    o_qkv[l] = take(n_qkv * H);
+    o_o[l] = take((size_t)H * qd);
+    o_gu[l] = take((size_t)2 * F * H);
+    o_dn[l] = take((size_t)H * F);
+  }
+  const size_t o_lm = c.tied_embeddings ? 0 : take((size_t)V * H);
+  const size_t o_emb = take((size_t)V * H);
+  for (int l = 0; l < Ly; ++l) {
+    o_an[l] = take(H);
+    o_qn[l] = take(D);
+    o_kn[l] = take(D);
+    o_mn[l] = take(H);
+  }
+  const size_t o_fn = take(H);
+  if (!h->arena || h->arena_bytes != off) {
+    if (h->arena) cudaFree(h->arena);
+    h->arena = nullptr;
+    if (cudaMalloc(&h->arena, off) != cudaSuccess) {
+      h->arena_bytes = 0;
+      return fail(h, MK_ERR_OOM, "cudaMalloc of the weight arena failed");
+    }
+    h->arena_bytes = off;
+  }
+  char *A = static_cast<char *>(h->arena);
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](size_t dst_off, const void *src, size_t bytes) {
+    if (e == cudaSuccess) e = cudaMemcpyAsync(A + dst_off, src, bytes, cudaMemcpyDefault, st);
+  };
+  const size_t row = 2 * (size_t)H;
+  for (int l = 0; l < Ly; ++l) {
+    for (int g = 0; g < c.n_kv_heads; ++g) {
+      const size_t dst = o_qkv[l] + (size_t)g * grp * row;
+      cp(dst, static_cast<const char *>(w->wq[l]) + (size_t)g * rep * D * row, (size_t)rep * D * row);
+      cp(dst + (size_t)rep * D * row, static_cast<const char *>(w->wk[l]) + (size_t)g * D * row,
+         (size_t)D * row);
+      cp(dst + (size_t)(rep + 1) * D * row,
+         static_cast<const char *>(w->wv[l]) + (size_t)g * D * row, (size_t)D * row);
+    }
+    cp(o_o[l], w->wo[l], (size_t)H * qd * 2);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(A + o_gu[l], 2 * row, w->w_gate[l], row, row, F, cudaMemcpyDefault, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(A + o_gu[l] + row, 2 * row, w->w_up[l], row, row, F, cudaMemcpyDefault,
+                            st);
+    cp(o_dn[l], w->w_down[l], (size_t)H * F * 2);
+    cp(o_an[l], w->attn_norm[l], (size_t)H * 2);
+    cp(o_qn[l], w->q_norm[l], (size_t)D * 2);
+    cp(o_kn[l], w->k_norm[l], (size_t)D * 2);
+    cp(o_mn[l], w->mlp_norm[l], (size_t)H * 2);
+  }
+  cp(o_emb, w->embed, (size_t)V * H * 2);
+  if (!c.tied_embeddings) cp(o_lm, w->lm_head, (size_t)V * H * 2);
+  cp(o_fn, w->final_norm, (size_t)H * 2);
+  if (e != cudaSuccess) return cuda_fail(h, e, "weight copy");
+  for (int l = 0; l < Ly; ++l) {
+    mk::DevLayer &L = h->layers[l];
+    L.w_qkv = reinterpret_cast<const uint16_t *>(A + o_qkv[l]);
+    L.w_o = reinterpret_cast<const uint16_t *>(A + o_o[l]);
+    L.w_gu = reinterpret_cast<const uint16_t *>(A + o_gu[l]);
+    L.w_down = reinterpret_cast<const uint16_t *>(A + o_dn[l]);
+    L.attn_norm = reinterpret_cast<const uint16_t *>(A + o_an[l]);
+    L.q_norm = reinterpret_cast<const uint16_t *>(A + o_qn[l]);
+    L.k_norm = reinterpret_cast<const uint16_t *>(A + o_kn[l]);
+    L.mlp_norm = reinterpret_cast<const uint16_t *>(A + o_mn[l]);
+  }
+  e = cudaMemcpyAsync(h->d_layers, h->layers.data(), sizeof(mk::DevLayer) * Ly,
+                      cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // the host array is reused
+  if (e != cudaSuccess) return cuda_fail(h, e, "layer table upload");
+  Params &p = h->base;
+  p.embed = reinterpret_cast<const uint16_t *>(A + o_emb);
+  p.lm_head = reinterpret_cast<const uint16_t *>(A + (c.tied_embeddings ? o_emb : o_lm));
+  p.final_norm = reinterpret_cast<const uint16_t *>(A + o_fn);
+  h->weight_bytes = 0;
+  for (int l = 0; l < Ly; ++l)
+    h->weight_bytes += 2 * ((int64_t)n_qkv * H + (int64_t)H * qd + 3LL * F * H + 2LL * H + 2LL * D);
+  h->weight_bytes += 2 * ((int64_t)(c.tied_embeddings ? 1 : 2) * V * H + H);
+  h->loaded = true;
+  return MK_OK;
+}
+
+static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int32_t *kvl,
+                           void *kc, void *vc, Params *p) {
+  if (!h) return fail(nullptr, MK_ERR_ARG, "null handle");
+  if (h->host_only) return fail(h, MK_ERR_ARG, "handle was made by mk_plan_graph");
+  if (!h->loaded) return fail(h, MK_ERR_NOT_LOADED, "mk_load_weights has not been called");
+  if (!tin || !tout || !kvl || !kc || !vc) return fail(h, MK_ERR_ARG, "null buffer");
+  *p = h->base;
+  p->tokens_in = tin;
+  p->tokens_out = tout;
+  p->kv_len = kvl;
+  p->k_cache = static_cast<uint16_t *>(kc);
+  p->v_cache = static_cast<uint16_t *>(vc);
+  return MK_OK;
+}
+
+mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
+                         int32_t *d_kv_len, void *d_k_cache, void *d_v_cache, float *d_logits,
+                         void *stream) {
+  Params p;
+  mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache, &p);
+  if (s != MK_OK) return s;
+  p.logits = d_logits;
+  p.persistent = 1;
+  cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
+  return MK_OK;
+}
+
+mk_status mk_decode_step_perop(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
+                               int32_t *d_kv_len, void *d_k_cache, void *d_v_cache,
+                               float *d_logits, void *stream) {
+  Params p;
+  mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache, &p);
+  if (s != MK_OK) return s;
+  p.logits = d_logits;
+  p.persistent = 0;
+  for (int o = 0; o + 1 < (int)h->op_offset.size(); ++o) {
+    const int n = h->op_offset[o + 1] - h->op_offset[o];
+    if (n == 0) continue;
+    p.task_list = h->d_op_tasks + h->op_offset[o];
+    cudaError_t e = mk::launch_tasks(p, n, h->smem, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(h, e, "per-operator launch");
+  }
+  return MK_OK;
+}
+
+mk_status mk_sync_status(mk_handle *h, void *stream, int32_t *detail) {
+  if (!h || h->host_only) return fail(h, MK_ERR_ARG, "no device state");
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+  int32_t st[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(st, h->base.status, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "status read");
+  if (detail) std::memcpy(detail, st, sizeof(st));
+  if (st[0] == mk::kDevTimeout) {
+    char buf[160];
+    std::snprintf(buf, sizeof(buf), "event wait timed out (task %d, event %d, block %d)", st[1],
+                  st[2], st[3]);
+    return fail(h, MK_ERR_TIMEOUT, buf);
+  }
+  if (st[0] != 0) {
+    char buf[160];
+    std::snprintf(buf, sizeof(buf), "device rejected the step inputs (sequence %d)", st[2]);
+    return fail(h, MK_ERR_DEVICE, buf);
+  }
+  return MK_OK;
+}
+
+mk_status mk_reset(mk_handle *h, void *stream) {
+  if (!h || h->host_only) return fail(h, MK_ERR_ARG, "no device state");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t ne = std::max<size_t>(1, h->graph.ev_count.size());
+  cudaError_t e = cudaMemsetAsync(h->base.counters, 0, 4 * ne, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->base.epoch, 0, 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->base.status, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "reset");
+  return MK_OK;
+}
+
+mk_status mk_graph_export(const mk_handle *h, mk_graph_view *out) {
+  if (!h || !out) return fail(nullptr, MK_ERR_ARG, "null argument");
+  const mk::TaskGraph &G = h->graph;
+  std::memset(out, 0, sizeof(*out));
+  out->n_tasks = (int32_t)G.type.size();
+  out->n_events = (int32_t)G.ev_count.size();
+  out->n_edges = (int32_t)G.edge_src.size();
+  out->num_workers = G.num_workers;
+  out->task_type = G.type.data();
+  out->task_op = G.op.data();
+  out->task_layer = G.layer.data();
+  out->task_idx = G.idx.data();
+  out->task_dep = G.dep.data();
+  out->task_trig = G.trig.data();
+  out->event_count = G.ev_count.data();
+  out->event_first = G.ev_first.data();
+  out->event_last = G.ev_last.data();
+  out->edge_src = G.edge_src.data();
+  out->edge_dst = G.edge_dst.data();
+  const mk::Tiling &T = G.tiling;
+  out->qkv_rows = T.qkv_rows;
+  out->o_rows = T.o_rows;
+  out->gu_rows = T.gu_rows;
+  out->down_rows = T.down_rows;
+  out->lm_rows = T.lm_rows;
+  out->attn_splits = T.attn_splits;
+  out->attn_chunk = T.attn_chunk;
+  return MK_OK;
+}
+
+mk_status mk_get_info(const mk_handle *h, mk_info *out) {
+  if (!h || !out) return fail(nullptr, MK_ERR_ARG, "null argument");
+  std::memset(out, 0, sizeof(*out));
+  out->device = h->device;
+  out->num_workers = h->tune.num_workers;
+  out->n_tasks = (int32_t)h->graph.type.size();
+  out->n_events = (int32_t)h->graph.ev_count.size();
+  out->n_ops = h->graph.n_ops;
+  out->smem_bytes = (int32_t)h->smem;
+  out->ring_stages = h->tune.ring_stages;
+  out->ring_stage_bytes = h->tune.ring_stage_bytes;
+  out->weight_bytes = h->weight_bytes;
+  out->act_bytes = h->act_bytes;
+  return MK_OK;
+}
+
+mk_status mk_final_hidden(const mk_handle *h, const float **d_ptr) {
+  if (!h || !d_ptr || h->host_only) return fail(nullptr, MK_ERR_ARG, "no device state");
+  *d_ptr = h->base.x_final;
+  return MK_OK;
+}
+
+mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *stream) {
+  if (!h || h->host_only) return fail(h, MK_ERR_ARG, "no device state");
+  if (event < 0 || event >= (int)h->graph.ev_count.size() || count < 0)
+    return fail(h, MK_ERR_ARG, "event out of range");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  uint32_t v = (uint32_t)count;
+  if (e == cudaSuccess)
+    e = cudaMemcpy((char *)h->base.events + sizeof(mk::DevEvent) * event, &v, 4,
+                   cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(h, e, "event table write");
+  return MK_OK;
+}
+
+mk_status mk_set_timeout_us(mk_handle *h, unsigned timeout_us) {
+  if (!h || timeout_us == 0) return fail(h, MK_ERR_ARG, "bad argument");
+  h->tune.wait_timeout_us = timeout_us;
+  h->base.timeout_ns = (unsigned long long)timeout_us * 1000ull;
+  return MK_OK;
+}
+
+const char *mk_last_error(const mk_handle *h) {
+  return h ? h->err.c_str() : g_last_error.c_str();
+}
+
+void mk_destroy(mk_handle *h) {
+  if (!h) return;
+  if (!h->host_only && h->device >= 0) {
+    cudaSetDevice(h->device);
+    if (h->dev_block) cudaFree(h->dev_block);
+    if (h->arena) cudaFree(h->arena);
+  }
+  delete h;
+}
+
+}  // extern "C"

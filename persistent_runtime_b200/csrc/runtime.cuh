@@ -1,0 +1,90 @@
+// Structures shared by the host API and the device runtime of the decode-step
+// megakernel.  Plain data only, so the host side can include this file
+// without nvcc.
+#pragma once
+
+#include <cstdint>
+
+namespace mk {
+
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = kComputeWarps * 32;  // threads that run task bodies
+constexpr int kThreads = kComputeThreads + 32;       // + one producer (TMA) warp
+constexpr int kMaxChunks = 8;          // 16-byte weight chunks per thread and row: K <= 16384
+constexpr int kMaxRowsPerStage = 64;   // GEMV rows in one ring stage
+constexpr int kMaxRep = 8;             // q heads per kv head
+constexpr int kMaxHeadDim = 128;
+constexpr int kMaxBatch = 16;
+
+// Device status words: [0] status code, [1] task, [2] event, [3] block.
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = -6, kDevBadInput = -7 };
+
+struct DevTask {  // 16 bytes
+  uint8_t type;
+  uint8_t pad;
+  uint16_t layer;  // 0xFFFF for EMBED / LM_HEAD / ARGMAX
+  uint32_t idx;    // index of the task within its operator
+  int32_t dep;     // event this task waits for, -1 = none
+  int32_t trig;    // event this task triggers, -1 = none
+};
+
+struct DevEvent {  // 16 bytes
+  uint32_t count;  // triggers needed per step
+  int32_t first, last;
+  uint32_t pad;
+};
+
+// Per-layer device pointers: weight arena slices and activation buffers.
+struct DevLayer {
+  const uint16_t *w_qkv;   // [n_kv_heads * (rep + 2) * D][H], group-major rows
+  const uint16_t *w_o;     // [H][Hq * D]
+  const uint16_t *w_gu;    // [2F][H], row 2i = gate_i, row 2i+1 = up_i
+  const uint16_t *w_down;  // [H][F]
+  const uint16_t *attn_norm, *q_norm, *k_norm, *mlp_norm;
+  float *qkv;   // [B][n_kv_heads * (rep + 2) * D]
+  float *part;  // [B][Hq][S][D + 2]: unnormalised o, running max, running sum
+  float *att;   // [B][Hq * D]
+  float *xm;    // [B][H]  residual stream after attention
+  float *h;     // [B][F]  SiLU(gate) * up
+  float *x_in;  // [B][H]  residual stream entering the layer
+  float *x_out; // [B][H]  residual stream leaving the layer
+};
+
+struct Params {
+  // graph
+  const DevTask *tasks;
+  const DevEvent *events;
+  uint32_t *counters;  // one per event, monotone: count * epoch after each step
+  uint32_t *epoch;     // steps completed by the persistent kernel
+  int32_t *status;     // 4 words, see DeviceStatus
+  int n_tasks;
+  int persistent;       // 1: worker w runs tasks w, w + W, ...; 0: one task per CTA
+  const int32_t *task_list;  // per-operator mode: task ids, one per CTA
+  // model
+  const DevLayer *layers;
+  const uint16_t *embed, *lm_head, *final_norm;
+  float *x0, *x_final;     // residual stream before layer 0 / after the last layer
+  float *lm_val;           // [B][n_lm] partial argmax values
+  int32_t *lm_idx;         // [B][n_lm] partial argmax indices
+  const float *rope;       // [kv_capacity][D/2][2] cos, sin
+  // step arguments
+  const int32_t *tokens_in;
+  int32_t *tokens_out;
+  int32_t *kv_len;
+  uint16_t *k_cache, *v_cache;  // [Ly][B][Hkv][Lcap][D]
+  float *logits;                // [B][V] or null
+  // shapes
+  int B, H, Hq, Hkv, D, F, V, Ly, Lcap, rep, grp, n_qkv, qdim;
+  float eps;
+  float attn_scale;  // 1 / sqrt(D)
+  // tiling
+  int qkv_rows, o_rows, gu_rows, down_rows, lm_rows, S, chunk, n_lm;
+  int rps_qkv, rps_o, rps_gu, rps_down, rps_lm;  // GEMV rows per ring stage
+  int pps;                                       // KV positions per ring stage
+  // ring
+  int ring_stages, stage_bytes;
+  int l2_prefetch_bytes;
+  unsigned long long timeout_ns;
+};
+
+}  // namespace mk

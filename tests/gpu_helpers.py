@@ -1,0 +1,111 @@
+"""Shared set-up for the GPU parity tests: seeded inputs, oracle run, comparison."""
+import numpy as np
+
+import oracle
+import synth
+
+# Tolerances of the bf16 decode step against the fp32 oracle.
+LOGIT_TOL = 2e-2      # max |d logit| <= LOGIT_TOL * max |logit|
+HIDDEN_TOL = 1e-2     # ||d hidden|| / ||hidden|| <= HIDDEN_TOL
+SEPARATION = 4e-2     # argmax must match exactly when top1 - top2 > SEPARATION * max|logit|
+
+
+def torch():
+    import torch as t
+    return t
+
+
+def dev_u16(a: np.ndarray):
+    """bf16 bit patterns on the GPU (int16 storage; only the bits matter)."""
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def dev_weights(weights: dict) -> dict:
+    out = {"embed": dev_u16(weights["embed"]), "final_norm": dev_u16(weights["final_norm"]),
+           "lm_head": None if weights["lm_head"] is None else dev_u16(weights["lm_head"]),
+           "layers": [{k: dev_u16(v) for k, v in lw.items()} for lw in weights["layers"]]}
+    return out
+
+
+class Case:
+    """One seeded workload instance: host inputs, oracle model, GPU handle."""
+
+    def __init__(self, w, seed=0, extra_cap=None, **tuning):
+        import persistent_runtime_b200 as prb
+        t = torch()
+        self.w = w
+        self.seed = seed
+        self.weights = synth.make_weights(w, seed)
+        self.lens = w.kv_lens(seed)
+        self.cap = int(self.lens.max()) + (w.steps if extra_cap is None else extra_cap)
+        self.k, self.v = synth.make_kv(w, self.lens, self.cap, seed)
+        self.tokens = synth.make_tokens(w, seed)
+        self.model = oracle.Model(w, self.weights, self.cap)
+        self.mk = prb.Megakernel(w, self.cap, 0, **tuning)
+        dw = dev_weights(self.weights)
+        self.mk.load_weights(dw)
+        t.cuda.synchronize()
+        del dw
+        self.reset_device_state()
+
+    def reset_device_state(self):
+        t = torch()
+        self.d_k = dev_u16(self.k)
+        self.d_v = dev_u16(self.v)
+        self.d_len = t.from_numpy(self.lens.copy()).cuda()
+        self.d_tok = t.from_numpy(self.tokens.copy()).cuda()
+        self.d_out = t.zeros(self.w.batch, dtype=t.int32, device="cuda")
+        self.d_logits = t.zeros((self.w.batch, self.w.vocab), dtype=t.float32, device="cuda")
+
+    def gpu_step(self, perop=False, tokens=None):
+        t = torch()
+        if tokens is not None:
+            self.d_tok.copy_(t.from_numpy(np.asarray(tokens, dtype=np.int32)))
+        fn = self.mk.decode_step_perop if perop else self.mk.decode_step
+        fn(self.d_tok, self.d_out, self.d_len, self.d_k, self.d_v, self.d_logits)
+        rc, detail = self.mk.sync_status()
+        assert rc == 0, (rc, detail)
+        n = self.w.batch * self.w.hidden
+        hidden = _wrap_device_f32(self.mk.final_hidden_ptr(), n).view(self.w.batch, -1).clone()
+        return {"tokens": self.d_out.cpu().numpy(), "logits": self.d_logits.cpu().numpy(),
+                "hidden": hidden.cpu().numpy(), "kv_len": self.d_len.cpu().numpy()}
+
+    def oracle_step(self, tokens=None, k=None, v=None, lens=None):
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        lens = self.lens if lens is None else lens
+        tok = self.tokens if tokens is None else tokens
+        return self.model.step(tok, lens, k, v)
+
+
+def _wrap_device_f32(ptr: int, n: int):
+    """A torch tensor viewing n fp32 values at a device address owned by the library."""
+    t = torch()
+
+    class _Holder:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False),
+                                    "version": 3, "strides": None}
+
+    return t.as_tensor(_Holder(), device="cuda")
+
+
+def compare_step(ref, got, w, ctx=""):
+    """Asserts the tolerances; returns a dict of the measured errors."""
+    out = {}
+    for b in range(w.batch):
+        lo, lg = ref["logits"][b].astype(np.float64), got["logits"][b].astype(np.float64)
+        scale = np.max(np.abs(lo))
+        err = np.max(np.abs(lo - lg))
+        assert err <= LOGIT_TOL * scale, f"{ctx} b={b}: max|dlogit| {err} > {LOGIT_TOL}*{scale}"
+        h0, h1 = ref["hidden"][b].astype(np.float64), got["hidden"][b].astype(np.float64)
+        rel = np.linalg.norm(h0 - h1) / np.linalg.norm(h0)
+        assert rel <= HIDDEN_TOL, f"{ctx} b={b}: hidden rel L2 {rel}"
+        top = np.sort(lo)[-2:]
+        tok = int(got["tokens"][b])
+        if top[1] - top[0] > SEPARATION * scale:
+            assert tok == int(ref["tokens"][b]), f"{ctx} b={b}: token {tok} != {ref['tokens'][b]}"
+        else:
+            assert lo[tok] >= top[1] - LOGIT_TOL * scale, f"{ctx} b={b}: token {tok} not near max"
+        out[b] = (float(err / scale), float(rel))
+    return out

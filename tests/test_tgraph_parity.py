@@ -1,0 +1,67 @@
+"""The library's host graph builder against the oracle's independent builder:
+bit-exact tables on every workload, hand-derived goldens and random graphs."""
+import numpy as np
+import pytest
+
+import graph_checks as gc
+import oracle
+import persistent_runtime_b200 as prb
+import synth
+
+pytestmark = pytest.mark.usefixtures("built_libs")
+
+CONFIGS = [(synth.TINY, 148), (synth.TINY, 1), (synth.TINY, 2), (synth.TINY, 7),
+           (synth.Q06B, 148), (synth.Q06B, 132), (synth.Q8B, 148), (synth.Q8B, 3),
+           (synth.Q8B_B8, 148), (synth.Q8B_B16, 148)]
+
+
+@pytest.mark.parametrize("w,W", CONFIGS, ids=[f"{w.name}-W{W}" for w, W in CONFIGS])
+def test_decode_graph_bit_exact_with_oracle(w, W):
+    cap = w.kv_capacity(0)
+    mine = prb.plan_graph(w, cap, W)
+    ref = oracle.tgraph_decode(w, cap, W)
+    gc.assert_graphs_equal(mine, ref)
+    np.testing.assert_array_equal(mine.edge_src, ref.edge_src)
+    np.testing.assert_array_equal(mine.edge_dst, ref.edge_dst)
+    assert mine.tiling == (ref.qkv_rows, ref.o_rows, ref.gu_rows, ref.down_rows, ref.lm_rows,
+                           ref.splits, ref.chunk)
+    gc.check_invariants(mine)
+
+
+@pytest.mark.parametrize("col_align,apw,min_chunk", [(8, 4, 64), (4, 2, 128), (32, 8, 64)])
+def test_tuning_variants_bit_exact(col_align, apw, min_chunk):
+    w = synth.Q8B_B8
+    cap = w.kv_capacity(3)
+    mine = prb.plan_graph(w, cap, 148, col_align=col_align, attn_tasks_per_worker=apw,
+                          attn_min_chunk=min_chunk)
+    ref = oracle.tgraph_decode(w, cap, 148, col_align, apw, min_chunk)
+    gc.assert_graphs_equal(mine, ref)
+
+
+@pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt"])
+def test_decode_goldens(name):
+    cfg, _, _, tasks, events = gc.load_golden(name)
+    w = synth.Workload("golden", cfg["layers"], cfg["hidden"], cfg["q_heads"], cfg["kv_heads"],
+                       cfg["head_dim"], cfg["ffn"], cfg["vocab"], 0, cfg["batch"], 1)
+    g = prb.plan_graph(w, cfg["kv_capacity"], cfg["workers"], col_align=cfg["col_align"],
+                       attn_tasks_per_worker=cfg["apw"], attn_min_chunk=cfg["min_chunk"])
+    gc.assert_tables_equal(g, tasks, events)
+
+
+@pytest.mark.parametrize("name", ["tgraph_norm_dep.txt", "tgraph_norm_trig.txt"])
+def test_normalisation_goldens(name):
+    _, nodes, edges, tasks, events = gc.load_golden(name)
+    index = {n[0]: i for i, n in enumerate(nodes)}
+    g = prb.graph_from_edges([n[1] for n in nodes], [n[2] for n in nodes],
+                             [(index[a], index[b]) for a, b in edges])
+    gc.assert_tables_equal(g, tasks, events)
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_random_dags_bit_exact(seed):
+    op, idx, edges = gc.random_dag(seed, n_ops=(3, 10), per_op=(1, 7))
+    mine = prb.graph_from_edges(op, idx, edges)
+    ref = oracle.tgraph_from_edges(op, idx, edges)
+    gc.assert_graphs_equal(mine, ref)
+    gc.check_invariants(mine)
+    gc.simulate_random(mine, seed)
