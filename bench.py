@@ -1,0 +1,438 @@
+"""Decode-step benchmark: one persistent launch per step vs one launch per operator.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mk|reference]
+
+Prints ONE JSON line (rank 0).  The workload defaults to the Qwen3-8B-shaped
+decoder at batch 1 with 1024 cached positions per sequence; all inputs are
+seeded synthetic data (bf16 weights ~N(0, 0.02), gains 1 + N(0, 0.1), cached
+K/V ~N(0, 1)).  `value` is microseconds per decode step (device time, CUDA
+events, max over ranks); per step the whole weight set (15.3 GB) streams from
+HBM, far more than the 126 MB L2, so no explicit L2 flush is needed.
+
+Multi-GPU: the decode step does not shard without a per-layer exchange, so N
+GPUs run N independent replicas (no data-path collective); a barrier brackets
+the timed region and the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "us per decode step & achieved HBM GB/s vs 8 TB/s (Qwen3-8B-shaped, bs=1)"
+UNIT = "us/step"
+HBM_NOMINAL_GBS = 8000.0
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic bytes
+# ----------------------------------------------------------------------------
+def step_bytes(w, lens) -> int:
+    """Bytes one decode step must move: every weight matrix and gain once, the B
+    embedding rows, L_b cached K and V rows per (layer, sequence, kv head) and
+    the appended K/V rows."""
+    H, F, D, Ly = w.hidden, w.ffn, w.head_dim, w.n_layers
+    rep = w.n_q_heads // w.n_kv_heads
+    n_qkv = w.n_kv_heads * (rep + 2) * D
+    per_layer = n_qkv * H + H * w.q_dim + 2 * F * H + H * F + 2 * H + 2 * D
+    weights = 2 * (Ly * per_layer + w.vocab * H + H)
+    emb = 2 * w.batch * H
+    kv_row = 2 * D * w.n_kv_heads * Ly * 2  # K and V, every layer and kv head
+    kv_read = kv_row * int(np.sum(lens))
+    kv_write = kv_row * w.batch
+    return int(weights + emb + kv_read + kv_write)
+
+
+def steps_bytes(w, lens0, k) -> int:
+    return sum(step_bytes(w, np.asarray(lens0) + i) for i in range(k))
+
+
+# ----------------------------------------------------------------------------
+# Clocks during the timed region (NVML reads only)
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: clocks stay unreported
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# Helpers
+# ----------------------------------------------------------------------------
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("mk_worker.cu", "runtime.cuh"):
+        with open(os.path.join(ROOT, "persistent_runtime_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record(workload: str):
+    """DRAM bytes per launch from a committed ncu summary of the same kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_hash") != kernel_hash():
+        return None
+    return ent
+
+
+def gen_inputs(w, seed, cap):
+    lens = w.kv_lens(seed)
+    tokens = synth.make_tokens(w, seed)
+    weights = synth.make_weights(w, seed)
+    k, v = synth.make_kv(w, lens, cap, seed)
+    return weights, lens, tokens, k, v
+
+
+def upload(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing
+# ----------------------------------------------------------------------------
+def oracle_time_step(w, weights, lens, tokens, k, v, cap, layers_run=-1, vocab_run=-1):
+    import oracle
+    oracle.build() if not os.path.exists(os.path.join(ROOT, "oracle", "libmk_oracle.so")) else None
+    m = oracle.Model(w, weights, cap)
+    kl = lens.copy()
+    t0 = time.perf_counter()
+    m.step(tokens, kl, k, v, want_logits=False, want_hidden=False, layers_run=layers_run,
+           vocab_run=vocab_run)
+    return time.perf_counter() - t0
+
+
+def sample_fraction(w, layers_run, vocab_run, lens):
+    """Share of a full step's bytes that a (layers_run, vocab_run) sample touches."""
+    full = step_bytes(w, lens)
+    D, H = w.head_dim, w.hidden
+    rep = w.n_q_heads // w.n_kv_heads
+    n_qkv = w.n_kv_heads * (rep + 2) * D
+    per_layer = 2 * (n_qkv * H + H * w.q_dim + 3 * w.ffn * H + 2 * H + 2 * D)
+    kv = 2 * D * w.n_kv_heads * 2 * int(np.sum(lens) + w.batch)
+    part = layers_run * (per_layer + kv) + 2 * vocab_run * H
+    return part / full
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    cap = w.kv_capacity(args.seed) + max(args.steps, args.warmup)
+    weights, lens, tokens, k, v = gen_inputs(w, args.seed, cap)
+    layers_run = max(1, w.n_layers // 18)
+    vocab_run = max(1, w.vocab // 18)
+    frac = sample_fraction(w, layers_run, vocab_run, lens)
+    for _ in range(args.warmup):
+        oracle_time_step(w, weights, lens, tokens, k, v, cap, layers_run, vocab_run)
+    times = [oracle_time_step(w, weights, lens, tokens, k, v, cap, layers_run, vocab_run)
+             for _ in range(args.steps)]
+    us = 1e6 * float(np.mean(times)) / frac
+    sample = (f"each step: {layers_run} of {w.n_layers} layers + {vocab_run} of {w.vocab} LM-head "
+              f"rows ({100 * frac:.1f}% of the step's bytes), time scaled by bytes")
+    out = {"impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1000,
+           "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic", "config": workload_config(w, lens, args.gpus),
+           "cpu_baseline": {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    return 0
+
+
+def workload_config(w, lens, n):
+    return {"workload": f"{w.name} bs{w.batch} kv{int(np.max(lens))}",
+            "model": f"{w.name}-shaped decoder, {w.n_layers} layers, hidden {w.hidden}, "
+                     f"{w.n_q_heads}/{w.n_kv_heads} heads x {w.head_dim}, ffn {w.ffn}, "
+                     f"vocab {w.vocab}, {'tied' if w.tied_embeddings else 'untied'} LM head",
+            "global_batch": w.batch * n, "seq_len": int(np.max(lens)),
+            "parallelism": "replicas" if n > 1 else "single GPU",
+            "l2": "inputs larger than L2: every step streams all weights (>100x L2)"}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the per-operator arms")
+    ap.add_argument("--tuning", default="", help="k=v,... passed to mk_tuning")
+    ap.add_argument("--trace", default="", help="write a Chrome trace of one step to this path")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import persistent_runtime_b200 as prb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+
+    w = synth.WORKLOADS[args.workload]
+    cap = int(w.kv_lens(args.seed).max()) + max(args.steps, args.warmup)
+    tuning = {}
+    for kv in filter(None, args.tuning.split(",")):
+        key, val = kv.split("=")
+        tuning[key] = int(val)
+
+    lens = w.kv_lens(args.seed)
+    tokens = synth.make_tokens(w, args.seed)
+    keep_host = rank == 0 and world == 1 and not args.no_cpu_baseline
+    weights = synth.make_weights(w, args.seed)
+    mk = prb.Megakernel(w, cap, dev, **tuning)
+    dw = {"embed": upload(torch, weights["embed"]), "final_norm": upload(torch, weights["final_norm"]),
+          "lm_head": None if weights["lm_head"] is None else upload(torch, weights["lm_head"]),
+          "layers": [{n: upload(torch, a) for n, a in lw.items()} for lw in weights["layers"]]}
+    mk.load_weights(dw)
+    torch.cuda.synchronize()
+    del dw
+    if not keep_host:
+        weights = None
+    torch.cuda.empty_cache()
+    k_host, v_host = synth.make_kv(w, lens, cap, args.seed)
+    d_k, d_v = upload(torch, k_host), upload(torch, v_host)
+    if not keep_host:
+        k_host = v_host = None
+    d_len = torch.from_numpy(lens.copy()).cuda()
+    d_tok = torch.from_numpy(tokens.copy()).cuda()
+    d_logits = None
+    stream = torch.cuda.current_stream()
+
+    def reset():
+        d_len.copy_(torch.from_numpy(lens))
+        d_tok.copy_(torch.from_numpy(tokens))
+
+    def check():
+        rc, detail = mk.sync_status()
+        if rc != 0:
+            raise RuntimeError(f"device status {rc} {detail}")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(fn, k):
+        reset()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        barrier()
+        check()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    step = lambda: mk.decode_step(d_tok, d_tok, d_len, d_k, d_v, d_logits)  # noqa: E731
+
+    # warm-up
+    reset()
+    for _ in range(args.warmup):
+        step()
+    check()
+
+    # timed region: persistent megakernel
+    with ClockSampler(dev) as clocks:
+        ms = timed(step, args.steps)
+    us_step = 1000.0 * ms / args.steps
+    bytes_k = steps_bytes(w, lens, args.steps)
+    gbs = bytes_k / (ms * 1e-3) / 1e9
+    tok_s = world * w.batch * args.steps / (ms * 1e-3)
+
+    # end to end through the public API with host buffers
+    h_tok = torch.from_numpy(tokens.copy()).pin_memory()
+    h_out = torch.empty_like(h_tok).pin_memory()
+
+    def e2e_step():
+        d_tok.copy_(h_tok, non_blocking=True)
+        mk.decode_step(d_tok, d_tok, d_len, d_k, d_v, d_logits)
+        h_out.copy_(d_tok, non_blocking=True)
+        stream.synchronize()
+        h_tok.copy_(h_out)
+
+    h_tok.copy_(torch.from_numpy(tokens))
+    e2e_ms = timed(e2e_step, args.steps)
+    e2e_us = 1000.0 * e2e_ms / args.steps
+
+    baselines = {}
+    n_ops = mk.info().n_ops
+    if not args.no_baselines:
+        perop = lambda: mk.decode_step_perop(d_tok, d_tok, d_len, d_k, d_v, d_logits)  # noqa
+        reset()
+        for _ in range(args.warmup):
+            perop()
+        check()
+        baselines["perop_eager_us"] = 1000.0 * timed(perop, args.steps) / args.steps
+        try:
+            g = torch.cuda.CUDAGraph()
+            reset()
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                perop()  # warm the side stream
+            torch.cuda.synchronize()
+            reset()
+            with torch.cuda.graph(g):
+                perop()
+            torch.cuda.synchronize()
+            for _ in range(args.warmup):
+                g.replay()
+            check()
+            baselines["perop_graph_us"] = 1000.0 * timed(g.replay, args.steps) / args.steps
+            del g
+        except Exception as e:  # capture refused: report why
+            baselines["perop_graph_error"] = str(e)[:200]
+        baselines["perop_launches_per_step"] = n_ops
+
+    trace_summary = None
+    if args.trace:
+        from persistent_runtime_b200 import trace as mktrace
+        g = mk.graph()
+        buf = torch.zeros(4 * g.n_tasks, dtype=torch.int64, device="cuda")
+        mk.set_trace(buf)
+        reset()
+        step()
+        check()
+        mk.set_trace(None)
+        tr = buf.cpu().numpy().view(np.uint64)
+        trace_summary = mktrace.summarize(tr, g)
+        mktrace.to_chrome(tr, g, args.trace)
+        trace_summary.pop("op_spans")
+
+    peak, peak_kind = measured_peaks()
+    traffic = traffic_record(args.workload)
+    result = {
+        "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us_step / 1000.0, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, lens, world),
+        "tokens_per_s": tok_s, "hbm_gbs": gbs, "frac_of_8tbs": gbs / HBM_NOMINAL_GBS,
+        "bytes_per_step": bytes_k / args.steps,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "mk_worker_kernel (persistent, one launch per step)",
+                     "traffic": None if traffic is None else traffic["dram_bytes_per_launch"]},
+        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": 4 * w.batch,
+                "d2h_bytes_per_step": 4 * w.batch},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "baselines": baselines,
+    }
+    if trace_summary is not None:
+        result["trace"] = trace_summary
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t = oracle_time_step(w, weights, lens, tokens, k_host, v_host, cap)
+        result["cpu_baseline"] = {"value": 1e6 * t, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                  "sample": "one full decode step of the same workload, "
+                                            "single-threaded fp32 oracle"}
+    mk.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -25,7 +25,7 @@ TASK_NAMES = {0: "GENERIC", 1: "EMBED", 2: "QKV", 3: "ATTN", 4: "MERGE", 5: "OPR
 EXPORTS = ("mk_plan_graph", "mk_graph_from_edges", "mk_build_graph", "mk_load_weights",
            "mk_decode_step", "mk_decode_step_perop", "mk_sync_status", "mk_reset",
            "mk_graph_export", "mk_get_info", "mk_final_hidden", "mk_debug_set_event_count",
-           "mk_set_timeout_us", "mk_last_error", "mk_destroy")
+           "mk_set_trace", "mk_set_timeout_us", "mk_last_error", "mk_destroy")
 
 
 class MkError(RuntimeError):
@@ -107,6 +107,7 @@ def lib():
         "mk_get_info": ([vp, ctypes.POINTER(Info)], st),
         "mk_final_hidden": ([vp, ctypes.POINTER(vp)], st),
         "mk_debug_set_event_count": ([vp, i32, i32, vp], st),
+        "mk_set_trace": ([vp, vp, ctypes.c_int64], st),
         "mk_set_timeout_us": ([vp, ctypes.c_uint], st),
         "mk_last_error": ([vp], ctypes.c_char_p),
         "mk_destroy": ([vp], None),
@@ -301,6 +302,14 @@ class Megakernel:
     def set_event_count(self, event: int, count: int, stream=None):
         _check(lib().mk_debug_set_event_count(self._h, event, count, _stream_ptr(stream)),
                self._h)
+
+    def set_trace(self, buf=None):
+        """buf: int64/uint64 torch tensor with >= 4 * n_tasks elements, or None."""
+        if buf is None:
+            _check(lib().mk_set_trace(self._h, None, 0), self._h)
+        else:
+            _check(lib().mk_set_trace(self._h, buf.data_ptr(), buf.numel() * buf.element_size()),
+                   self._h)
 
     def set_timeout_us(self, us: int):
         _check(lib().mk_set_timeout_us(self._h, us), self._h)

@@ -15,7 +15,7 @@
 #include "tgraph.hpp"
 
 namespace mk {
-size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim);
+size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int rep_p);
 cudaError_t worker_configure(size_t smem);
 cudaError_t worker_max_blocks(int *blocks, size_t smem);
 cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream);
@@ -195,11 +195,13 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     delete h;
     return fail(nullptr, MK_ERR_ARG, "ring_stage_bytes must be a multiple of 1024");
   }
+  const int rep0 = c.n_q_heads / c.n_kv_heads;
+  const int rep_p = rep0 <= 1 ? 1 : rep0 <= 2 ? 2 : rep0 <= 4 ? 4 : 8;
   // shared memory: shrink the stage size until the CTA fits
   size_t smem = 0;
   for (;;) {
     const int pps = t.ring_stage_bytes / (4 * D);
-    smem = mk::worker_smem_bytes(t.ring_stages, t.ring_stage_bytes, pps, D);
+    smem = mk::worker_smem_bytes(t.ring_stages, t.ring_stage_bytes, pps, D, rep_p);
     if ((int)smem <= smem_optin) break;
     t.ring_stage_bytes -= 1024;
     if (t.ring_stage_bytes < 2 * std::max(std::max(c.hidden, c.ffn), c.n_q_heads * D)) {
@@ -351,12 +353,20 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.rope = reinterpret_cast<const float *>(base + o_rope);
   p.B = B; p.H = H; p.Hq = c.n_q_heads; p.Hkv = c.n_kv_heads; p.D = D; p.F = F; p.V = V;
   p.Ly = Ly; p.Lcap = c.kv_capacity; p.rep = rep; p.grp = grp; p.n_qkv = n_qkv; p.qdim = qd;
+  p.rep_p = rep_p;
   p.eps = c.rms_eps;
   p.attn_scale = (float)(1.0 / std::sqrt((double)D));
   p.qkv_rows = T.qkv_rows; p.o_rows = T.o_rows; p.gu_rows = T.gu_rows;
   p.down_rows = T.down_rows; p.lm_rows = T.lm_rows; p.S = S; p.chunk = T.attn_chunk;
   p.n_lm = T.n_lm;
-  auto rps = [&](int K) { return std::max(1, std::min(mk::kMaxRowsPerStage, t.ring_stage_bytes / (2 * K))); };
+  // GEMV rows per ring stage: a multiple of 8 when at least 8 rows fit,
+  // else 6, 4, 2 or 1 (the kernel batches rows 8 or fewer at a time)
+  auto rps = [&](int K) {
+    const int raw = std::min(mk::kMaxRowsPerStage, t.ring_stage_bytes / (2 * K));
+    if (raw >= 8) return raw / 8 * 8;
+    for (int r : {6, 4, 2}) if (raw >= r) return r;
+    return 1;
+  };
   p.rps_qkv = rps(H);
   p.rps_o = rps(qd);
   p.rps_gu = std::max(2, rps(H) & ~1);
@@ -367,6 +377,12 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.stage_bytes = t.ring_stage_bytes;
   p.l2_prefetch_bytes = t.l2_prefetch_bytes;
   p.timeout_ns = (unsigned long long)t.wait_timeout_us * 1000ull;
+  p.trace = nullptr;
+  if (S > 1 && 2 * rep * S > mk::kComputeWarps * rep_p * (D + 2)) {
+    mk_destroy(h);
+    return fail(nullptr, MK_ERR_ARG, "too many attention splits for the merge scratch; "
+                                     "raise attn_min_chunk");
+  }
   *out = h;
   return MK_OK;
 }
@@ -620,6 +636,14 @@ mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *str
     e = cudaMemcpy((char *)h->base.events + sizeof(mk::DevEvent) * event, &v, 4,
                    cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(h, e, "event table write");
+  return MK_OK;
+}
+
+mk_status mk_set_trace(mk_handle *h, void *d_buf, int64_t bytes) {
+  if (!h || h->host_only) return fail(h, MK_ERR_ARG, "no device state");
+  if (d_buf && bytes < (int64_t)32 * (int64_t)h->graph.type.size())
+    return fail(h, MK_ERR_ARG, "trace buffer smaller than 32 bytes per task");
+  h->base.trace = static_cast<unsigned long long *>(d_buf);
   return MK_OK;
 }
 

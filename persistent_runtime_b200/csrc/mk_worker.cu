@@ -130,6 +130,63 @@ __device__ __forceinline__ float dot8(const uint4 w, const float *x) {
   return a;
 }
 
+// (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32x2 FMA (sm_100).
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float w0, float w1, float x0,
+                                      float x1) {
+  asm("{\n\t.reg .b64 A, W, X;\n\t"
+      "mov.b64 A, {%0, %1};\n\t"
+      "mov.b64 W, {%2, %3};\n\t"
+      "mov.b64 X, {%4, %5};\n\t"
+      "fma.rn.f32x2 A, W, X, A;\n\t"
+      "mov.b64 {%0, %1}, A;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
+// acc (even, odd element partial sums) += w (8 bf16) . x (8 fp32)
+__device__ __forceinline__ void dot8_acc(const uint4 w, const float *x, float (&acc)[2]) {
+  ffma2(acc[0], acc[1], bf_lo(w.x), bf_hi(w.x), x[0], x[1]);
+  ffma2(acc[0], acc[1], bf_lo(w.y), bf_hi(w.y), x[2], x[3]);
+  ffma2(acc[0], acc[1], bf_lo(w.z), bf_hi(w.z), x[4], x[5]);
+  ffma2(acc[0], acc[1], bf_lo(w.w), bf_hi(w.w), x[6], x[7]);
+}
+
+// One step of a transposed warp reduction: lanes that differ in bit OFF swap
+// halves of their value arrays, so each lane keeps HALF partial sums.  After
+// the steps for every lane bit, each lane holds the full warp sum of one of
+// the original values (which one follows from its lane bits).
+template <int HALF, int OFF>
+__device__ __forceinline__ void transpose_step(float *v, int lane) {
+  const bool up = (lane & OFF) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float send = up ? v[i] : v[i + HALF];
+    const float keep = up ? v[i + HALF] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+  }
+}
+
+// Warp sums of 8 values with 9 shuffles; lane 4*i returns the sum of v[i].
+__device__ __forceinline__ float warp_sum8(float (&v)[8], int lane) {
+  transpose_step<4, 16>(v, lane);
+  transpose_step<2, 8>(v, lane);
+  transpose_step<1, 4>(v, lane);
+  float r = v[0];
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
+// Warp sums of 32 values with 31 shuffles; lane i returns the sum of v[i].
+__device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
+  transpose_step<16, 16>(v, lane);
+  transpose_step<8, 8>(v, lane);
+  transpose_step<4, 4>(v, lane);
+  transpose_step<2, 2>(v, lane);
+  transpose_step<1, 1>(v, lane);
+  return v[0];
+}
+
 // ---------------------------------------------------------------------------
 // Shared memory layout (identical computation on host: see smem_bytes()).
 // ---------------------------------------------------------------------------
@@ -140,16 +197,16 @@ struct Smem {
   uint64_t *full, *empty;
   volatile int *ctl;
   // GEMV scratch
-  float *red;   // [2][kMaxRowsPerStage][kComputeWarps]
+  float *red;   // [kRedRows][kComputeWarps] warp partial sums of tile rows
   float *ss;    // [kComputeWarps]
-  float *lmv;   // [kMaxRowsPerStage]
-  int *lmi;     // [kMaxRowsPerStage]
+  float *lmv;   // [kComputeThreads] partial argmax values (LM head)
+  int *lmi;     // [kComputeThreads] partial argmax indices
   // attention scratch
   float *q;     // [kMaxRep][kMaxHeadDim]
   uint16_t *knew, *vnew;  // [kMaxHeadDim] bf16
-  float *sc;    // [kMaxRep][pps]
-  float *mls;   // [3][kMaxRep]: running max, running sum, rescale
-  float *ored;  // [npg][kMaxRep][kMaxHeadDim]
+  float *sc;    // per warp: [32] probabilities, [kMaxRep] rescale factors
+  float *mls;   // [3][kMaxRep]
+  float *ored;  // per warp and head: [D] output, running max, running sum (merge: weights)
 };
 
 __host__ __device__ inline size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -159,7 +216,7 @@ struct SmemOffsets {
 };
 
 __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes, int pps,
-                                                    int head_dim) {
+                                                    int head_dim, int rep_p) {
   SmemOffsets o;
   size_t p = (size_t)stages * stage_bytes;
   o.full = p;
@@ -172,13 +229,13 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   // GEMV scratch
   size_t g = p;
   o.red = g;
-  g += 4 * 2 * kMaxRowsPerStage * kComputeWarps;
+  g += 4 * kRedRows * kComputeWarps;
   o.ss = g;
   g += 4 * kComputeWarps;
   o.lmv = g;
-  g += 4 * kMaxRowsPerStage;
+  g += 4 * kComputeThreads;
   o.lmi = g;
-  g += 4 * kMaxRowsPerStage;
+  g += 4 * kComputeThreads;
   // attention scratch (shares the same bytes: a CTA runs one task at a time)
   size_t a = p;
   o.q = a;
@@ -187,20 +244,19 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   a += 2 * kMaxHeadDim;
   o.vnew = a;
   a += 2 * kMaxHeadDim;
-  o.sc = a;
-  a += 4 * (size_t)kMaxRep * pps;
+  o.sc = a;  // per warp: 32 probabilities + kMaxRep rescale factors
+  a += 4 * (size_t)kComputeWarps * (32 + kMaxRep);
   o.mls = a;
   a += 4 * 3 * kMaxRep;
   a = align_to(a, 16);
-  o.ored = a;
-  int npg = kComputeThreads / (head_dim / 2);
-  a += 4 * (size_t)npg * kMaxRep * head_dim;
+  o.ored = a;  // per warp and head: o[D], running max, running sum
+  a += 4 * (size_t)kComputeWarps * rep_p * (head_dim + 2);
   o.total = align_to(g > a ? g : a, 128);
   return o;
 }
 
 __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
-  SmemOffsets o = smem_offsets(p.ring_stages, p.stage_bytes, p.pps, p.D);
+  SmemOffsets o = smem_offsets(p.ring_stages, p.stage_bytes, p.pps, p.D, p.rep_p);
   Smem s;
   s.ring = base;
   s.full = reinterpret_cast<uint64_t *>(base + o.full);
@@ -345,10 +401,33 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const int NS = p.ring_stages;
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
+  // L2 prefetch cursor: stays up to l2_prefetch_bytes ahead of the ring in the
+  // worker's stream of stages, across task boundaries, so HBM keeps streaming
+  // the next tiles while the compute warps wait on an event.
+  const long long dist = p.l2_prefetch_bytes;
+  int pf_n = 0, pf_st = 0, pf_ns = -1;
+  long long ahead = 0;
   for (int n = 0; n < q.count; ++n) {
     const DevTask t = p.tasks[q.first + n * q.stride];
     const int ns = task_stages(p, t);
     for (int st = 0; st < ns; ++st) {
+      if (dist > 0) {
+        while (ahead < dist && pf_n < q.count) {
+          const DevTask pt = p.tasks[q.first + pf_n * q.stride];
+          if (pf_ns < 0) pf_ns = task_stages(p, pt);
+          if (pf_st >= pf_ns) {
+            ++pf_n;
+            pf_st = 0;
+            pf_ns = -1;
+            continue;
+          }
+          const Copy pc = stage_copy(p, pt, pf_st);
+          prefetch_l2(pc.src0, pc.bytes0);
+          if (pc.bytes1) prefetch_l2(pc.src1, pc.bytes1);
+          ahead += pc.bytes0 + pc.bytes1;
+          ++pf_st;
+        }
+      }
       const int slot = (int)(k % NS);
       const uint32_t use = k / NS;
       if (use > 0) {
@@ -372,6 +451,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       mbar_arrive_expect_tx(&sm.full[slot], c.bytes0 + c.bytes1);
       bulk_g2s(dst, c.src0, c.bytes0, &sm.full[slot]);
       if (c.bytes1) bulk_g2s(dst + p.stage_bytes / 2, c.src1, c.bytes1, &sm.full[slot]);
+      ahead -= c.bytes0 + c.bytes1;
       ++k;
     }
   }
@@ -429,8 +509,51 @@ __device__ bool wait_event(const Params &p, int e, uint32_t epoch, int task) {
 // ---------------------------------------------------------------------------
 // GEMV task body (batch 1): prologue RMSNorm, weight stream, fused epilogue.
 // ---------------------------------------------------------------------------
-__device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uint32_t &k,
-                          int task_id) {
+// Epilogue of `n` finished tile rows whose warp partials sit in sm.red, the
+// first of them at arena row `row0`.  Runs on all compute threads.
+__device__ __forceinline__ void gemv_finish(const Params &p, const Smem &sm, int type,
+                                            const DevLayer *L, int row0, int n, int wpg,
+                                            float &best_v, int &best_i) {
+  const int tid = threadIdx.x;
+  if (type == 6) {  // rows (2i, 2i+1) = (gate_i, up_i): h_i = silu(g) * u
+    for (int f = tid; f < n / 2; f += kComputeThreads) {
+      float gv = 0.f, uv = 0.f;
+      for (int w = 0; w < wpg; ++w) {
+        gv += sm.red[(2 * f) * kComputeWarps + w];
+        uv += sm.red[(2 * f + 1) * kComputeWarps + w];
+      }
+      L->h[(row0 >> 1) + f] = gv / (1.f + __expf(-gv)) * uv;
+    }
+    return;
+  }
+  for (int f = tid; f < n; f += kComputeThreads) {
+    float v = 0.f;
+    for (int w = 0; w < wpg; ++w) v += sm.red[f * kComputeWarps + w];
+    const int r = row0 + f;
+    if (type == 2) {
+      L->qkv[r] = v;
+    } else if (type == 5) {
+      L->xm[r] = __ldcg(L->x_in + r) + v;
+    } else if (type == 7) {
+      L->x_out[r] = __ldcg(L->xm + r) + v;
+    } else {
+      if (p.logits) p.logits[r] = v;
+      if (v > best_v || (v == best_v && r < best_i)) {
+        best_v = v;
+        best_i = r;
+      }
+    }
+  }
+}
+
+// GEMV task (batch 1).  Prologue: the input vector in registers, RMSNorm
+// applied when the operator has one.  Main loop: every warp walks the ring
+// stages on its own (wait full, accumulate, release its share), writing warp
+// partial sums of each row to shared memory; no CTA barrier per stage.  The
+// epilogue runs once per task (or per kRedRows rows) on all threads.
+template <int CPT, int NR>
+__device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t,
+                                          uint32_t &k, int task_id) {
   const int type = t.type;
   const int layer = t.layer;
   const Gemv g = gemv_of(p, type, layer, (int)t.idx);
@@ -451,14 +574,13 @@ __device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uin
   const int grp = tid / tpg, li = tid - grp * tpg;
   const bool active = grp < ngroups;
   const int wpg = tpg >> 5, wig = li >> 5;  // warps per group, warp index in group
-  const int cpt = (nch + tpg - 1) / tpg;
 
   // activation chunks of this thread
-  float x[kMaxChunks][8];
+  float x[CPT][8];
 #pragma unroll
-  for (int j = 0; j < kMaxChunks; ++j) {
+  for (int j = 0; j < CPT; ++j) {
     const int c = li + j * tpg;
-    if (active && j < cpt && c < nch) {
+    if (active && c < nch) {
       const float4 a = __ldcg(reinterpret_cast<const float4 *>(act + 8 * c));
       const float4 b = __ldcg(reinterpret_cast<const float4 *>(act + 8 * c + 4));
       x[j][0] = a.x; x[j][1] = a.y; x[j][2] = a.z; x[j][3] = a.w;
@@ -471,7 +593,7 @@ __device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uin
   if (gain) {
     float ss = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j)
+    for (int j = 0; j < CPT; ++j)
 #pragma unroll
       for (int i = 0; i < 8; ++i) ss = fmaf(x[j][i], x[j][i], ss);
     ss = warp_sum(ss);
@@ -482,9 +604,9 @@ __device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uin
       for (int w = 0; w < wpg; ++w) tot += sm.ss[grp * wpg + w];
     const float inv = rsqrtf(tot / (float)K + p.eps);
 #pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) {
+    for (int j = 0; j < CPT; ++j) {
       const int c = li + j * tpg;
-      if (active && j < cpt && c < nch) {
+      if (active && c < nch) {
         const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gain + 8 * c));
         x[j][0] *= inv * bf_lo(gw.x); x[j][1] *= inv * bf_hi(gw.x);
         x[j][2] *= inv * bf_lo(gw.y); x[j][3] *= inv * bf_hi(gw.y);
@@ -496,77 +618,78 @@ __device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uin
 
   const int rows = g.row1 - g.row0;
   const int nst = (rows + g.rps - 1) / g.rps;
+  const int row16 = K >> 3;  // 16-byte chunks per row
   float best_v = -INFINITY;
   int best_i = 0x7fffffff;
+  int buf0 = 0;  // first tile row whose partials sm.red holds
   for (int st = 0; st < nst; ++st) {
-    const int r_here = min(g.rps, rows - st * g.rps);
-    if (!wait_full(p, sm, k, task_id)) {
-      sm.ctl[kAbort] = 1;
+    const int r0 = st * g.rps;
+    const int r_here = min(g.rps, rows - r0);
+    if (r0 + r_here - buf0 > kRedRows) {  // shared partials full: finish them
+      compute_sync();
+      if (!sm.ctl[kAbort]) gemv_finish(p, sm, type, L, g.row0 + buf0, r0 - buf0, wpg, best_v, best_i);
+      compute_sync();
+      buf0 = r0;
     }
-    if (!sm.ctl[kAbort]) {
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (got) {
       const uint16_t *ws =
           reinterpret_cast<const uint16_t *>(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
-      float *red = sm.red + (st & 1) * kMaxRowsPerStage * kComputeWarps;
       if (active) {
-        for (int r = grp; r < r_here; r += ngroups) {
-          const uint4 *wr = reinterpret_cast<const uint4 *>(ws + (size_t)r * K);
-          float acc = 0.f;
+        // NR rows at a time: NR independent (even, odd) accumulator pairs per
+        // thread fed by packed FMAs, then one transposed warp reduction
+        for (int rb = grp * NR; rb < r_here; rb += ngroups * NR) {
+          const int nr = min(NR, r_here - rb);
+          const uint4 *wr = reinterpret_cast<const uint4 *>(ws + (size_t)rb * K);
+          float acc[NR][2];
 #pragma unroll
-          for (int j = 0; j < kMaxChunks; ++j) {
-            const int c = li + j * tpg;
-            if (j < cpt && c < nch) acc += dot8(wr[c], x[j]);
+          for (int i = 0; i < NR; ++i) acc[i][0] = acc[i][1] = 0.f;
+          if (nr == NR) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+              const int c = li + j * tpg;
+              if (c < nch) {
+                uint4 w[NR];
+#pragma unroll
+                for (int i = 0; i < NR; ++i) w[i] = wr[i * row16 + c];
+#pragma unroll
+                for (int i = 0; i < NR; ++i) dot8_acc(w[i], x[j], acc[i]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+              const int c = li + j * tpg;
+              if (c < nch) {
+#pragma unroll
+                for (int i = 0; i < NR; ++i)
+                  if (i < nr) dot8_acc(wr[i * row16 + c], x[j], acc[i]);
+              }
+            }
           }
-          acc = warp_sum(acc);
-          if (lane == 0) red[r * kComputeWarps + wig] = acc;
+          float v8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v8[i] = i < NR ? acc[i][0] + acc[i][1] : 0.f;
+          const float v = warp_sum8(v8, lane);
+          if ((lane & 3) == 0 && (lane >> 2) < nr)
+            sm.red[(r0 - buf0 + rb + (lane >> 2)) * kComputeWarps + wig] = v;
         }
       }
-    }
-    release_stage(sm, p, k);
-    ++k;
-    compute_sync();
-    if (sm.ctl[kAbort]) return false;
-    const float *red = sm.red + (st & 1) * kMaxRowsPerStage * kComputeWarps;
-    const int n0 = g.row0 + st * g.rps;  // first arena row of the stage
-    if (type == 6) {
-      if (tid < r_here / 2) {
-        float gv = 0.f, uv = 0.f;
-        for (int w = 0; w < wpg; ++w) {
-          gv += red[(2 * tid) * kComputeWarps + w];
-          uv += red[(2 * tid + 1) * kComputeWarps + w];
-        }
-        const float hv = gv / (1.f + __expf(-gv)) * uv;
-        L->h[(n0 >> 1) + tid] = hv;
-      }
-    } else if (tid < r_here) {
-      float v = 0.f;
-      for (int w = 0; w < wpg; ++w) v += red[tid * kComputeWarps + w];
-      const int n = n0 + tid;
-      if (type == 2) {
-        L->qkv[n] = v;
-      } else if (type == 5) {
-        L->xm[n] = __ldcg(L->x_in + n) + v;
-      } else if (type == 7) {
-        L->x_out[n] = __ldcg(L->xm + n) + v;
-      } else {
-        if (p.logits) p.logits[n] = v;
-        if (v > best_v || (v == best_v && n < best_i)) {
-          best_v = v;
-          best_i = n;
-        }
-      }
+      release_stage(sm, p, k);
+      ++k;
     }
   }
+  compute_sync();
+  if (sm.ctl[kAbort]) return false;
+  gemv_finish(p, sm, type, L, g.row0 + buf0, rows - buf0, wpg, best_v, best_i);
   if (type == 8) {
-    if (tid < kMaxRowsPerStage) {
-      sm.lmv[tid] = best_v;
-      sm.lmi[tid] = best_i;
-    }
+    sm.lmv[tid] = best_v;
+    sm.lmi[tid] = best_i;
     compute_sync();
     if (tid == 0) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
-      const int nf = min(g.rps, rows);
-      for (int f = 0; f < nf; ++f) {
+      for (int f = 0; f < kComputeThreads; ++f) {
         const float v = sm.lmv[f];
         const int i = sm.lmi[f];
         if (v > bv || (v == bv && i < bi)) {
@@ -585,89 +708,105 @@ __device__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t, uin
 // ---------------------------------------------------------------------------
 // Attention: one (sequence b, kv head g, split s).
 // ---------------------------------------------------------------------------
-// Scores, softmax update and PV for n rows of K and V held in shared memory.
-__device__ __forceinline__ void attn_block(const Params &p, const Smem &sm, const uint16_t *Ks,
-                                           const uint16_t *Vs, int n, const float (&qr)[kMaxRep][4],
-                                           float (&o)[kMaxRep][2]) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int D = p.D, rep = p.rep, dpl = D >> 5;
-  // 1. scores s[h][j] = q_h . k_j (q already scaled by 1/sqrt(D))
-  for (int j = warp; j < n; j += kComputeWarps) {
-    float kf[4];
-    if (dpl == 4) {
-      const uint2 kv = *reinterpret_cast<const uint2 *>(Ks + (size_t)j * D + 4 * lane);
-      kf[0] = bf_lo(kv.x); kf[1] = bf_hi(kv.x); kf[2] = bf_lo(kv.y); kf[3] = bf_hi(kv.y);
-    } else {
-      const uint32_t kv = *reinterpret_cast<const uint32_t *>(Ks + (size_t)j * D + 2 * lane);
-      kf[0] = bf_lo(kv); kf[1] = bf_hi(kv); kf[2] = 0.f; kf[3] = 0.f;
-    }
-    float mine = 0.f;
+// One block of up to NP = 32 / RP positions for one warp: scores, online
+// softmax update of the warp's running state, and PV.  RP = q heads per kv head
+// rounded up to a power of two (heads >= rep are padding).  Lane l covers dims
+// [dpl*l, dpl*l + dpl) of every head; after the transposed score reduction lane
+// l holds the score of head l / NP at position l % NP, and keeps the running
+// max and sum of that head.  pw / aw: the warp's probability / rescale scratch.
+template <int RP>
+__device__ __forceinline__ void attn_block(const Params &p, float *pw, float *aw,
+                                           const uint16_t *Ks, const uint16_t *Vs, int j0, int n,
+                                           const float (&qr)[RP][4], float &m_run, float &l_run,
+                                           float (&o)[RP][4]) {
+  constexpr int NP = 32 / RP;
+  const int lane = threadIdx.x & 31;
+  const int D = p.D, dpl = D >> 5;
+  float v[32];
 #pragma unroll
-    for (int h = 0; h < kMaxRep; ++h) {
-      if (h < rep) {
-        float d = qr[h][0] * kf[0];
-        d = fmaf(qr[h][1], kf[1], d);
-        d = fmaf(qr[h][2], kf[2], d);
-        d = fmaf(qr[h][3], kf[3], d);
-        d = warp_sum(d);
-        if (lane == h) mine = d;
+  for (int jj = 0; jj < NP; ++jj) {
+    float kf[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j0 + jj < n) {
+      if (dpl == 4) {
+        const uint2 kv = *reinterpret_cast<const uint2 *>(Ks + (size_t)(j0 + jj) * D + 4 * lane);
+        kf[0] = bf_lo(kv.x); kf[1] = bf_hi(kv.x); kf[2] = bf_lo(kv.y); kf[3] = bf_hi(kv.y);
+      } else {
+        const uint32_t kv = *reinterpret_cast<const uint32_t *>(Ks + (size_t)(j0 + jj) * D + 2 * lane);
+        kf[0] = bf_lo(kv); kf[1] = bf_hi(kv);
       }
     }
-    if (lane < rep) sm.sc[lane * p.pps + j] = mine;
-  }
-  compute_sync();
-  // 2. online softmax update, one warp per head
-  if (warp < rep) {
-    const int h = warp;
-    float *s = sm.sc + h * p.pps;
-    const float m_old = sm.mls[h];
-    float mx = -INFINITY;
-    for (int j = lane; j < n; j += 32) mx = fmaxf(mx, s[j]);
-    mx = warp_max(mx);
-    const float m_new = fmaxf(m_old, mx);
-    float sum = 0.f;
-    for (int j = lane; j < n; j += 32) {
-      const float e = __expf(s[j] - m_new);
-      s[j] = e;
-      sum += e;
-    }
-    sum = warp_sum(sum);
-    if (lane == 0) {
-      const float alpha = m_old == -INFINITY ? 0.f : __expf(m_old - m_new);
-      sm.mls[h] = m_new;
-      sm.mls[kMaxRep + h] = sm.mls[kMaxRep + h] * alpha + sum;
-      sm.mls[2 * kMaxRep + h] = alpha;
-    }
-  }
-  compute_sync();
-  // 3. o = alpha * o + sum_j p_j v_j on (dim pair, position group)
-  const int half = D >> 1;
-  const int dp = tid % half, pg = tid / half, npg = kComputeThreads / half;
 #pragma unroll
-  for (int h = 0; h < kMaxRep; ++h) {
-    if (h < rep) {
-      const float a = sm.mls[2 * kMaxRep + h];
-      o[h][0] *= a;
-      o[h][1] *= a;
+    for (int h = 0; h < RP; ++h) {
+      float d = qr[h][0] * kf[0];
+      d = fmaf(qr[h][1], kf[1], d);
+      d = fmaf(qr[h][2], kf[2], d);
+      d = fmaf(qr[h][3], kf[3], d);
+      v[h * NP + jj] = d;
     }
   }
-  for (int j = pg; j < n; j += npg) {
-    const uint32_t vv = *reinterpret_cast<const uint32_t *>(Vs + (size_t)j * D + 2 * dp);
-    const float v0 = bf_lo(vv), v1 = bf_hi(vv);
+  float sc = warp_sum32(v, lane);
+  const int h = lane / NP, jj = lane % NP;
+  const bool valid = h < p.rep && j0 + jj < n;
+  sc = valid ? sc : -INFINITY;
+  float mx = sc;
 #pragma unroll
-    for (int h = 0; h < kMaxRep; ++h) {
-      if (h < rep) {
-        const float pj = sm.sc[h * p.pps + j];
-        o[h][0] = fmaf(pj, v0, o[h][0]);
-        o[h][1] = fmaf(pj, v1, o[h][1]);
+  for (int off = NP / 2; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  const float m_new = fmaxf(m_run, mx);
+  const float pj = valid ? __expf(sc - m_new) : 0.f;
+  float sum = pj;
+#pragma unroll
+  for (int off = NP / 2; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float alpha = m_run == -INFINITY ? 0.f : __expf(m_run - m_new);
+  l_run = l_run * alpha + sum;
+  m_run = m_new;
+  pw[jj * RP + h] = pj;
+  if (jj == 0) aw[h] = alpha;
+  __syncwarp();
+#pragma unroll
+  for (int hh = 0; hh < RP; ++hh) {
+    const float a = aw[hh];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[hh][i] *= a;
+  }
+#pragma unroll
+  for (int t = 0; t < NP; ++t) {
+    if (j0 + t < n) {
+      float vf[4] = {0.f, 0.f, 0.f, 0.f};
+      if (dpl == 4) {
+        const uint2 vv = *reinterpret_cast<const uint2 *>(Vs + (size_t)(j0 + t) * D + 4 * lane);
+        vf[0] = bf_lo(vv.x); vf[1] = bf_hi(vv.x); vf[2] = bf_lo(vv.y); vf[3] = bf_hi(vv.y);
+      } else {
+        const uint32_t vv = *reinterpret_cast<const uint32_t *>(Vs + (size_t)(j0 + t) * D + 2 * lane);
+        vf[0] = bf_lo(vv); vf[1] = bf_hi(vv);
       }
+      float pr[RP];
+      if constexpr (RP >= 4) {
+#pragma unroll
+        for (int q = 0; q < RP; q += 4) {
+          const float4 p4 = *reinterpret_cast<const float4 *>(pw + t * RP + q);
+          pr[q] = p4.x; pr[q + 1] = p4.y; pr[q + 2] = p4.z; pr[q + 3] = p4.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < RP; ++q) pr[q] = pw[t * RP + q];
+      }
+#pragma unroll
+      for (int hh = 0; hh < RP; ++hh)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[hh][i] = fmaf(pr[hh], vf[i], o[hh][i]);
     }
   }
-  compute_sync();
+  __syncwarp();
 }
 
-__device__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t, uint32_t &k,
-                          int task_id) {
+// Decode attention for one (sequence b, kv head g, split s): q/k RMSNorm and
+// RoPE prologue, K/V append, then every warp runs flash-decoding style over
+// its own positions (no CTA barrier inside the loop) and the warps' states
+// are merged once at the end.
+template <int RP>
+__device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
+                                       uint32_t &k, int task_id) {
+  constexpr int NP = 32 / RP;
   const AttnSpan a = attn_span(p, (int)t.idx);
   if (!a.active) return true;  // the split starts past the new row: nothing to do
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -711,93 +850,123 @@ __device__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t, uin
       }
     }
   }
-  if (tid < kMaxRep) {
-    sm.mls[tid] = -INFINITY;
-    sm.mls[kMaxRep + tid] = 0.f;
-    sm.mls[2 * kMaxRep + tid] = 1.f;
-  }
   compute_sync();
-  float qr[kMaxRep][4];
+  float qr[RP][4];
 #pragma unroll
-  for (int h = 0; h < kMaxRep; ++h)
+  for (int h = 0; h < RP; ++h)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       qr[h][i] = (h < rep && i < dpl) ? sm.q[h * kMaxHeadDim + dpl * lane + i] : 0.f;
-  float o[kMaxRep][2];
+  float o[RP][4];
 #pragma unroll
-  for (int h = 0; h < kMaxRep; ++h) o[h][0] = o[h][1] = 0.f;
+  for (int h = 0; h < RP; ++h)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[h][i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  float *pw = sm.sc + warp * (32 + kMaxRep);
+  float *aw = pw + 32;
 
   const int cached = a.cached_end - a.p0;
   const int nst = cached > 0 ? (cached + p.pps - 1) / p.pps : 0;
   for (int st = 0; st < nst; ++st) {
     const int n = min(p.pps, cached - st * p.pps);
-    bool ok = wait_full(p, sm, k, task_id);
-    if (!ok) sm.ctl[kAbort] = 1;
-    compute_sync();
-    if (sm.ctl[kAbort]) {
-      release_stage(sm, p, k);
-      ++k;
-      return false;
-    }
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (!got) continue;
     const uint16_t *Ks =
         reinterpret_cast<const uint16_t *>(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
     const uint16_t *Vs = Ks + p.stage_bytes / 4;  // second half of the stage
-    attn_block(p, sm, Ks, Vs, n, qr, o);
+    for (int j0 = warp * NP; j0 < n; j0 += kComputeWarps * NP)
+      attn_block<RP>(p, pw, aw, Ks, Vs, j0, n, qr, m_run, l_run, o);
     release_stage(sm, p, k);
     ++k;
   }
-  if (a.has_new) attn_block(p, sm, sm.knew, sm.vnew, 1, qr, o);
+  // the new row: one more block, on the warp after the last cached block
+  if (a.has_new && warp == ((cached + NP - 1) / NP) % kComputeWarps)
+    attn_block<RP>(p, pw, aw, sm.knew, sm.vnew, 0, 1, qr, m_run, l_run, o);
 
-  // reduce the position groups, then write the normalised output (one split)
-  // or the unnormalised partial with its running max and sum (several splits)
-  const int half = D >> 1;
-  const int dp = tid % half, pg = tid / half, npg = kComputeThreads / half;
+  // merge the warps' states
+  const int stride = D + 2;
+  float *st_w = sm.ored + (size_t)warp * RP * stride;
 #pragma unroll
-  for (int h = 0; h < kMaxRep; ++h) {
-    if (h < rep) {
-      sm.ored[(pg * kMaxRep + h) * D + 2 * dp] = o[h][0];
-      sm.ored[(pg * kMaxRep + h) * D + 2 * dp + 1] = o[h][1];
-    }
+  for (int h = 0; h < RP; ++h)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < dpl) st_w[h * stride + dpl * lane + i] = o[h][i];
+  if (lane % NP == 0) {
+    const int h = lane / NP;
+    st_w[h * stride + D] = m_run;
+    st_w[h * stride + D + 1] = l_run;
   }
   compute_sync();
+  if (sm.ctl[kAbort]) return false;
   for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
     const int h = oi / D, d = oi - h * D;
-    float v = 0.f;
-    for (int q = 0; q < npg; ++q) v += sm.ored[(q * kMaxRep + h) * D + d];
+    float M = -INFINITY;
+    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, sm.ored[((size_t)w * RP + h) * stride + D]);
+    float num = 0.f, den = 0.f;
+    for (int w = 0; w < kComputeWarps; ++w) {
+      const float *sw = sm.ored + ((size_t)w * RP + h) * stride;
+      const float mw = sw[D];
+      const float e = mw == -INFINITY ? 0.f : __expf(mw - M);
+      den = fmaf(e, sw[D + 1], den);
+      num = fmaf(e, sw[d], num);
+    }
     const int head = a.g * rep + h;
     if (p.S == 1) {
-      L.att[(size_t)a.b * p.qdim + head * D + d] = v / sm.mls[kMaxRep + h];
+      L.att[(size_t)a.b * p.qdim + head * D + d] = num / den;
     } else {
       float *dst = L.part + (((size_t)a.b * p.Hq + head) * p.S + a.s) * (D + 2);
-      dst[d] = v;
+      dst[d] = num;
       if (d == 0) {
-        dst[D] = sm.mls[h];
-        dst[D + 1] = sm.mls[kMaxRep + h];
+        dst[D] = M;
+        dst[D + 1] = den;
       }
     }
   }
   return true;
 }
 
-__device__ void merge_task(const Params &p, const DevTask &t) {
+// Online-softmax merge of the splits of one (sequence, kv head):
+//   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
+__device__ void merge_task(const Params &p, const Smem &sm, const DevTask &t) {
   const int b = (int)t.idx / p.Hkv, g = (int)t.idx % p.Hkv;
   const DevLayer &L = p.layers[t.layer];
   const int Lb = p.kv_len[b];
   const int ns = min(p.S, Lb / p.chunk + 1);  // splits that hold any position
-  const int D = p.D;
-  for (int oi = threadIdx.x; oi < p.rep * D; oi += kComputeThreads) {
-    const int h = oi / D, d = oi - h * D;
-    const int head = g * p.rep + h;
-    const float *base = L.part + ((size_t)b * p.Hq + head) * p.S * (D + 2);
+  const int D = p.D, rep = p.rep;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float *wgt = sm.ored;               // [rep][ns]
+  float *sum_l = sm.ored + rep * ns;  // [rep][ns]
+  const float *part = L.part + (size_t)b * p.Hq * p.S * (D + 2);
+  for (int i = tid; i < rep * ns; i += kComputeThreads) {
+    const int h = i / ns, s = i - h * ns;
+    const float *src = part + ((size_t)(g * rep + h) * p.S + s) * (D + 2);
+    wgt[i] = __ldcg(src + D);
+    sum_l[i] = __ldcg(src + D + 1);
+  }
+  compute_sync();
+  if (warp < rep) {
+    const int h = warp;
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, __ldcg(base + s * (D + 2) + D));
-    float den = 0.f, num = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const float w = __expf(__ldcg(base + s * (D + 2) + D) - M);
-      den = fmaf(w, __ldcg(base + s * (D + 2) + D + 1), den);
-      num = fmaf(w, __ldcg(base + s * (D + 2) + d), num);
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, wgt[h * ns + s]);
+    M = warp_max(M);
+    float den = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+      const float w = __expf(wgt[h * ns + s] - M);
+      wgt[h * ns + s] = w;
+      den = fmaf(w, sum_l[h * ns + s], den);
     }
-    L.att[(size_t)b * p.qdim + head * D + d] = num / den;
+    den = warp_sum(den);
+    if (lane == 0) sm.mls[h] = 1.f / den;
+  }
+  compute_sync();
+  for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
+    const int h = oi / D, d = oi - h * D;
+    const float *src = part + (size_t)(g * rep + h) * p.S * (D + 2) + d;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) acc = fmaf(wgt[h * ns + s], __ldcg(src + (size_t)s * (D + 2)), acc);
+    L.att[(size_t)b * p.qdim + (g * rep + h) * D + d] = acc * sm.mls[h];
   }
 }
 
@@ -831,7 +1000,7 @@ __device__ void argmax_task(const Params &p, uint32_t epoch) {
 // ---------------------------------------------------------------------------
 // The worker kernel
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const Smem sm = carve(smem_raw, p);
   const int tid = threadIdx.x;
@@ -878,28 +1047,59 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const Params p) 
   } else {
     const uint32_t epoch = (uint32_t)sm.ctl[kEpoch];
     uint32_t k = 0;
+    const int rp = p.rep_p;
     for (int n = 0; n < q.count; ++n) {
       const int id = q.first + n * q.stride;
       const DevTask t = p.tasks[id];
+      uint64_t t_wait = 0, t_ready = 0;
+      if (p.trace && tid == 0) t_wait = global_timer();
       if (p.persistent && t.dep >= 0 && tid == 0) {
         if (!wait_event(p, t.dep, epoch, id)) sm.ctl[kAbort] = 1;
       }
       compute_sync();
       if (sm.ctl[kAbort]) break;
+      if (p.trace && tid == 0) t_ready = global_timer();
       bool ok = true;
       switch (t.type) {
         case 1: embed_task(p); break;
-        case 2: case 5: case 6: case 7: case 8: ok = gemv_task(p, sm, t, k, id); break;
-        case 3: ok = attn_task(p, sm, t, k, id); break;
-        case 4: merge_task(p, t); break;
+        case 2: case 5: case 6: case 7: case 8: {
+          const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
+          const int nch = K >> 3;
+          const int cpt = nch <= kComputeThreads ? 1 : (nch + kComputeThreads - 1) / kComputeThreads;
+          const int rps = t.type == 2 ? p.rps_qkv : t.type == 5 ? p.rps_o : t.type == 6 ? p.rps_gu
+                        : t.type == 7 ? p.rps_down : p.rps_lm;
+          if (cpt == 1 && rps >= 8) ok = gemv_task<1, 8>(p, sm, t, k, id);
+          else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id);
+          else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id);
+          else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id);
+          else ok = gemv_task<8, 8>(p, sm, t, k, id);
+          break;
+        }
+        case 3:
+          ok = rp == 1 ? attn_task<1>(p, sm, t, k, id)
+             : rp == 2 ? attn_task<2>(p, sm, t, k, id)
+             : rp == 4 ? attn_task<4>(p, sm, t, k, id)
+                       : attn_task<8>(p, sm, t, k, id);
+          break;
+        case 4: merge_task(p, sm, t); break;
         case 9: argmax_task(p, epoch); break;
         default: break;  // empty task
       }
       if (!ok) break;
       compute_sync();
-      if (p.persistent && t.trig >= 0 && tid == 0) {
-        __threadfence();
-        red_release_add(p.counters + t.trig, 1u);
+      if (tid == 0) {
+        // bar.sync above orders every compute thread's stores before this
+        // release, which is cumulative at gpu scope
+        if (p.persistent && t.trig >= 0) red_release_add(p.counters + t.trig, 1u);
+        if (p.trace) {
+          uint32_t smid;
+          asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+          unsigned long long *tr = p.trace + 4 * (size_t)id;
+          tr[0] = t_wait;
+          tr[1] = t_ready;
+          tr[2] = global_timer();
+          tr[3] = ((unsigned long long)smid << 32) | blockIdx.x;
+        }
       }
     }
     if (tid == 0) sm.ctl[kConsumed] = (int)k;
@@ -921,8 +1121,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const Params p) 
 
 }  // namespace
 
-size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim) {
-  return smem_offsets(stages, stage_bytes, pps, head_dim).total;
+size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int rep_p) {
+  return smem_offsets(stages, stage_bytes, pps, head_dim, rep_p).total;
 }
 
 cudaError_t worker_configure(size_t smem) {

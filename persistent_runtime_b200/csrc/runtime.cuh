@@ -12,6 +12,7 @@ constexpr int kComputeThreads = kComputeWarps * 32;  // threads that run task bo
 constexpr int kThreads = kComputeThreads + 32;       // + one producer (TMA) warp
 constexpr int kMaxChunks = 8;          // 16-byte weight chunks per thread and row: K <= 16384
 constexpr int kMaxRowsPerStage = 64;   // GEMV rows in one ring stage
+constexpr int kRedRows = 256;          // GEMV rows whose warp partials shared memory holds
 constexpr int kMaxRep = 8;             // q heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxBatch = 16;
@@ -75,6 +76,7 @@ struct Params {
   float *logits;                // [B][V] or null
   // shapes
   int B, H, Hq, Hkv, D, F, V, Ly, Lcap, rep, grp, n_qkv, qdim;
+  int rep_p;  // rep rounded up to a power of two (1, 2, 4 or 8)
   float eps;
   float attn_scale;  // 1 / sqrt(D)
   // tiling
@@ -83,8 +85,10 @@ struct Params {
   int pps;                                       // KV positions per ring stage
   // ring
   int ring_stages, stage_bytes;
-  int l2_prefetch_bytes;
+  int l2_prefetch_bytes;  // per worker: L2 prefetch distance ahead of the ring
   unsigned long long timeout_ns;
+  // optional task trace: per task id {wait begin, ready, end, worker} (%globaltimer ns)
+  unsigned long long *trace;
 };
 
 }  // namespace mk

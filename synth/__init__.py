@@ -114,7 +114,11 @@ Q8B_B8 = Workload("qwen3-8b-b8", 36, 4096, 32, 8, 128, 12288, 151936, 0, 8, None
                   kv_len_range=(256, 4096), steps=64)
 Q8B_B16 = Workload("qwen3-8b-b16", 36, 4096, 32, 8, 128, 12288, 151936, 0, 16, 8192, steps=32)
 
-WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16)}
+# Profiling case: the 8B layer shapes with 4 layers (2.7 GB of weights), small
+# enough for multi-pass counter captures.
+Q8B_4L = Q8B.with_(name="qwen3-8b-4layer", n_layers=4)
+
+WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16, Q8B_4L)}
 
 # ----------------------------------------------------------------------------
 # Stream ids (one counter stream per tensor)

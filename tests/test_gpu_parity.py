@@ -8,8 +8,11 @@ from gpu_helpers import Case, compare_step, torch
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("built_libs")]
 
 
-def _kv_rows_close(case, ref_k, ref_v, lens):
-    """Rows appended at position lens[b]: GPU and oracle agree to bf16 rounding."""
+def _kv_rows_close(case, ref_k, ref_v, lens, untouched=None):
+    """Rows appended at position lens[b]: the GPU's and the oracle's fp32 values
+    differ only in summation order, so after rounding to bf16 almost every
+    element is bit-identical and the rest differ by about one bf16 step of the
+    row's scale."""
     gk = case.d_k.cpu().numpy().view(np.uint16)
     gv = case.d_v.cpu().numpy().view(np.uint16)
     for b in range(case.w.batch):
@@ -17,9 +20,12 @@ def _kv_rows_close(case, ref_k, ref_v, lens):
         for arr_g, arr_r in ((gk, ref_k), (gv, ref_v)):
             a = synth.bf16_to_f32(arr_g[:, b, :, L]).astype(np.float64)
             r = synth.bf16_to_f32(arr_r[:, b, :, L]).astype(np.float64)
-            assert np.all(np.abs(a - r) <= 2 ** -7 * np.abs(r) + 1e-6), "appended K/V row differs"
-        # rows before L are untouched
-        np.testing.assert_array_equal(gk[:, b, :, :L], case.k[:, b, :, :L])
+            scale = np.max(np.abs(r), axis=-1, keepdims=True)
+            assert np.all(np.abs(a - r) <= 1e-2 * scale), "appended K/V row differs"
+            assert np.mean(arr_g[:, b, :, L] == arr_r[:, b, :, L]) > 0.9
+        # rows the steps never wrote are untouched
+        U = L if untouched is None else int(untouched[b])
+        np.testing.assert_array_equal(gk[:, b, :, :U], case.k[:, b, :, :U])
 
 
 @pytest.mark.parametrize("tied", [0, 1])
@@ -94,7 +100,7 @@ def test_qwen3_06b_step_matches_oracle():
         ref = c.oracle_step(tokens=tok, k=k, v=v, lens=lens)
         compare_step(ref, got, w, f"0.6b step{step}")
         tok = ref["tokens"].copy()
-    _kv_rows_close(c, k, v, c.lens + 1)
+    _kv_rows_close(c, k, v, c.lens + 1, untouched=c.lens)
 
 
 def test_bad_inputs_are_rejected_and_write_nothing():
@@ -144,3 +150,16 @@ def test_event_wait_times_out_cleanly_and_recovers():
     got = c.gpu_step()
     ref = c.oracle_step(k=c.k.copy(), v=c.v.copy(), lens=c.lens.copy())
     compare_step(ref, got, w, "after-timeout")
+
+
+def test_qwen3_8b_bs1_full_size_step_matches_oracle():
+    # The bench's workload and launch configuration: 36 layers, hidden 4096,
+    # 151936 vocab, 1024 cached rows, capacity 1024 + 64, one CTA per SM.
+    w = synth.Q8B
+    c = Case(w, seed=0, extra_cap=64)
+    assert c.mk.info().num_workers == torch().cuda.get_device_properties(0).multi_processor_count
+    k, v, lens = c.k.copy(), c.v.copy(), c.lens.copy()
+    got = c.gpu_step()
+    ref = c.oracle_step(k=k, v=v, lens=lens)
+    compare_step(ref, got, w, "8b")
+    _kv_rows_close(c, k, v, c.lens)
