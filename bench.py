@@ -389,7 +389,7 @@ def main():
     if args.trace:
         from persistent_runtime_b200 import trace as mktrace
         g = mk.graph()
-        buf = torch.zeros(4 * g.n_tasks, dtype=torch.int64, device="cuda")
+        buf = torch.zeros(8 * g.n_tasks, dtype=torch.int64, device="cuda")
         mk.set_trace(buf)
         reset()
         step()

@@ -232,10 +232,11 @@ mk_status mk_final_hidden(const mk_handle *h, const float **d_ptr);
  * that event time out, which exercises the bounded-wait error path. */
 mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *stream);
 
-/* mk_set_trace - record, for every task of later steps, four uint64 words
- * {wait begin, ready, end, (smid << 32) | worker} (%globaltimer ns) into the
- * caller's device buffer d_buf of `bytes` >= 32 * n_tasks bytes (task id
- * order).  d_buf = NULL turns tracing off.  The buffer must outlive the steps
+/* mk_set_trace - record, for every task of later steps, eight uint64 words
+ * {wait begin, ready, end, (smid << 32) | worker, prologue done, streaming
+ * done, 0, 0} (%globaltimer ns; the two marks are 0 for tasks without those
+ * phases) into the caller's device buffer d_buf of `bytes` >= 64 * n_tasks
+ * bytes (task id order).  d_buf = NULL turns tracing off.  The buffer must outlive the steps
  * that use it.  This is the "--profiling" trace of the MPK page, section 7.2. */
 mk_status mk_set_trace(mk_handle *h, void *d_buf, int64_t bytes);
 

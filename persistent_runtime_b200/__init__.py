@@ -304,7 +304,7 @@ class Megakernel:
                self._h)
 
     def set_trace(self, buf=None):
-        """buf: int64/uint64 torch tensor with >= 4 * n_tasks elements, or None."""
+        """buf: int64/uint64 torch tensor with >= 8 * n_tasks elements, or None."""
         if buf is None:
             _check(lib().mk_set_trace(self._h, None, 0), self._h)
         else:

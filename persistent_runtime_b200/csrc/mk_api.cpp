@@ -641,8 +641,8 @@ mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *str
 
 mk_status mk_set_trace(mk_handle *h, void *d_buf, int64_t bytes) {
   if (!h || h->host_only) return fail(h, MK_ERR_ARG, "no device state");
-  if (d_buf && bytes < (int64_t)32 * (int64_t)h->graph.type.size())
-    return fail(h, MK_ERR_ARG, "trace buffer smaller than 32 bytes per task");
+  if (d_buf && bytes < (int64_t)64 * (int64_t)h->graph.type.size())
+    return fail(h, MK_ERR_ARG, "trace buffer smaller than 64 bytes per task");
   h->base.trace = static_cast<unsigned long long *>(d_buf);
   return MK_OK;
 }

@@ -196,6 +196,7 @@ struct Smem {
   uint8_t *ring;
   uint64_t *full, *empty;
   volatile int *ctl;
+  unsigned long long *tmark;  // [4] trace marks: prologue done, streaming done, ready
   // GEMV scratch
   float *red;   // [kRedRows][kComputeWarps] warp partial sums of tile rows
   float *ss;    // [kComputeWarps]
@@ -212,7 +213,7 @@ struct Smem {
 __host__ __device__ inline size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct SmemOffsets {
-  size_t full, empty, ctl, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, total;
+  size_t full, empty, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, total;
 };
 
 __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes, int pps,
@@ -226,6 +227,8 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   o.ctl = p;
   p += 4 * kCtlWords;
   p = align_to(p, 16);
+  o.tmark = p;
+  p += 32;
   // GEMV scratch
   size_t g = p;
   o.red = g;
@@ -262,6 +265,7 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
   s.full = reinterpret_cast<uint64_t *>(base + o.full);
   s.empty = reinterpret_cast<uint64_t *>(base + o.empty);
   s.ctl = reinterpret_cast<volatile int *>(base + o.ctl);
+  s.tmark = reinterpret_cast<unsigned long long *>(base + o.tmark);
   s.red = reinterpret_cast<float *>(base + o.red);
   s.ss = reinterpret_cast<float *>(base + o.ss);
   s.lmv = reinterpret_cast<float *>(base + o.lmv);
@@ -273,6 +277,11 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
   s.mls = reinterpret_cast<float *>(base + o.mls);
   s.ored = reinterpret_cast<float *>(base + o.ored);
   return s;
+}
+
+// Trace mark i (0: prologue done, 1: streaming done) of the running task.
+__device__ __forceinline__ void trace_mark(const Params &p, const Smem &sm, int i) {
+  if (p.trace && threadIdx.x == 0) sm.tmark[i] = global_timer();
 }
 
 __device__ void record_error(const Params &p, int code, int task, int event) {
@@ -401,32 +410,32 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const int NS = p.ring_stages;
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
-  // L2 prefetch cursor: stays up to l2_prefetch_bytes ahead of the ring in the
-  // worker's stream of stages, across task boundaries, so HBM keeps streaming
-  // the next tiles while the compute warps wait on an event.
+  // L2 prefetch cursor (stage index pf_k in the worker's stream of stages,
+  // across task boundaries).  While the producer is blocked on a full ring it
+  // prefetches the next stages into L2, up to l2_prefetch_bytes ahead of the
+  // ring, so HBM keeps streaming while the compute warps wait on an event.
   const long long dist = p.l2_prefetch_bytes;
   int pf_n = 0, pf_st = 0, pf_ns = -1;
+  uint32_t pf_k = 0;
   long long ahead = 0;
   for (int n = 0; n < q.count; ++n) {
     const DevTask t = p.tasks[q.first + n * q.stride];
     const int ns = task_stages(p, t);
     for (int st = 0; st < ns; ++st) {
       if (dist > 0) {
-        while (ahead < dist && pf_n < q.count) {
-          const DevTask pt = p.tasks[q.first + pf_n * q.stride];
-          if (pf_ns < 0) pf_ns = task_stages(p, pt);
+        // stages before k were issued without a prefetch: move the cursor on
+        while (pf_k < k && pf_n < q.count) {
+          if (pf_ns < 0) pf_ns = task_stages(p, p.tasks[q.first + pf_n * q.stride]);
           if (pf_st >= pf_ns) {
             ++pf_n;
             pf_st = 0;
             pf_ns = -1;
             continue;
           }
-          const Copy pc = stage_copy(p, pt, pf_st);
-          prefetch_l2(pc.src0, pc.bytes0);
-          if (pc.bytes1) prefetch_l2(pc.src1, pc.bytes1);
-          ahead += pc.bytes0 + pc.bytes1;
           ++pf_st;
+          ++pf_k;
         }
+        if (pf_k <= k) ahead = 0;
       }
       const int slot = (int)(k % NS);
       const uint32_t use = k / NS;
@@ -436,7 +445,24 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
         uint32_t spins = 0;
         while (!mbar_test(&sm.empty[slot], par)) {
           if (sm.ctl[kAbort]) goto out;
-          if ((++spins & 255u) == 0) {
+          ++spins;
+          if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count) {
+            const DevTask pt = p.tasks[q.first + pf_n * q.stride];
+            if (pf_ns < 0) pf_ns = task_stages(p, pt);
+            if (pf_st >= pf_ns) {
+              ++pf_n;
+              pf_st = 0;
+              pf_ns = -1;
+            } else {
+              const Copy pc = stage_copy(p, pt, pf_st);
+              prefetch_l2(pc.src0, pc.bytes0);
+              if (pc.bytes1) prefetch_l2(pc.src1, pc.bytes1);
+              ahead += pc.bytes0 + pc.bytes1;
+              ++pf_st;
+              ++pf_k;
+            }
+          }
+          if ((spins & 255u) == 0) {
             uint64_t now = global_timer();
             if (t0 == 0) t0 = now;
             else if (now - t0 > budget) {
@@ -451,7 +477,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       mbar_arrive_expect_tx(&sm.full[slot], c.bytes0 + c.bytes1);
       bulk_g2s(dst, c.src0, c.bytes0, &sm.full[slot]);
       if (c.bytes1) bulk_g2s(dst + p.stage_bytes / 2, c.src1, c.bytes1, &sm.full[slot]);
-      ahead -= c.bytes0 + c.bytes1;
+      if (dist > 0 && pf_k > k) ahead -= c.bytes0 + c.bytes1;  // stage k was prefetched
       ++k;
     }
   }
@@ -506,6 +532,25 @@ __device__ bool wait_event(const Params &p, int e, uint32_t epoch, int task) {
   }
 }
 
+// The wait for a task's dependency event.  Task bodies first issue the loads
+// that do not depend on this step's results (gains, RoPE factors), then call
+// this; every compute thread calls it exactly once per task.
+struct DepWait {
+  const Params &p;
+  const Smem &sm;
+  int dep;
+  uint32_t epoch;
+  int task;
+  __device__ __forceinline__ bool operator()() const {
+    if (p.persistent && dep >= 0 && threadIdx.x == 0) {
+      if (!wait_event(p, dep, epoch, task)) sm.ctl[kAbort] = 1;
+    }
+    compute_sync();
+    if (p.trace && threadIdx.x == 0) sm.tmark[2] = global_timer();
+    return !sm.ctl[kAbort];
+  }
+};
+
 // ---------------------------------------------------------------------------
 // GEMV task body (batch 1): prologue RMSNorm, weight stream, fused epilogue.
 // ---------------------------------------------------------------------------
@@ -513,7 +558,7 @@ __device__ bool wait_event(const Params &p, int e, uint32_t epoch, int task) {
 // first of them at arena row `row0`.  Runs on all compute threads.
 __device__ __forceinline__ void gemv_finish(const Params &p, const Smem &sm, int type,
                                             const DevLayer *L, int row0, int n, int wpg,
-                                            float &best_v, int &best_i) {
+                                            float res, float &best_v, int &best_i) {
   const int tid = threadIdx.x;
   if (type == 6) {  // rows (2i, 2i+1) = (gate_i, up_i): h_i = silu(g) * u
     for (int f = tid; f < n / 2; f += kComputeThreads) {
@@ -533,9 +578,9 @@ __device__ __forceinline__ void gemv_finish(const Params &p, const Smem &sm, int
     if (type == 2) {
       L->qkv[r] = v;
     } else if (type == 5) {
-      L->xm[r] = __ldcg(L->x_in + r) + v;
+      L->xm[r] = (f == tid ? res : __ldcg(L->x_in + r)) + v;
     } else if (type == 7) {
-      L->x_out[r] = __ldcg(L->xm + r) + v;
+      L->x_out[r] = (f == tid ? res : __ldcg(L->xm + r)) + v;
     } else {
       if (p.logits) p.logits[r] = v;
       if (v > best_v || (v == best_v && r < best_i)) {
@@ -553,7 +598,7 @@ __device__ __forceinline__ void gemv_finish(const Params &p, const Smem &sm, int
 // epilogue runs once per task (or per kRedRows rows) on all threads.
 template <int CPT, int NR>
 __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const DevTask &t,
-                                          uint32_t &k, int task_id) {
+                                          uint32_t &k, int task_id, const DepWait &dep_wait) {
   const int type = t.type;
   const int layer = t.layer;
   const Gemv g = gemv_of(p, type, layer, (int)t.idx);
@@ -575,6 +620,15 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
   const bool active = grp < ngroups;
   const int wpg = tpg >> 5, wig = li >> 5;  // warps per group, warp index in group
 
+  // norm gains of this thread's chunks: weights, so loaded before the wait
+  uint4 gw[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int c = li + j * tpg;
+    gw[j] = (gain && active && c < nch) ? __ldg(reinterpret_cast<const uint4 *>(gain + 8 * c))
+                                        : make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (!dep_wait()) return false;
   // activation chunks of this thread
   float x[CPT][8];
 #pragma unroll
@@ -607,11 +661,10 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
     for (int j = 0; j < CPT; ++j) {
       const int c = li + j * tpg;
       if (active && c < nch) {
-        const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gain + 8 * c));
-        x[j][0] *= inv * bf_lo(gw.x); x[j][1] *= inv * bf_hi(gw.x);
-        x[j][2] *= inv * bf_lo(gw.y); x[j][3] *= inv * bf_hi(gw.y);
-        x[j][4] *= inv * bf_lo(gw.z); x[j][5] *= inv * bf_hi(gw.z);
-        x[j][6] *= inv * bf_lo(gw.w); x[j][7] *= inv * bf_hi(gw.w);
+        x[j][0] *= inv * bf_lo(gw[j].x); x[j][1] *= inv * bf_hi(gw[j].x);
+        x[j][2] *= inv * bf_lo(gw[j].y); x[j][3] *= inv * bf_hi(gw[j].y);
+        x[j][4] *= inv * bf_lo(gw[j].z); x[j][5] *= inv * bf_hi(gw[j].z);
+        x[j][6] *= inv * bf_lo(gw[j].w); x[j][7] *= inv * bf_hi(gw[j].w);
       }
     }
   }
@@ -619,15 +672,20 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
   const int rows = g.row1 - g.row0;
   const int nst = (rows + g.rps - 1) / g.rps;
   const int row16 = K >> 3;  // 16-byte chunks per row
+  // residual of the row this thread finishes, loaded now to hide its latency
+  float res = 0.f;
+  if (tid < rows && (type == 5 || type == 7))
+    res = __ldcg((type == 5 ? L->x_in : L->xm) + g.row0 + tid);
   float best_v = -INFINITY;
   int best_i = 0x7fffffff;
   int buf0 = 0;  // first tile row whose partials sm.red holds
+  trace_mark(p, sm, 0);
   for (int st = 0; st < nst; ++st) {
     const int r0 = st * g.rps;
     const int r_here = min(g.rps, rows - r0);
     if (r0 + r_here - buf0 > kRedRows) {  // shared partials full: finish them
       compute_sync();
-      if (!sm.ctl[kAbort]) gemv_finish(p, sm, type, L, g.row0 + buf0, r0 - buf0, wpg, best_v, best_i);
+      if (!sm.ctl[kAbort]) gemv_finish(p, sm, type, L, g.row0 + buf0, r0 - buf0, wpg, res, best_v, best_i);
       compute_sync();
       buf0 = r0;
     }
@@ -641,9 +699,14 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
         for (int rb = grp * NR; rb < r_here; rb += ngroups * NR) {
           const int nr = min(NR, r_here - rb);
           const uint4 *wr = reinterpret_cast<const uint4 *>(ws + (size_t)rb * K);
-          float acc[NR][2];
+          // few rows per batch: spread the chunks over AS accumulator sets so
+          // every thread still has >= 8 independent FMA chains
+          constexpr int AS = NR >= 4 ? 1 : (CPT >= 3 ? 3 : CPT);
+          float acc[NR][AS][2];
 #pragma unroll
-          for (int i = 0; i < NR; ++i) acc[i][0] = acc[i][1] = 0.f;
+          for (int i = 0; i < NR; ++i)
+#pragma unroll
+            for (int a = 0; a < AS; ++a) acc[i][a][0] = acc[i][a][1] = 0.f;
           if (nr == NR) {
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
@@ -653,7 +716,7 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 #pragma unroll
                 for (int i = 0; i < NR; ++i) w[i] = wr[i * row16 + c];
 #pragma unroll
-                for (int i = 0; i < NR; ++i) dot8_acc(w[i], x[j], acc[i]);
+                for (int i = 0; i < NR; ++i) dot8_acc(w[i], x[j], acc[i][j % AS]);
               }
             }
           } else {
@@ -663,13 +726,20 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
               if (c < nch) {
 #pragma unroll
                 for (int i = 0; i < NR; ++i)
-                  if (i < nr) dot8_acc(wr[i * row16 + c], x[j], acc[i]);
+                  if (i < nr) dot8_acc(wr[i * row16 + c], x[j], acc[i][j % AS]);
               }
             }
           }
           float v8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v8[i] = i < NR ? acc[i][0] + acc[i][1] : 0.f;
+          for (int i = 0; i < 8; ++i) {
+            float v = 0.f;
+            if (i < NR) {
+#pragma unroll
+              for (int a = 0; a < AS; ++a) v += acc[i][a][0] + acc[i][a][1];
+            }
+            v8[i] = v;
+          }
           const float v = warp_sum8(v8, lane);
           if ((lane & 3) == 0 && (lane >> 2) < nr)
             sm.red[(r0 - buf0 + rb + (lane >> 2)) * kComputeWarps + wig] = v;
@@ -679,27 +749,45 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
       ++k;
     }
   }
+  trace_mark(p, sm, 1);
   compute_sync();
   if (sm.ctl[kAbort]) return false;
-  gemv_finish(p, sm, type, L, g.row0 + buf0, rows - buf0, wpg, best_v, best_i);
+  gemv_finish(p, sm, type, L, g.row0 + buf0, rows - buf0, wpg, res, best_v, best_i);
   if (type == 8) {
-    sm.lmv[tid] = best_v;
-    sm.lmi[tid] = best_i;
+    // (max, lowest index) over the threads: warp shuffles, then warp 0
+    float bv = best_v;
+    int bi = best_i;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      sm.lmv[warp] = bv;
+      sm.lmi[warp] = bi;
+    }
     compute_sync();
-    if (tid == 0) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int f = 0; f < kComputeThreads; ++f) {
-        const float v = sm.lmv[f];
-        const int i = sm.lmi[f];
-        if (v > bv || (v == bv && i < bi)) {
-          bv = v;
-          bi = i;
+    if (warp == 0) {
+      bv = lane < kComputeWarps ? sm.lmv[lane] : -INFINITY;
+      bi = lane < kComputeWarps ? sm.lmi[lane] : 0x7fffffff;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
         }
       }
-      if (bi == 0x7fffffff) bi = g.row0;  // all values NaN: keep a valid index
-      p.lm_val[(int)t.idx] = bv;
-      p.lm_idx[(int)t.idx] = bi;
+      if (lane == 0) {
+        if (bi == 0x7fffffff) bi = g.row0;  // all values NaN: keep a valid index
+        p.lm_val[(int)t.idx] = bv;
+        p.lm_idx[(int)t.idx] = bi;
+      }
     }
   }
   return true;
@@ -805,15 +893,27 @@ __device__ __forceinline__ void attn_block(const Params &p, float *pw, float *aw
 // are merged once at the end.
 template <int RP>
 __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
-                                       uint32_t &k, int task_id) {
+                                          uint32_t &k, int task_id, const DepWait &dep_wait) {
   constexpr int NP = 32 / RP;
   const AttnSpan a = attn_span(p, (int)t.idx);
-  if (!a.active) return true;  // the split starts past the new row: nothing to do
+  if (!a.active) return dep_wait();  // the split starts past the new row: nothing to do
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int D = p.D, rep = p.rep, dpl = D >> 5;
   const DevLayer &L = p.layers[t.layer];
   const float *qkv = L.qkv + (size_t)a.b * p.n_qkv + (size_t)a.g * p.grp;
   const float *rope = p.rope + (size_t)a.L * D;  // [D/2][2]
+  // gains and RoPE factors of this lane's dims: independent of the step's
+  // results, so loaded before the wait
+  float gq[4], gk[4], rc[2], rs[2];
+  for (int i = 0; i < dpl; ++i) {
+    gq[i] = bf2f(L.q_norm[lane + 32 * i]);
+    gk[i] = bf2f(L.k_norm[lane + 32 * i]);
+  }
+  for (int i = 0; i < (dpl >> 1); ++i) {
+    rc[i] = rope[2 * (lane + 32 * i)];
+    rs[i] = rope[2 * (lane + 32 * i) + 1];
+  }
+  if (!dep_wait()) return false;
 
   // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
   // holds position L; v is only rounded)
@@ -822,16 +922,14 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     float v[4];
     for (int i = 0; i < dpl; ++i) v[i] = __ldcg(qkv + row * D + lane + 32 * i);
     if (row <= rep) {  // q heads and k
-      const uint16_t *gain = row < rep ? L.q_norm : L.k_norm;
       float ss = 0.f;
       for (int i = 0; i < dpl; ++i) ss = fmaf(v[i], v[i], ss);
       ss = warp_sum(ss);
       const float inv = rsqrtf(ss / (float)D + p.eps);
-      for (int i = 0; i < dpl; ++i) v[i] = v[i] * inv * bf2f(gain[lane + 32 * i]);
+      for (int i = 0; i < dpl; ++i) v[i] = v[i] * inv * (row < rep ? gq[i] : gk[i]);
       const int hp = dpl >> 1;  // dims lane + 32 i pair with lane + 32 (i + hp)
       for (int i = 0; i < hp; ++i) {
-        const int d = lane + 32 * i;
-        const float c = rope[2 * d], s = rope[2 * d + 1];
+        const float c = rc[i], s = rs[i];
         const float x0 = v[i], x1 = v[i + hp];
         v[i] = x0 * c - x1 * s;
         v[i + hp] = x1 * c + x0 * s;
@@ -863,6 +961,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[h][i] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
+  trace_mark(p, sm, 0);
   float *pw = sm.sc + warp * (32 + kMaxRep);
   float *aw = pw + 32;
 
@@ -884,6 +983,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
   if (a.has_new && warp == ((cached + NP - 1) / NP) % kComputeWarps)
     attn_block<RP>(p, pw, aw, sm.knew, sm.vnew, 0, 1, qr, m_run, l_run, o);
 
+  trace_mark(p, sm, 1);
   // merge the warps' states
   const int stride = D + 2;
   float *st_w = sm.ored + (size_t)warp * RP * stride;
@@ -928,46 +1028,61 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
 
 // Online-softmax merge of the splits of one (sequence, kv head):
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
-__device__ void merge_task(const Params &p, const Smem &sm, const DevTask &t) {
+// Online-softmax merge of the splits of one (sequence, kv head):
+//   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
+// No shared memory and no barriers: each warp owns (head, 64 dims) slices and
+// issues a pass of kPass splits' loads at once; passes combine online.
+__device__ bool merge_task(const Params &p, const Smem &sm, const DevTask &t,
+                           const DepWait &dep_wait) {
+  constexpr int kPass = 16;
   const int b = (int)t.idx / p.Hkv, g = (int)t.idx % p.Hkv;
   const DevLayer &L = p.layers[t.layer];
   const int Lb = p.kv_len[b];
   const int ns = min(p.S, Lb / p.chunk + 1);  // splits that hold any position
   const int D = p.D, rep = p.rep;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float *wgt = sm.ored;               // [rep][ns]
-  float *sum_l = sm.ored + rep * ns;  // [rep][ns]
-  const float *part = L.part + (size_t)b * p.Hq * p.S * (D + 2);
-  for (int i = tid; i < rep * ns; i += kComputeThreads) {
-    const int h = i / ns, s = i - h * ns;
-    const float *src = part + ((size_t)(g * rep + h) * p.S + s) * (D + 2);
-    wgt[i] = __ldcg(src + D);
-    sum_l[i] = __ldcg(src + D + 1);
-  }
-  compute_sync();
-  if (warp < rep) {
-    const int h = warp;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, wgt[h * ns + s]);
-    M = warp_max(M);
-    float den = 0.f;
-    for (int s = lane; s < ns; s += 32) {
-      const float w = __expf(wgt[h * ns + s] - M);
-      wgt[h * ns + s] = w;
-      den = fmaf(w, sum_l[h * ns + s], den);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (!dep_wait()) return false;
+  trace_mark(p, sm, 0);
+  const int per_head = D / 64;  // warps per head (64 dims each, 2 per lane)
+  for (int slice = warp; slice < rep * per_head; slice += kComputeWarps) {
+    const int h = slice / per_head;
+    const int d0 = (slice % per_head) * 64 + lane;
+    const float *src = L.part + (((size_t)b * p.Hq + g * rep + h) * p.S) * (D + 2);
+    float M = -INFINITY, den = 0.f, n0 = 0.f, n1 = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += kPass) {
+      float m[kPass], l[kPass], o0[kPass], o1[kPass];
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) {
+        const bool ok = s0 + i < ns;
+        const float *ps = src + (size_t)(s0 + i) * (D + 2);
+        m[i] = ok ? __ldcg(ps + D) : -INFINITY;
+        l[i] = ok ? __ldcg(ps + D + 1) : 0.f;
+        o0[i] = ok ? __ldcg(ps + d0) : 0.f;
+        o1[i] = ok ? __ldcg(ps + d0 + 32) : 0.f;
+      }
+      float Mp = M;
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) Mp = fmaxf(Mp, m[i]);
+      const float r = M == -INFINITY ? 0.f : __expf(M - Mp);
+      den *= r;
+      n0 *= r;
+      n1 *= r;
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) {
+        const float w = m[i] == -INFINITY ? 0.f : __expf(m[i] - Mp);
+        den = fmaf(w, l[i], den);
+        n0 = fmaf(w, o0[i], n0);
+        n1 = fmaf(w, o1[i], n1);
+      }
+      M = Mp;
     }
-    den = warp_sum(den);
-    if (lane == 0) sm.mls[h] = 1.f / den;
+    float *dst = L.att + (size_t)b * p.qdim + (g * rep + h) * D;
+    const float inv = 1.f / den;
+    dst[d0] = n0 * inv;
+    dst[d0 + 32] = n1 * inv;
   }
-  compute_sync();
-  for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
-    const int h = oi / D, d = oi - h * D;
-    const float *src = part + (size_t)(g * rep + h) * p.S * (D + 2) + d;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < ns; ++s) acc = fmaf(wgt[h * ns + s], __ldcg(src + (size_t)s * (D + 2)), acc);
-    L.att[(size_t)b * p.qdim + (g * rep + h) * D + d] = acc * sm.mls[h];
-  }
+  trace_mark(p, sm, 1);
+  return true;
 }
 
 __device__ void embed_task(const Params &p) {
@@ -1051,39 +1166,37 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     for (int n = 0; n < q.count; ++n) {
       const int id = q.first + n * q.stride;
       const DevTask t = p.tasks[id];
-      uint64_t t_wait = 0, t_ready = 0;
-      if (p.trace && tid == 0) t_wait = global_timer();
-      if (p.persistent && t.dep >= 0 && tid == 0) {
-        if (!wait_event(p, t.dep, epoch, id)) sm.ctl[kAbort] = 1;
+      uint64_t t_wait = 0;
+      if (p.trace && tid == 0) {
+        t_wait = global_timer();
+        sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = 0;
       }
-      compute_sync();
-      if (sm.ctl[kAbort]) break;
-      if (p.trace && tid == 0) t_ready = global_timer();
+      const DepWait dw{p, sm, t.dep, epoch, id};
       bool ok = true;
       switch (t.type) {
-        case 1: embed_task(p); break;
+        case 1: ok = dw(); if (ok) embed_task(p); break;
         case 2: case 5: case 6: case 7: case 8: {
           const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
           const int nch = K >> 3;
           const int cpt = nch <= kComputeThreads ? 1 : (nch + kComputeThreads - 1) / kComputeThreads;
           const int rps = t.type == 2 ? p.rps_qkv : t.type == 5 ? p.rps_o : t.type == 6 ? p.rps_gu
                         : t.type == 7 ? p.rps_down : p.rps_lm;
-          if (cpt == 1 && rps >= 8) ok = gemv_task<1, 8>(p, sm, t, k, id);
-          else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id);
-          else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id);
-          else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id);
-          else ok = gemv_task<8, 8>(p, sm, t, k, id);
+          if (cpt == 1 && rps >= 8) ok = gemv_task<1, 8>(p, sm, t, k, id, dw);
+          else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id, dw);
+          else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id, dw);
+          else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id, dw);
+          else ok = gemv_task<8, 8>(p, sm, t, k, id, dw);
           break;
         }
         case 3:
-          ok = rp == 1 ? attn_task<1>(p, sm, t, k, id)
-             : rp == 2 ? attn_task<2>(p, sm, t, k, id)
-             : rp == 4 ? attn_task<4>(p, sm, t, k, id)
-                       : attn_task<8>(p, sm, t, k, id);
+          ok = rp == 1 ? attn_task<1>(p, sm, t, k, id, dw)
+             : rp == 2 ? attn_task<2>(p, sm, t, k, id, dw)
+             : rp == 4 ? attn_task<4>(p, sm, t, k, id, dw)
+                       : attn_task<8>(p, sm, t, k, id, dw);
           break;
-        case 4: merge_task(p, sm, t); break;
-        case 9: argmax_task(p, epoch); break;
-        default: break;  // empty task
+        case 4: ok = merge_task(p, sm, t, dw); break;
+        case 9: ok = dw(); if (ok) argmax_task(p, epoch); break;
+        default: ok = dw(); break;  // empty task
       }
       if (!ok) break;
       compute_sync();
@@ -1094,11 +1207,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
         if (p.trace) {
           uint32_t smid;
           asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-          unsigned long long *tr = p.trace + 4 * (size_t)id;
+          unsigned long long *tr = p.trace + 8 * (size_t)id;
           tr[0] = t_wait;
-          tr[1] = t_ready;
+          tr[1] = sm.tmark[2];
           tr[2] = global_timer();
           tr[3] = ((unsigned long long)smid << 32) | blockIdx.x;
+          tr[4] = sm.tmark[0];
+          tr[5] = sm.tmark[1];
         }
       }
     }
