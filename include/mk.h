@@ -58,8 +58,9 @@ enum {
   MK_TASK_GENERIC = 0, /* task of a graph built by mk_graph_from_edges */
   MK_TASK_EMBED = 1,   /* x0[b] = float(E[token_b])                                  */
   MK_TASK_QKV = 2,     /* RMSNorm prologue, q/k/v rows of one kv-group-aligned tile    */
-  MK_TASK_ATTN = 3,    /* one (sequence, kv head, KV split) of decode attention        */
-  MK_TASK_MERGE = 4,   /* online-softmax merge of the splits of one (sequence, kv head) */
+  MK_TASK_ATTN = 3,    /* one (sequence, kv head, KV split) of decode attention; the   */
+                       /* split that finishes last merges the splits (online softmax)  */
+  MK_TASK_MERGE = 4,   /* reserved (decode graphs merge inside the last ATTN split)    */
   MK_TASK_OPROJ = 5,   /* O projection tile, residual add epilogue                     */
   MK_TASK_GATEUP = 6,  /* RMSNorm prologue, gate/up tile, SiLU(g)*u epilogue           */
   MK_TASK_DOWN = 7,    /* down projection tile, residual add epilogue                  */

@@ -19,7 +19,9 @@
 //               (else n = G), so no task spans two kv groups.
 //               ATTN: S' = ceil(apw * W / (B * Hkv)),
 //               chunk = max(min_chunk, align_up(ceil(Lcap / S'), 64)),
-//               S = ceil(Lcap / chunk); a MERGE op exists iff S > 1.
+//               S = ceil(Lcap / chunk).  Every split writes its partial
+//               and may write the merged head block: the split of (b, g) that
+//               finishes last merges the partials (no separate merge op).
 //   regions     each task reads and writes rectangles of named buffers;
 //               activations are single-assignment (one buffer per layer/op).
 //   raw events  task a -> task c when op(a) < op(c) and a region of a and a
@@ -452,21 +454,13 @@ Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_
         for (int s = 0; s < S; ++s) {
           std::vector<Rect> regs = {R(B_QKV(l), b, b + 1, g * G, (g + 1) * G),
                                     R(B_KVLEN, b, b + 1, 0, 1)};
-          if (S > 1)
-            regs.push_back(Wr(B_PART(l), b, b + 1, g * S + s, g * S + s + 1));
-          else
-            regs.push_back(Wr(B_ATT(l), b, b + 1, g * rep * D, (g + 1) * rep * D));
+          // every split may produce the merged head block: the split that
+          // finishes last merges all partials of (b, g)
+          if (S > 1) regs.push_back(Wr(B_PART(l), b, b + 1, g * S + s, g * S + s + 1));
+          regs.push_back(Wr(B_ATT(l), b, b + 1, g * rep * D, (g + 1) * rep * D));
           add(T_ATTN, l, (b * Hkv + g) * S + s, regs);
         }
     ++op;
-    if (S > 1) {
-      for (int b = 0; b < B; ++b)
-        for (int g = 0; g < Hkv; ++g)
-          add(T_MERGE, l, b * Hkv + g,
-              {R(B_PART(l), b, b + 1, g * S, (g + 1) * S),
-               Wr(B_ATT(l), b, b + 1, g * rep * D, (g + 1) * rep * D)});
-      ++op;
-    }
     for (int j = 0; j * L.o_rows < H; ++j) {
       int c0 = j * L.o_rows, c1 = std::min(H, c0 + L.o_rows);
       add(T_OPROJ, l, j, {R(B_ATT(l), 0, B, 0, qd), R(B_X(l), 0, B, c0, c1),

@@ -94,7 +94,7 @@ std::string check_gpu_shape(const mk_model_config &c) {
   if (rep > mk::kMaxRep) return "at most 8 q heads per kv head";
   if (c.hidden % 256 || c.ffn % 256 || qd % 256)
     return "hidden, ffn and n_q_heads*head_dim must be multiples of 256";
-  if (std::max(std::max(c.hidden, c.ffn), qd) > mk::kMaxChunks * 8 * mk::kComputeThreads)
+  if (std::max(std::max(c.hidden, c.ffn), qd) > mk::kMaxCpt * 8 * mk::kComputeThreads)
     return "projection input width above 16384";
   if (c.batch > 1)
     return "batch > 1 needs the tensor-core projection path, which this build does not have";
@@ -250,6 +250,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   const size_t o_tasks = take(sizeof(mk::DevTask) * G.type.size());
   const size_t o_events = take(sizeof(mk::DevEvent) * std::max<size_t>(1, G.ev_count.size()));
   const size_t o_counters = take(4 * std::max<size_t>(1, G.ev_count.size()));
+  const size_t o_arrivals = take(4 * (size_t)c.n_layers * c.batch * c.n_kv_heads);
   const size_t o_epoch = take(4);
   const size_t o_status = take(16);
   const size_t o_layers = take(sizeof(mk::DevLayer) * Ly);
@@ -342,6 +343,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.tasks = reinterpret_cast<const mk::DevTask *>(base + o_tasks);
   p.events = reinterpret_cast<const mk::DevEvent *>(base + o_events);
   p.counters = reinterpret_cast<uint32_t *>(base + o_counters);
+  p.arrivals = reinterpret_cast<uint32_t *>(base + o_arrivals);
   p.epoch = reinterpret_cast<uint32_t *>(base + o_epoch);
   p.status = reinterpret_cast<int32_t *>(base + o_status);
   p.n_tasks = (int)tasks.size();
@@ -378,11 +380,6 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.l2_prefetch_bytes = t.l2_prefetch_bytes;
   p.timeout_ns = (unsigned long long)t.wait_timeout_us * 1000ull;
   p.trace = nullptr;
-  if (S > 1 && 2 * rep * S > mk::kComputeWarps * rep_p * (D + 2)) {
-    mk_destroy(h);
-    return fail(nullptr, MK_ERR_ARG, "too many attention splits for the merge scratch; "
-                                     "raise attn_min_chunk");
-  }
   *out = h;
   return MK_OK;
 }
@@ -568,6 +565,9 @@ mk_status mk_reset(mk_handle *h, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t ne = std::max<size_t>(1, h->graph.ev_count.size());
   cudaError_t e = cudaMemsetAsync(h->base.counters, 0, 4 * ne, st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(h->base.arrivals, 0,
+                        4 * (size_t)h->cfg.n_layers * h->cfg.batch * h->cfg.n_kv_heads, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->base.epoch, 0, 4, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->base.status, 0, 16, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "reset");

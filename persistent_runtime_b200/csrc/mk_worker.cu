@@ -87,6 +87,13 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -116,18 +123,6 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-__device__ __forceinline__ float dot8(const uint4 w, const float *x) {
-  float a = bf_lo(w.x) * x[0];
-  a = fmaf(bf_hi(w.x), x[1], a);
-  a = fmaf(bf_lo(w.y), x[2], a);
-  a = fmaf(bf_hi(w.y), x[3], a);
-  a = fmaf(bf_lo(w.z), x[4], a);
-  a = fmaf(bf_hi(w.z), x[5], a);
-  a = fmaf(bf_lo(w.w), x[6], a);
-  a = fmaf(bf_hi(w.w), x[7], a);
-  return a;
 }
 
 // (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32x2 FMA (sm_100).
@@ -190,7 +185,7 @@ __device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 // ---------------------------------------------------------------------------
 // Shared memory layout (identical computation on host: see smem_bytes()).
 // ---------------------------------------------------------------------------
-enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kCtlWords = 16 };
+enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kCtlWords = 16 };
 
 struct Smem {
   uint8_t *ring;
@@ -200,8 +195,8 @@ struct Smem {
   // GEMV scratch
   float *red;   // [kRedRows][kComputeWarps] warp partial sums of tile rows
   float *ss;    // [kComputeWarps]
-  float *lmv;   // [kComputeThreads] partial argmax values (LM head)
-  int *lmi;     // [kComputeThreads] partial argmax indices
+  float *lmv;   // [kComputeWarps] partial argmax values (LM head)
+  int *lmi;     // [kComputeWarps] partial argmax indices
   // attention scratch
   float *q;     // [kMaxRep][kMaxHeadDim]
   uint16_t *knew, *vnew;  // [kMaxHeadDim] bf16
@@ -236,9 +231,9 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   o.ss = g;
   g += 4 * kComputeWarps;
   o.lmv = g;
-  g += 4 * kComputeThreads;
+  g += 4 * kComputeWarps;
   o.lmi = g;
-  g += 4 * kComputeThreads;
+  g += 4 * kComputeWarps;
   // attention scratch (shares the same bytes: a CTA runs one task at a time)
   size_t a = p;
   o.q = a;
@@ -253,7 +248,7 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   a += 4 * 3 * kMaxRep;
   a = align_to(a, 16);
   o.ored = a;  // per warp and head: o[D], running max, running sum
-  a += 4 * (size_t)kComputeWarps * rep_p * (head_dim + 2);
+  a += 4 * (size_t)kStateSlots * rep_p * (head_dim + 2);
   o.total = align_to(g > a ? g : a, 128);
   return o;
 }
@@ -357,46 +352,37 @@ __device__ __forceinline__ size_t kv_row(const Params &p, int layer, int b, int 
   return ((((size_t)layer * p.B + b) * p.Hkv + g) * p.Lcap + row) * p.D;
 }
 
-// Number of ring stages a task consumes.
-__device__ __forceinline__ int task_stages(const Params &p, const DevTask &t) {
-  int type = t.type;
-  if (type == 2 || (type >= 5 && type <= 8)) {
-    Gemv g = gemv_of(p, type, t.layer, (int)t.idx);
-    return (g.row1 - g.row0 + g.rps - 1) / g.rps;
-  }
-  if (type == 3) {
-    AttnSpan a = attn_span(p, (int)t.idx);
-    int n = a.cached_end - a.p0;
-    return n > 0 ? (n + p.pps - 1) / p.pps : 0;
-  }
-  return 0;
-}
-
-// Source ranges of stage `st` of a task: up to two contiguous byte ranges.
-struct Copy {
-  const void *src0, *src1;
-  uint32_t bytes0, bytes1;
+// Everything the producer needs to stream one task, computed once per task so
+// that issuing a stage is pure address arithmetic (no dependent loads).
+struct Stream {
+  const uint8_t *src0, *src1;  // stage 0 sources (src1: V rows of attention, else null)
+  uint32_t bytes, last_bytes;  // bytes of a full / of the last stage (per source)
+  uint32_t stride;             // bytes between consecutive stages of one source
+  int nst;                     // stages
 };
 
-__device__ __forceinline__ Copy stage_copy(const Params &p, const DevTask &t, int st) {
-  Copy c{nullptr, nullptr, 0u, 0u};
-  int type = t.type;
+__device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t) {
+  Stream s{nullptr, nullptr, 0u, 0u, 0u, 0};
+  const int type = t.type;
   if (type == 3) {
-    AttnSpan a = attn_span(p, (int)t.idx);
-    int r0 = a.p0 + st * p.pps;
-    int n = min(p.pps, a.cached_end - r0);
-    size_t off = kv_row(p, t.layer, a.b, a.g, r0);
-    c.src0 = p.k_cache + off;
-    c.src1 = p.v_cache + off;
-    c.bytes0 = c.bytes1 = (uint32_t)(n * p.D * 2);
-  } else {
-    Gemv g = gemv_of(p, type, t.layer, (int)t.idx);
-    int r0 = g.row0 + st * g.rps;
-    int n = min(g.rps, g.row1 - r0);
-    c.src0 = g.w + (size_t)r0 * g.K;
-    c.bytes0 = (uint32_t)((size_t)n * g.K * 2);
+    const AttnSpan a = attn_span(p, (int)t.idx);
+    const int n = a.cached_end - a.p0;
+    if (n <= 0) return s;
+    s.nst = (n + p.pps - 1) / p.pps;
+    const size_t off = kv_row(p, t.layer, a.b, a.g, a.p0);
+    s.src0 = reinterpret_cast<const uint8_t *>(p.k_cache + off);
+    s.src1 = reinterpret_cast<const uint8_t *>(p.v_cache + off);
+    s.stride = s.bytes = (uint32_t)(p.pps * p.D * 2);
+    s.last_bytes = (uint32_t)((n - (s.nst - 1) * p.pps) * p.D * 2);
+  } else if (type == 2 || (type >= 5 && type <= 8)) {
+    const Gemv g = gemv_of(p, type, t.layer, (int)t.idx);
+    const int rows = g.row1 - g.row0;
+    s.nst = (rows + g.rps - 1) / g.rps;
+    s.src0 = reinterpret_cast<const uint8_t *>(g.w + (size_t)g.row0 * g.K);
+    s.stride = s.bytes = (uint32_t)((size_t)g.rps * g.K * 2);
+    s.last_bytes = (uint32_t)((size_t)(rows - (s.nst - 1) * g.rps) * g.K * 2);
   }
-  return c;
+  return s;
 }
 
 // ---------------------------------------------------------------------------
@@ -410,26 +396,27 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const int NS = p.ring_stages;
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
-  // L2 prefetch cursor (stage index pf_k in the worker's stream of stages,
-  // across task boundaries).  While the producer is blocked on a full ring it
-  // prefetches the next stages into L2, up to l2_prefetch_bytes ahead of the
-  // ring, so HBM keeps streaming while the compute warps wait on an event.
+  // L2 prefetch cursor (task pf_n, stage pf_st, global stage index pf_k) in
+  // the worker's stream of stages, across task boundaries.  While the
+  // producer is blocked on a full ring it prefetches the next stages into L2,
+  // up to l2_prefetch_bytes ahead of the ring.
   const long long dist = p.l2_prefetch_bytes;
-  int pf_n = 0, pf_st = 0, pf_ns = -1;
+  int pf_n = 0, pf_st = 0;
+  Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1};
   uint32_t pf_k = 0;
   long long ahead = 0;
   for (int n = 0; n < q.count; ++n) {
-    const DevTask t = p.tasks[q.first + n * q.stride];
-    const int ns = task_stages(p, t);
-    for (int st = 0; st < ns; ++st) {
+    const Stream ts = task_stream(p, p.tasks[q.first + n * q.stride]);
+    for (int st = 0; st < ts.nst; ++st) {
+      const uint32_t nb = st == ts.nst - 1 ? ts.last_bytes : ts.bytes;
       if (dist > 0) {
         // stages before k were issued without a prefetch: move the cursor on
         while (pf_k < k && pf_n < q.count) {
-          if (pf_ns < 0) pf_ns = task_stages(p, p.tasks[q.first + pf_n * q.stride]);
-          if (pf_st >= pf_ns) {
+          if (pfs.nst < 0) pfs = task_stream(p, p.tasks[q.first + pf_n * q.stride]);
+          if (pf_st >= pfs.nst) {
             ++pf_n;
             pf_st = 0;
-            pf_ns = -1;
+            pfs.nst = -1;
             continue;
           }
           ++pf_st;
@@ -447,17 +434,17 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
           if (sm.ctl[kAbort]) goto out;
           ++spins;
           if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count) {
-            const DevTask pt = p.tasks[q.first + pf_n * q.stride];
-            if (pf_ns < 0) pf_ns = task_stages(p, pt);
-            if (pf_st >= pf_ns) {
+            if (pfs.nst < 0) pfs = task_stream(p, p.tasks[q.first + pf_n * q.stride]);
+            if (pf_st >= pfs.nst) {
               ++pf_n;
               pf_st = 0;
-              pf_ns = -1;
+              pfs.nst = -1;
             } else {
-              const Copy pc = stage_copy(p, pt, pf_st);
-              prefetch_l2(pc.src0, pc.bytes0);
-              if (pc.bytes1) prefetch_l2(pc.src1, pc.bytes1);
-              ahead += pc.bytes0 + pc.bytes1;
+              const uint32_t pb = pf_st == pfs.nst - 1 ? pfs.last_bytes : pfs.bytes;
+              prefetch_l2(pfs.src0 + (size_t)pf_st * pfs.stride, pb);
+              if (pfs.src1) prefetch_l2(pfs.src1 + (size_t)pf_st * pfs.stride, pb);
+              ahead += pfs.src1 ? 2 * pb : pb;
+              if (p.trace) sm.tmark[3] += pfs.src1 ? 2 * pb : pb;
               ++pf_st;
               ++pf_k;
             }
@@ -472,12 +459,11 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
           }
         }
       }
-      const Copy c = stage_copy(p, t, st);
       uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes;
-      mbar_arrive_expect_tx(&sm.full[slot], c.bytes0 + c.bytes1);
-      bulk_g2s(dst, c.src0, c.bytes0, &sm.full[slot]);
-      if (c.bytes1) bulk_g2s(dst + p.stage_bytes / 2, c.src1, c.bytes1, &sm.full[slot]);
-      if (dist > 0 && pf_k > k) ahead -= c.bytes0 + c.bytes1;  // stage k was prefetched
+      mbar_arrive_expect_tx(&sm.full[slot], ts.src1 ? 2 * nb : nb);
+      bulk_g2s(dst, ts.src0 + (size_t)st * ts.stride, nb, &sm.full[slot]);
+      if (ts.src1) bulk_g2s(dst + p.stage_bytes / 2, ts.src1 + (size_t)st * ts.stride, nb, &sm.full[slot]);
+      if (dist > 0 && pf_k > k) ahead -= ts.src1 ? 2 * nb : nb;  // stage k was prefetched
       ++k;
     }
   }
@@ -707,27 +693,17 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
           for (int i = 0; i < NR; ++i)
 #pragma unroll
             for (int a = 0; a < AS; ++a) acc[i][a][0] = acc[i][a][1] = 0.f;
-          if (nr == NR) {
+          // a partial last batch still reads NR rows: rb + NR <= rps keeps them
+          // inside the slot, and rows >= nr (stale data) are never stored
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) {
-              const int c = li + j * tpg;
-              if (c < nch) {
-                uint4 w[NR];
+          for (int j = 0; j < CPT; ++j) {
+            const int c = li + j * tpg;
+            if (c < nch) {
+              uint4 w[NR];
 #pragma unroll
-                for (int i = 0; i < NR; ++i) w[i] = wr[i * row16 + c];
+              for (int i = 0; i < NR; ++i) w[i] = wr[i * row16 + c];
 #pragma unroll
-                for (int i = 0; i < NR; ++i) dot8_acc(w[i], x[j], acc[i][j % AS]);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < CPT; ++j) {
-              const int c = li + j * tpg;
-              if (c < nch) {
-#pragma unroll
-                for (int i = 0; i < NR; ++i)
-                  if (i < nr) dot8_acc(wr[i * row16 + c], x[j], acc[i][j % AS]);
-              }
+              for (int i = 0; i < NR; ++i) dot8_acc(w[i], x[j], acc[i][j % AS]);
             }
           }
           float v8[8];
@@ -796,6 +772,71 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 // ---------------------------------------------------------------------------
 // Attention: one (sequence b, kv head g, split s).
 // ---------------------------------------------------------------------------
+// Split-KV attention: after writing its partial, a split arrives on the
+// (layer, sequence, kv head) counter; the split that arrives last merges all
+// partials (online softmax:  M = max_s m_s,  w_s = exp(m_s - M),
+// o = sum_s w_s o_s / sum_s w_s l_s) into the head block of att and resets the
+// counter, so no separate merge task (and no extra event) is needed.  The
+// acquire-release atomic orders every split's partial before the merge reads.
+// Each warp owns (head, 64 dims) slices and issues a pass of kPass splits'
+// loads at once; passes combine online.
+__device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Smem &sm, int layer,
+                                                      int b, int g) {
+  constexpr int kPass = 16;
+  compute_sync();  // every thread's partial stores precede the arrival
+  uint32_t *ctr = p.arrivals + ((size_t)layer * p.B + b) * p.Hkv + g;
+  if (threadIdx.x == 0) {
+    const uint32_t old = atom_acq_rel_add(ctr, 1u);
+    sm.ctl[kLast] = old + 1u == (uint32_t)p.S;
+  }
+  compute_sync();
+  if (!sm.ctl[kLast]) return true;
+  if (threadIdx.x == 0) *ctr = 0u;  // every split of this step has arrived
+  const DevLayer &L = p.layers[layer];
+  const int ns = min(p.S, p.kv_len[b] / p.chunk + 1);  // splits that hold any position
+  const int D = p.D, rep = p.rep;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_head = D / 64;  // warps per head (64 dims each, 2 per lane)
+  for (int slice = warp; slice < rep * per_head; slice += kComputeWarps) {
+    const int h = slice / per_head;
+    const int d0 = (slice % per_head) * 64 + lane;
+    const float *src = L.part + (((size_t)b * p.Hq + g * rep + h) * p.S) * (D + 2);
+    float M = -INFINITY, den = 0.f, n0 = 0.f, n1 = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += kPass) {
+      float m[kPass], l[kPass], o0[kPass], o1[kPass];
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) {
+        const bool ok = s0 + i < ns;
+        const float *ps = src + (size_t)(s0 + i) * (D + 2);
+        m[i] = ok ? __ldcg(ps + D) : -INFINITY;
+        l[i] = ok ? __ldcg(ps + D + 1) : 0.f;
+        o0[i] = ok ? __ldcg(ps + d0) : 0.f;
+        o1[i] = ok ? __ldcg(ps + d0 + 32) : 0.f;
+      }
+      float Mp = M;
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) Mp = fmaxf(Mp, m[i]);
+      const float r = M == -INFINITY ? 0.f : __expf(M - Mp);
+      den *= r;
+      n0 *= r;
+      n1 *= r;
+#pragma unroll
+      for (int i = 0; i < kPass; ++i) {
+        const float w = m[i] == -INFINITY ? 0.f : __expf(m[i] - Mp);
+        den = fmaf(w, l[i], den);
+        n0 = fmaf(w, o0[i], n0);
+        n1 = fmaf(w, o1[i], n1);
+      }
+      M = Mp;
+    }
+    float *dst = L.att + (size_t)b * p.qdim + (g * rep + h) * D;
+    const float inv = 1.f / den;
+    dst[d0] = n0 * inv;
+    dst[d0 + 32] = n1 * inv;
+  }
+  return true;
+}
+
 // One block of up to NP = 32 / RP positions for one warp: scores, online
 // softmax update of the warp's running state, and PV.  RP = q heads per kv head
 // rounded up to a power of two (heads >= rep are padding).  Lane l covers dims
@@ -896,7 +937,10 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
                                           uint32_t &k, int task_id, const DepWait &dep_wait) {
   constexpr int NP = 32 / RP;
   const AttnSpan a = attn_span(p, (int)t.idx);
-  if (!a.active) return dep_wait();  // the split starts past the new row: nothing to do
+  if (!a.active) {  // the split starts past the new row: it only arrives
+    if (!dep_wait()) return false;
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int D = p.D, rep = p.rep, dpl = D >> 5;
   const DevLayer &L = p.layers[t.layer];
@@ -984,27 +1028,64 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     attn_block<RP>(p, pw, aw, sm.knew, sm.vnew, 0, 1, qr, m_run, l_run, o);
 
   trace_mark(p, sm, 1);
-  // merge the warps' states
+  // merge the warps' states: warps >= kStateSlots first fold into warp
+  // (w - kStateSlots), then the kStateSlots states are combined per output
   const int stride = D + 2;
-  float *st_w = sm.ored + (size_t)warp * RP * stride;
+  if (kComputeWarps > kStateSlots) {
+    if (warp >= kStateSlots) {
+      float *st_w = sm.ored + (size_t)(warp - kStateSlots) * RP * stride;
 #pragma unroll
-  for (int h = 0; h < RP; ++h)
+      for (int h = 0; h < RP; ++h)
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (i < dpl) st_w[h * stride + dpl * lane + i] = o[h][i];
-  if (lane % NP == 0) {
-    const int h = lane / NP;
-    st_w[h * stride + D] = m_run;
-    st_w[h * stride + D + 1] = l_run;
+        for (int i = 0; i < 4; ++i)
+          if (i < dpl) st_w[h * stride + dpl * lane + i] = o[h][i];
+      if (lane % NP == 0) {
+        st_w[(lane / NP) * stride + D] = m_run;
+        st_w[(lane / NP) * stride + D + 1] = l_run;
+      }
+    }
+    compute_sync();
+    if (warp < kStateSlots) {
+      const float *st_p = sm.ored + (size_t)warp * RP * stride;
+#pragma unroll
+      for (int h = 0; h < RP; ++h) {
+        const float m_me = __shfl_sync(0xffffffffu, m_run, h * NP);
+        const float m_pa = st_p[h * stride + D];
+        const float M = fmaxf(m_me, m_pa);
+        const float a = m_me == -INFINITY ? 0.f : __expf(m_me - M);
+        const float b = m_pa == -INFINITY ? 0.f : __expf(m_pa - M);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < dpl) o[h][i] = a * o[h][i] + b * st_p[h * stride + dpl * lane + i];
+        if (lane / NP == h) {
+          l_run = a * l_run + b * st_p[h * stride + D + 1];
+          m_run = M;
+        }
+      }
+    }
+    compute_sync();
+  }
+  if (warp < kStateSlots) {
+    float *st_w = sm.ored + (size_t)warp * RP * stride;
+#pragma unroll
+    for (int h = 0; h < RP; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (i < dpl) st_w[h * stride + dpl * lane + i] = o[h][i];
+    if (lane % NP == 0) {
+      const int h = lane / NP;
+      st_w[h * stride + D] = m_run;
+      st_w[h * stride + D + 1] = l_run;
+    }
   }
   compute_sync();
   if (sm.ctl[kAbort]) return false;
   for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
     const int h = oi / D, d = oi - h * D;
     float M = -INFINITY;
-    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, sm.ored[((size_t)w * RP + h) * stride + D]);
+    for (int w = 0; w < kStateSlots; ++w) M = fmaxf(M, sm.ored[((size_t)w * RP + h) * stride + D]);
     float num = 0.f, den = 0.f;
-    for (int w = 0; w < kComputeWarps; ++w) {
+    for (int w = 0; w < kStateSlots; ++w) {
       const float *sw = sm.ored + ((size_t)w * RP + h) * stride;
       const float mw = sw[D];
       const float e = mw == -INFINITY ? 0.f : __expf(mw - M);
@@ -1023,68 +1104,12 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
       }
     }
   }
-  return true;
+  if (p.S == 1) return true;
+  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
 }
 
 // Online-softmax merge of the splits of one (sequence, kv head):
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
-// Online-softmax merge of the splits of one (sequence, kv head):
-//   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
-// No shared memory and no barriers: each warp owns (head, 64 dims) slices and
-// issues a pass of kPass splits' loads at once; passes combine online.
-__device__ bool merge_task(const Params &p, const Smem &sm, const DevTask &t,
-                           const DepWait &dep_wait) {
-  constexpr int kPass = 16;
-  const int b = (int)t.idx / p.Hkv, g = (int)t.idx % p.Hkv;
-  const DevLayer &L = p.layers[t.layer];
-  const int Lb = p.kv_len[b];
-  const int ns = min(p.S, Lb / p.chunk + 1);  // splits that hold any position
-  const int D = p.D, rep = p.rep;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (!dep_wait()) return false;
-  trace_mark(p, sm, 0);
-  const int per_head = D / 64;  // warps per head (64 dims each, 2 per lane)
-  for (int slice = warp; slice < rep * per_head; slice += kComputeWarps) {
-    const int h = slice / per_head;
-    const int d0 = (slice % per_head) * 64 + lane;
-    const float *src = L.part + (((size_t)b * p.Hq + g * rep + h) * p.S) * (D + 2);
-    float M = -INFINITY, den = 0.f, n0 = 0.f, n1 = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += kPass) {
-      float m[kPass], l[kPass], o0[kPass], o1[kPass];
-#pragma unroll
-      for (int i = 0; i < kPass; ++i) {
-        const bool ok = s0 + i < ns;
-        const float *ps = src + (size_t)(s0 + i) * (D + 2);
-        m[i] = ok ? __ldcg(ps + D) : -INFINITY;
-        l[i] = ok ? __ldcg(ps + D + 1) : 0.f;
-        o0[i] = ok ? __ldcg(ps + d0) : 0.f;
-        o1[i] = ok ? __ldcg(ps + d0 + 32) : 0.f;
-      }
-      float Mp = M;
-#pragma unroll
-      for (int i = 0; i < kPass; ++i) Mp = fmaxf(Mp, m[i]);
-      const float r = M == -INFINITY ? 0.f : __expf(M - Mp);
-      den *= r;
-      n0 *= r;
-      n1 *= r;
-#pragma unroll
-      for (int i = 0; i < kPass; ++i) {
-        const float w = m[i] == -INFINITY ? 0.f : __expf(m[i] - Mp);
-        den = fmaf(w, l[i], den);
-        n0 = fmaf(w, o0[i], n0);
-        n1 = fmaf(w, o1[i], n1);
-      }
-      M = Mp;
-    }
-    float *dst = L.att + (size_t)b * p.qdim + (g * rep + h) * D;
-    const float inv = 1.f / den;
-    dst[d0] = n0 * inv;
-    dst[d0 + 32] = n1 * inv;
-  }
-  trace_mark(p, sm, 1);
-  return true;
-}
-
 __device__ void embed_task(const Params &p) {
   for (int b = 0; b < p.B; ++b) {
     const uint16_t *e = p.embed + (size_t)p.tokens_in[b] * p.H;
@@ -1152,6 +1177,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     sm.ctl[kEpoch] = p.persistent ? (int)(*(volatile uint32_t *)p.epoch + 1u) : 0;
     sm.ctl[kConsumed] = 0;
     sm.ctl[kIssued] = 0;
+    sm.tmark[3] = 0;
   }
   __syncthreads();
   if (sm.ctl[kAbort]) return;  // nothing issued yet
@@ -1169,7 +1195,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       uint64_t t_wait = 0;
       if (p.trace && tid == 0) {
         t_wait = global_timer();
-        sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = 0;
+        sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = 0;  // tmark[3] accumulates
       }
       const DepWait dw{p, sm, t.dep, epoch, id};
       bool ok = true;
@@ -1185,16 +1211,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id, dw);
           else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id, dw);
           else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id, dw);
-          else ok = gemv_task<8, 8>(p, sm, t, k, id, dw);
+          else ok = gemv_task<kMaxCpt, 8>(p, sm, t, k, id, dw);
           break;
         }
         case 3:
-          ok = rp == 1 ? attn_task<1>(p, sm, t, k, id, dw)
-             : rp == 2 ? attn_task<2>(p, sm, t, k, id, dw)
+          ok = rp <= 2 ? attn_task<2>(p, sm, t, k, id, dw)
              : rp == 4 ? attn_task<4>(p, sm, t, k, id, dw)
                        : attn_task<8>(p, sm, t, k, id, dw);
           break;
-        case 4: ok = merge_task(p, sm, t, dw); break;
         case 9: ok = dw(); if (ok) argmax_task(p, epoch); break;
         default: ok = dw(); break;  // empty task
       }
@@ -1214,6 +1238,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           tr[3] = ((unsigned long long)smid << 32) | blockIdx.x;
           tr[4] = sm.tmark[0];
           tr[5] = sm.tmark[1];
+          tr[6] = sm.tmark[3];  // bytes this worker has prefetched into L2 so far
         }
       }
     }

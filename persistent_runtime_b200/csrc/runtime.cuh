@@ -8,9 +8,11 @@
 namespace mk {
 
 constexpr int kComputeWarps = 8;
+constexpr int kStateSlots = kComputeWarps < 8 ? kComputeWarps : 8;  // attention warp states in smem
 constexpr int kComputeThreads = kComputeWarps * 32;  // threads that run task bodies
 constexpr int kThreads = kComputeThreads + 32;       // + one producer (TMA) warp
-constexpr int kMaxChunks = 8;          // 16-byte weight chunks per thread and row: K <= 16384
+constexpr int kMaxChunks = 8;          // 16-byte weight chunks per thread and row
+constexpr int kMaxCpt = (16384 / 8 + kComputeThreads - 1) / kComputeThreads;  // K <= 16384
 constexpr int kMaxRowsPerStage = 64;   // GEMV rows in one ring stage
 constexpr int kRedRows = 256;          // GEMV rows whose warp partials shared memory holds
 constexpr int kMaxRep = 8;             // q heads per kv head
@@ -56,6 +58,7 @@ struct Params {
   const DevTask *tasks;
   const DevEvent *events;
   uint32_t *counters;  // one per event, monotone: count * epoch after each step
+  uint32_t *arrivals;  // per (layer, sequence, kv head): attention splits finished this step
   uint32_t *epoch;     // steps completed by the persistent kernel
   int32_t *status;     // 4 words, see DeviceStatus
   int n_tasks;

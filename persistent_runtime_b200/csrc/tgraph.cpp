@@ -140,21 +140,11 @@ std::string lower(const ModelShape &m, const GraphTuning &t, Lowering *L) {
           int id = task(kAttn, l, (b * m.n_kv_heads + g) * S + s);
           acc(id, lbuf(l, 0), b, b + 1, g * grp, (g + 1) * grp, false);
           acc(id, kKvLen, b, b + 1, 0, 1, false);
-          if (S > 1)
-            acc(id, lbuf(l, 1), b, b + 1, g * S + s, g * S + s + 1, true);
-          else
-            acc(id, lbuf(l, 2), b, b + 1, g * rep * m.head_dim, (g + 1) * rep * m.head_dim,
-                true);
-        }
-    if (S > 1) {
-      new_op();
-      for (int b = 0; b < B; ++b)
-        for (int g = 0; g < m.n_kv_heads; ++g) {
-          int id = task(kMerge, l, b * m.n_kv_heads + g);
-          acc(id, lbuf(l, 1), b, b + 1, g * S, (g + 1) * S, false);
+          // the split of (b, g) that finishes last merges the partials of all
+          // splits, so every split declares the merged head block as written
+          if (S > 1) acc(id, lbuf(l, 1), b, b + 1, g * S + s, g * S + s + 1, true);
           acc(id, lbuf(l, 2), b, b + 1, g * rep * m.head_dim, (g + 1) * rep * m.head_dim, true);
         }
-    }
     new_op();
     for (int j = 0; j < T.n_o; ++j) {
       int c0 = j * T.o_rows, c1 = std::min(m.hidden, c0 + T.o_rows);

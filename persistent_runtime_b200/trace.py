@@ -59,7 +59,11 @@ def summarize(trace: np.ndarray, graph) -> dict:
         sel = ops == o
         op_spans.append((int(o), (int(r[sel].min()) - origin) / 1e3,
                          (int(e[sel].max()) - origin) / 1e3))
-    return {"span_us": span, "workers": n_workers,
+    pf = np.asarray(trace, dtype=np.uint64).reshape(-1, WORDS)[:, 6].astype(np.int64)
+    pf_total = 0
+    for w in np.unique(worker[ran]):
+        pf_total += int(pf[ran & (worker == w)].max())
+    return {"span_us": span, "workers": n_workers, "l2_prefetch_bytes_total": pf_total,
             "event_wait_frac": float(wait.sum() / (n_workers * span)),
             "busy_frac": float(body.sum() / (n_workers * span)),
             "per_type": per_type, "op_spans": op_spans}

@@ -163,12 +163,11 @@ def closed_form_counts(w, kv_capacity, W, col_align=16, apw=4, min_chunk=64):
     chunk = max(min_chunk, aup(cdiv(kv_capacity, sp), 64))
     S = cdiv(kv_capacity, chunk)
     n_attn = w.batch * w.n_kv_heads * S
-    n_merge = w.batch * w.n_kv_heads if S > 1 else 0
-    per_layer = t_qkv + n_attn + n_merge + tiles(w.hidden) + tiles(w.ffn) + tiles(w.hidden)
+    per_layer = t_qkv + n_attn + tiles(w.hidden) + tiles(w.ffn) + tiles(w.hidden)
     tasks = 1 + w.n_layers * per_layer + tiles(w.vocab) + 1
-    # events per layer: x (QKV input), one per kv group (QKV -> ATTN), one per
-    # (b, g) when split (ATTN -> MERGE), attention output, O output, GATE_UP output;
-    # plus the final hidden state (-> LM_HEAD) and the LM partials (-> ARGMAX).
-    ev_layer = 1 + w.n_kv_heads + (w.batch * w.n_kv_heads if S > 1 else 0) + 3
+    # events per layer: x (QKV input), one per kv group (QKV -> ATTN), attention
+    # output (ATTN -> O), O output, GATE_UP output; plus the final hidden state
+    # (-> LM_HEAD) and the LM partials (-> ARGMAX).
+    ev_layer = 1 + w.n_kv_heads + 3
     events = w.n_layers * ev_layer + 2
     return tasks, events

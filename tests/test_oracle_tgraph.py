@@ -53,10 +53,10 @@ def test_decode_graph_invariants_counts_and_semantics(w, W):
 
 
 def test_qwen3_8b_bs1_graph_size():
-    # 36 layers x (QKV 128 + ATTN 136 + MERGE 8 + O 128 + GATE_UP 128 + DOWN 128)
-    # + EMBED + LM_HEAD 147 + ARGMAX on 148 workers.
+    # 36 layers x (QKV 128 + ATTN 136 + O 128 + GATE_UP 128 + DOWN 128)
+    # + EMBED + LM_HEAD 147 + ARGMAX on 148 workers; 36 x 12 + 2 events.
     g = oracle.tgraph_decode(synth.Q8B, synth.Q8B.kv_capacity(0), 148)
-    assert g.n_tasks == 23765 and g.n_events == 722
+    assert g.n_tasks == 23477 and g.n_events == 434
     assert (g.qkv_rows, g.o_rows, g.gu_rows, g.down_rows, g.lm_rows) == (48, 32, 96, 32, 1040)
     assert (g.splits, g.chunk) == (17, 64)
 
