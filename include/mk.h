@@ -209,6 +209,32 @@ mk_status mk_decode_step_perop(mk_handle *h, const int32_t *d_tokens_in, int32_t
                                int32_t *d_kv_len, void *d_k_cache, void *d_v_cache,
                                float *d_logits, void *stream);
 
+/*
+ * mk_decode_step_noalloc - mk_decode_step that allocates nothing and keeps
+ * every per-step working buffer (event and arrival counters, step epoch,
+ * activations, attention partials, LM-head partials, per-layer pointer table)
+ * in one static device region of 16 MiB instead of the handle's own buffers.
+ * The pages have no counterpart: this exists for callers that cannot call
+ * cudaMalloc when they need another stepping context -- cudaMalloc may
+ * synchronise the device and cannot run while a stream is being captured,
+ * and some programs hand all device memory out through their own allocator
+ * once the model is loaded.  The handle (graph tables, weights, status word)
+ * is used as built; its own working buffers, and so mk_final_hidden, are left
+ * untouched.  Arguments, results and device-side error reporting
+ * (mk_sync_status, mk_reset) are those of mk_decode_step.
+ * The region is a file-scope static array: every GPU that loads the library
+ * holds it until the process exits.  The first call on a device looks up the
+ * region's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * region and clear its counters first, so calls that overlap on the GPU race:
+ * order them on one stream.  Errors: MK_ERR_ARG when the step needs more than
+ * 16 MiB of working memory (or for bad arguments), MK_ERR_NOT_LOADED,
+ * MK_ERR_CUDA.
+ */
+mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
+                                 int32_t *d_kv_len, void *d_k_cache, void *d_v_cache,
+                                 float *d_logits, void *stream);
+
 /* mk_sync_status - synchronize `stream`, then return the device status word
  * (MK_OK, MK_ERR_TIMEOUT or MK_ERR_DEVICE).  detail (nullable, 4 ints):
  * {status, task id, event id, block}.  The word stays set until mk_reset. */

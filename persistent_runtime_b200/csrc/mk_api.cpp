@@ -14,38 +14,9 @@
 #include "runtime.cuh"
 #include "tgraph.hpp"
 
-namespace mk {
-size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int rep_p);
-cudaError_t worker_configure(size_t smem);
-cudaError_t worker_max_blocks(int *blocks, size_t smem);
-cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream);
-cudaError_t launch_tasks(const Params &p, int n_ctas, size_t smem, cudaStream_t stream);
-}  // namespace mk
+#include "mk_handle.hpp"
 
 using mk::Params;
-
-struct mk_handle {
-  mk_model_config cfg{};
-  mk_tuning tune{};
-  mk::TaskGraph graph;
-  bool host_only = true;
-  int device = -1;
-  std::string err;
-  // device state
-  void *dev_block = nullptr;  // graph tables, counters, activations, rope table
-  size_t dev_block_bytes = 0;
-  void *arena = nullptr;      // weights
-  size_t arena_bytes = 0;
-  bool loaded = false;
-  mk::DevLayer *d_layers = nullptr;
-  std::vector<mk::DevLayer> layers;
-  std::vector<int32_t> op_offset;  // into d_op_tasks
-  int32_t *d_op_tasks = nullptr;
-  Params base{};
-  size_t smem = 0;
-  int64_t act_bytes = 0;
-  int64_t weight_bytes = 0;
-};
 
 namespace {
 
