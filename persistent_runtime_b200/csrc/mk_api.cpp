@@ -34,14 +34,16 @@ mk_status cuda_fail(mk_handle *h, cudaError_t e, const char *what) {
   return fail(h, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
-mk_tuning fill_defaults(const mk_tuning *t) {
+mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   mk_tuning d{};
   if (t) d = *t;
   if (d.col_align <= 0) d.col_align = 16;
   if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 4;
   if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
-  if (d.ring_stages <= 0) d.ring_stages = 4;
-  if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
+  // the same bytes in flight per SM; the tensor-core tiles of batch >= 2 use
+  // more, smaller stages (at most 24 k-blocks per stage)
+  if (d.ring_stages <= 0) d.ring_stages = batch > 1 ? 8 : 4;
+  if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = (batch > 1 ? 24 : 48) * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
   if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
   return d;
@@ -67,8 +69,6 @@ std::string check_gpu_shape(const mk_model_config &c) {
     return "hidden, ffn and n_q_heads*head_dim must be multiples of 256";
   if (std::max(std::max(c.hidden, c.ffn), qd) > mk::kMaxCpt * 8 * mk::kComputeThreads)
     return "projection input width above 16384";
-  if (c.batch > 1)
-    return "batch > 1 needs the tensor-core projection path, which this build does not have";
   if (c.batch > mk::kMaxBatch) return "batch above 16";
   return "";
 }
@@ -106,7 +106,7 @@ mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int
   mk_handle *h = new (std::nothrow) mk_handle();
   if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
   h->cfg = *cfg;
-  h->tune = fill_defaults(tuning);
+  h->tune = fill_defaults(tuning, cfg->batch);
   h->tune.num_workers = num_workers;
   mk_status s = plan(cfg, h->tune, num_workers, h);
   if (s != MK_OK) {
@@ -158,13 +158,17 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   h->host_only = false;
   h->device = device;
   h->cfg = *cfg;
-  h->tune = fill_defaults(tuning);
+  h->tune = fill_defaults(tuning, cfg->batch);
   mk_tuning &t = h->tune;
   const mk_model_config &c = *cfg;
   const int D = c.head_dim;
   if (t.ring_stage_bytes % 1024) {
     delete h;
     return fail(nullptr, MK_ERR_ARG, "ring_stage_bytes must be a multiple of 1024");
+  }
+  if (c.batch > 1 && t.col_align % 16) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "batch > 1 needs col_align to be a multiple of 16");
   }
   const int rep0 = c.n_q_heads / c.n_kv_heads;
   const int rep_p = rep0 <= 1 ? 1 : rep0 <= 2 ? 2 : rep0 <= 4 ? 4 : 8;
@@ -239,6 +243,23 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     o_xm[l] = take(4 * (size_t)B * H);
     o_h[l] = take(4 * (size_t)B * F);
   }
+  // batch >= 2: fragment-ordered hi/lo bf16 operands (8 or 16 columns) and
+  // the per-16-row sums of squares of the streams that feed an RMSNorm
+  const bool mma = B > 1;
+  const int nn = B > 8 ? 2 : 1, Bp = 8 * nn, n_parts = H / 16;
+  std::vector<size_t> o_xa(Ly + 1), o_ssa(Ly + 1), o_attb(Ly), o_xmb(Ly), o_ssm(Ly), o_hb(Ly);
+  if (mma) {
+    for (int l = 0; l <= Ly; ++l) {  // entry Ly: the final hidden state (LM head input)
+      o_xa[l] = take(4 * (size_t)Bp * H);
+      o_ssa[l] = take(4 * (size_t)B * n_parts);
+    }
+    for (int l = 0; l < Ly; ++l) {
+      o_attb[l] = take(4 * (size_t)Bp * qd);
+      o_xmb[l] = take(4 * (size_t)Bp * H);
+      o_ssm[l] = take(4 * (size_t)B * n_parts);
+      o_hb[l] = take(4 * (size_t)Bp * F);
+    }
+  }
   h->act_bytes = (int64_t)(off - act0);
   h->dev_block_bytes = off;
   ce = cudaMalloc(&h->dev_block, off);
@@ -288,6 +309,16 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     L.h = reinterpret_cast<float *>(base + o_h[l]);
     L.x_in = reinterpret_cast<float *>(base + o_x) + (size_t)l * B * H;
     L.x_out = reinterpret_cast<float *>(base + o_x) + (size_t)(l + 1) * B * H;
+    if (mma) {
+      L.xa = reinterpret_cast<uint16_t *>(base + o_xa[l]);
+      L.ssa = reinterpret_cast<float *>(base + o_ssa[l]);
+      L.attb = reinterpret_cast<uint16_t *>(base + o_attb[l]);
+      L.xmb = reinterpret_cast<uint16_t *>(base + o_xmb[l]);
+      L.ssm = reinterpret_cast<float *>(base + o_ssm[l]);
+      L.hb = reinterpret_cast<uint16_t *>(base + o_hb[l]);
+      L.xa_next = reinterpret_cast<uint16_t *>(base + o_xa[l + 1]);
+      L.ssa_next = reinterpret_cast<float *>(base + o_ssa[l + 1]);
+    }
   }
   ce = cudaMemcpy(base + o_tasks, tasks.data(), sizeof(mk::DevTask) * tasks.size(),
                   cudaMemcpyHostToDevice);
@@ -346,6 +377,33 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.rps_down = rps(F);
   p.rps_lm = rps(H);
   p.pps = t.ring_stage_bytes / (4 * D);
+  if (mma) {
+    // m-tiles per row block: the task's rows up to the accumulator limit;
+    // k-blocks per stage: what the stage holds for that many m-tiles, a
+    // multiple of 8 (one share per warp), at most 8 per warp and stage
+    const int units = t.ring_stage_bytes / 512;
+    auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
+    auto kcb_of = [&](int mb) { return std::min(mk::kMmaMaxKCB, units / mb / 8 * 8); };
+    p.mma = 1;
+    p.nn = nn;
+    p.n_parts = n_parts;
+    p.mb_qkv = mb_of(T.qkv_rows);
+    p.mb_o = mb_of(T.o_rows);
+    p.mb_gu = mb_of(2 * T.gu_rows);
+    p.mb_down = mb_of(T.down_rows);
+    p.mb_lm = mb_of(T.lm_rows);
+    p.kcb_qkv = kcb_of(p.mb_qkv);
+    p.kcb_o = kcb_of(p.mb_o);
+    p.kcb_gu = kcb_of(p.mb_gu);
+    p.kcb_down = kcb_of(p.mb_down);
+    p.kcb_lm = kcb_of(p.mb_lm);
+    p.xfb = reinterpret_cast<uint16_t *>(base + o_xa[Ly]);
+    p.ssf = reinterpret_cast<float *>(base + o_ssa[Ly]);
+    if (std::min({p.kcb_qkv, p.kcb_o, p.kcb_gu, p.kcb_down, p.kcb_lm}) < 8) {
+      mk_destroy(h);
+      return fail(nullptr, MK_ERR_ARG, "ring stage too small for the tensor-core tiles");
+    }
+  }
   p.ring_stages = t.ring_stages;
   p.stage_bytes = t.ring_stage_bytes;
   p.l2_prefetch_bytes = t.l2_prefetch_bytes;
@@ -385,7 +443,13 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     o_gu[l] = take((size_t)2 * F * H);
     o_dn[l] = take((size_t)H * F);
   }
-  const size_t o_lm = c.tied_embeddings ? 0 : take((size_t)V * H);
+  // batch >= 2: projection matrices in mma.sync fragment order, the LM head
+  // padded to whole 16-row m-tiles and kept apart from the (row-major)
+  // embedding table even when the two are tied
+  const bool mma = h->base.mma != 0;
+  const size_t Vp = mma ? ((size_t)V + 15) / 16 * 16 : (size_t)V;
+  const bool lm_shares_embed = c.tied_embeddings && !mma;
+  const size_t o_lm = lm_shares_embed ? 0 : take(Vp * H);
   const size_t o_emb = take((size_t)V * H);
   for (int l = 0; l < Ly; ++l) {
     o_an[l] = take(H);
@@ -405,33 +469,77 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
   }
   char *A = static_cast<char *>(h->arena);
   cudaError_t e = cudaSuccess;
-  auto cp = [&](size_t dst_off, const void *src, size_t bytes) {
-    if (e == cudaSuccess) e = cudaMemcpyAsync(A + dst_off, src, bytes, cudaMemcpyDefault, st);
+  auto cpy = [&](char *dst, const void *src, size_t bytes) {
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st);
   };
+  auto cp = [&](size_t dst_off, const void *src, size_t bytes) { cpy(A + dst_off, src, bytes); };
   const size_t row = 2 * (size_t)H;
-  for (int l = 0; l < Ly; ++l) {
+  // Row-major matrices in arena row order, written at dst: QKV group-major,
+  // gate/up interleaved.
+  auto put_qkv = [&](char *dst, int l) {
     for (int g = 0; g < c.n_kv_heads; ++g) {
-      const size_t dst = o_qkv[l] + (size_t)g * grp * row;
-      cp(dst, static_cast<const char *>(w->wq[l]) + (size_t)g * rep * D * row, (size_t)rep * D * row);
-      cp(dst + (size_t)rep * D * row, static_cast<const char *>(w->wk[l]) + (size_t)g * D * row,
-         (size_t)D * row);
-      cp(dst + (size_t)(rep + 1) * D * row,
-         static_cast<const char *>(w->wv[l]) + (size_t)g * D * row, (size_t)D * row);
+      char *d = dst + (size_t)g * grp * row;
+      cpy(d, static_cast<const char *>(w->wq[l]) + (size_t)g * rep * D * row, (size_t)rep * D * row);
+      cpy(d + (size_t)rep * D * row, static_cast<const char *>(w->wk[l]) + (size_t)g * D * row,
+          (size_t)D * row);
+      cpy(d + (size_t)(rep + 1) * D * row,
+          static_cast<const char *>(w->wv[l]) + (size_t)g * D * row, (size_t)D * row);
     }
-    cp(o_o[l], w->wo[l], (size_t)H * qd * 2);
+  };
+  auto put_gu = [&](char *dst, int l) {
     if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(A + o_gu[l], 2 * row, w->w_gate[l], row, row, F, cudaMemcpyDefault, st);
+      e = cudaMemcpy2DAsync(dst, 2 * row, w->w_gate[l], row, row, F, cudaMemcpyDefault, st);
     if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(A + o_gu[l] + row, 2 * row, w->w_up[l], row, row, F, cudaMemcpyDefault,
-                            st);
-    cp(o_dn[l], w->w_down[l], (size_t)H * F * 2);
+      e = cudaMemcpy2DAsync(dst + row, 2 * row, w->w_up[l], row, row, F, cudaMemcpyDefault, st);
+  };
+  const void *lm_src = c.tied_embeddings ? w->embed : w->lm_head;
+  if (!mma) {
+    for (int l = 0; l < Ly; ++l) {
+      put_qkv(A + o_qkv[l], l);
+      cp(o_o[l], w->wo[l], (size_t)H * qd * 2);
+      put_gu(A + o_gu[l], l);
+      cp(o_dn[l], w->w_down[l], (size_t)H * F * 2);
+    }
+    if (!c.tied_embeddings) cp(o_lm, w->lm_head, (size_t)V * H * 2);
+  } else {
+    // each matrix goes row-major into a staging buffer, then a kernel writes
+    // it to the arena in fragment order; the LM head goes in row slabs
+    const size_t tmp_bytes =
+        2 * std::max({n_qkv * H, (size_t)H * qd, (size_t)2 * F * H, (size_t)H * F});
+    void *tmp = nullptr;
+    if (cudaMalloc(&tmp, tmp_bytes) != cudaSuccess)
+      return fail(h, MK_ERR_OOM, "cudaMalloc of the weight staging buffer failed");
+    char *T = static_cast<char *>(tmp);
+    auto frag = [&](size_t dst_off, int rows, int K) {
+      if (e == cudaSuccess) e = mk::permute_to_fragments(A + dst_off, T, rows, K, st);
+    };
+    for (int l = 0; l < Ly; ++l) {
+      put_qkv(T, l);
+      frag(o_qkv[l], (int)n_qkv, H);
+      cpy(T, w->wo[l], (size_t)H * qd * 2);
+      frag(o_o[l], H, (int)qd);
+      put_gu(T, l);
+      frag(o_gu[l], 2 * F, H);
+      cpy(T, w->w_down[l], (size_t)H * F * 2);
+      frag(o_dn[l], H, F);
+    }
+    const int slab = (int)std::min<size_t>((size_t)V, tmp_bytes / row / 16 * 16);
+    for (int r0 = 0; r0 < V; r0 += slab) {
+      const int n = std::min(slab, V - r0);
+      cpy(T, static_cast<const char *>(lm_src) + (size_t)r0 * row, (size_t)n * row);
+      // m-tile r0 / 16 of the padded head: 512-byte blocks, H / 16 per m-tile
+      frag(o_lm + (size_t)(r0 / 16) * (H / 16) * 512, n, H);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // the staging buffer is freed next
+    cudaFree(tmp);
+  }
+  for (int l = 0; l < Ly; ++l) {
     cp(o_an[l], w->attn_norm[l], (size_t)H * 2);
     cp(o_qn[l], w->q_norm[l], (size_t)D * 2);
     cp(o_kn[l], w->k_norm[l], (size_t)D * 2);
     cp(o_mn[l], w->mlp_norm[l], (size_t)H * 2);
   }
   cp(o_emb, w->embed, (size_t)V * H * 2);
-  if (!c.tied_embeddings) cp(o_lm, w->lm_head, (size_t)V * H * 2);
   cp(o_fn, w->final_norm, (size_t)H * 2);
   if (e != cudaSuccess) return cuda_fail(h, e, "weight copy");
   for (int l = 0; l < Ly; ++l) {
@@ -444,6 +552,7 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     L.q_norm = reinterpret_cast<const uint16_t *>(A + o_qn[l]);
     L.k_norm = reinterpret_cast<const uint16_t *>(A + o_kn[l]);
     L.mlp_norm = reinterpret_cast<const uint16_t *>(A + o_mn[l]);
+    L.gain_next = reinterpret_cast<const uint16_t *>(A + (l + 1 < Ly ? o_an[l + 1] : o_fn));
   }
   e = cudaMemcpyAsync(h->d_layers, h->layers.data(), sizeof(mk::DevLayer) * Ly,
                       cudaMemcpyHostToDevice, st);
@@ -451,7 +560,7 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
   if (e != cudaSuccess) return cuda_fail(h, e, "layer table upload");
   Params &p = h->base;
   p.embed = reinterpret_cast<const uint16_t *>(A + o_emb);
-  p.lm_head = reinterpret_cast<const uint16_t *>(A + (c.tied_embeddings ? o_emb : o_lm));
+  p.lm_head = reinterpret_cast<const uint16_t *>(A + (lm_shares_embed ? o_emb : o_lm));
   p.final_norm = reinterpret_cast<const uint16_t *>(A + o_fn);
   h->weight_bytes = 0;
   for (int l = 0; l < Ly; ++l)

@@ -38,6 +38,9 @@ size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 struct Layout {
   size_t counters, arrivals, epoch, status, layers, lm_val, lm_idx, x, total;
   std::vector<size_t> qkv, part, att, xm, h;
+  // batch >= 2: operands and sums of squares (index n_layers of xa / ssa: the
+  // final hidden state)
+  std::vector<size_t> xa, ssa, attb, xmb, ssm, hb;
 };
 
 Layout layout_of(const mk_model_config &c, const mk::TaskGraph &g) {
@@ -67,6 +70,19 @@ Layout layout_of(const mk_model_config &c, const mk::TaskGraph &g) {
     L.att.push_back(take(4 * (size_t)B * qd));
     L.xm.push_back(take(4 * (size_t)B * H));
     L.h.push_back(take(4 * (size_t)B * F));
+  }
+  if (B > 1) {
+    const int Bp = B > 8 ? 16 : 8, n_parts = H / 16;
+    for (int l = 0; l <= Ly; ++l) {
+      L.xa.push_back(take(4 * (size_t)Bp * H));
+      L.ssa.push_back(take(4 * (size_t)B * n_parts));
+    }
+    for (int l = 0; l < Ly; ++l) {
+      L.attb.push_back(take(4 * (size_t)Bp * qd));
+      L.xmb.push_back(take(4 * (size_t)Bp * H));
+      L.ssm.push_back(take(4 * (size_t)B * n_parts));
+      L.hb.push_back(take(4 * (size_t)Bp * F));
+    }
   }
   L.total = off;
   return L;
@@ -147,6 +163,16 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
     d.h = reinterpret_cast<float *>(base + L.h[l]);
     d.x_in = x + (size_t)l * B * H;
     d.x_out = x + (size_t)(l + 1) * B * H;
+    if (B > 1) {
+      d.xa = reinterpret_cast<uint16_t *>(base + L.xa[l]);
+      d.ssa = reinterpret_cast<float *>(base + L.ssa[l]);
+      d.attb = reinterpret_cast<uint16_t *>(base + L.attb[l]);
+      d.xmb = reinterpret_cast<uint16_t *>(base + L.xmb[l]);
+      d.ssm = reinterpret_cast<float *>(base + L.ssm[l]);
+      d.hb = reinterpret_cast<uint16_t *>(base + L.hb[l]);
+      d.xa_next = reinterpret_cast<uint16_t *>(base + L.xa[l + 1]);
+      d.ssa_next = reinterpret_cast<float *>(base + L.ssa[l + 1]);
+    }
   }
   // The region keeps the previous call's contents: counters, arrival counters
   // and the epoch must start at zero (activations are fully rewritten).
@@ -169,6 +195,10 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
   p.x_final = x + (size_t)Ly * B * H;
   p.lm_val = reinterpret_cast<float *>(base + L.lm_val);
   p.lm_idx = reinterpret_cast<int32_t *>(base + L.lm_idx);
+  if (B > 1) {
+    p.xfb = reinterpret_cast<uint16_t *>(base + L.xa[Ly]);
+    p.ssf = reinterpret_cast<float *>(base + L.ssa[Ly]);
+  }
   p.trace = nullptr;
   p.tokens_in = d_tokens_in;
   p.tokens_out = d_tokens_out;

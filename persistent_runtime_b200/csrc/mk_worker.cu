@@ -183,6 +183,46 @@ __device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 }
 
 // ---------------------------------------------------------------------------
+// Tensor cores (batch >= 2): mma.sync.m16n8k16, A = weights (16 rows x 16 k,
+// row major), B = activations (16 k x 8 sequences), fp32 accumulators.
+// Fragment ownership (PTX ISA, "Matrix Fragments for mma.m16n8k16"), lane l,
+// g = l / 4, t = l % 4:  A regs {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..),
+// (g+8, 2t+8..)};  B regs {(2t..2t+1, g), (2t+8..2t+9, g)};  C {(g, 2t),
+// (g, 2t+1), (g+8, 2t), (g+8, 2t+1)}.  Weights and activations are stored in
+// exactly this order, so each lane fetches its fragment with one 16-byte
+// (A) or 8-byte (B) load.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, const uint2 &b) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y));
+}
+
+// Activation operands are two-term bf16 expansions x = hi + lo, hi = bf16(x),
+// lo = bf16(x - hi): about 16 significant bits, so W x = W hi + W lo (two MMAs
+// into one fp32 accumulator) keeps the projection inputs close to fp32 while
+// the weights stay exactly bf16.  A single bf16 rounding of every input would
+// cost ~0.4 % of the residual stream per layer.
+//
+// Element (k, sequence b) of an operand with nn 8-column tiles, in bf16
+// units: 512-byte blocks per (16-row k-block, column tile), 16 bytes per lane
+// inside a block: {hi b0, hi b1, lo b0, lo b1} of the lane's B fragment.
+// Returns the position of hi; lo is 4 elements further.
+__device__ __forceinline__ size_t opnd_off(int k, int b, int nn) {
+  const int kk = k & 15;
+  return ((size_t)(k >> 4) * nn + (b >> 3)) * 256 + ((b & 7) * 4 + ((kk & 7) >> 1)) * 8 +
+         (kk >> 3) * 2 + (kk & 1);
+}
+
+__device__ __forceinline__ void put_opnd(uint16_t *buf, int k, int b, int nn, float x) {
+  const size_t o = opnd_off(k, b, nn);
+  const uint16_t hi = f2bf(x);
+  buf[o] = hi;
+  buf[o + 4] = f2bf(x - bf2f(hi));
+}
+
+// ---------------------------------------------------------------------------
 // Shared memory layout (identical computation on host: see smem_bytes()).
 // ---------------------------------------------------------------------------
 enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kCtlWords = 16 };
@@ -203,12 +243,18 @@ struct Smem {
   float *sc;    // per warp: [32] probabilities, [kMaxRep] rescale factors
   float *mls;   // [3][kMaxRep]
   float *ored;  // per warp and head: [D] output, running max, running sum (merge: weights)
+  // tensor-core projection scratch
+  float *cred;  // [warp][m-tile of the pass][16 rows][8 nn + 1] accumulator partials
+  float *minv;  // [kMaxBatch] 1 / rms of each sequence's input
+  float *mlv;   // [16] partial argmax values (LM head)
+  int *mli;     // [16] partial argmax indices
 };
 
 __host__ __device__ inline size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct SmemOffsets {
-  size_t full, empty, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, total;
+  size_t full, empty, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, cred, minv,
+      mlv, mli, total;
 };
 
 __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes, int pps,
@@ -249,7 +295,19 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   a = align_to(a, 16);
   o.ored = a;  // per warp and head: o[D], running max, running sum
   a += 4 * (size_t)kStateSlots * rep_p * (head_dim + 2);
-  o.total = align_to(g > a ? g : a, 128);
+  // tensor-core projection scratch (same bytes again)
+  size_t m = p;
+  o.cred = m;
+  m += 4 * (size_t)kMmaCredFloats;
+  o.minv = m;
+  m += 4 * kMaxBatch;
+  o.mlv = m;
+  m += 4 * 16;
+  o.mli = m;
+  m += 4 * 16;
+  size_t top = g > a ? g : a;
+  top = top > m ? top : m;
+  o.total = align_to(top, 128);
   return o;
 }
 
@@ -271,6 +329,10 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
   s.sc = reinterpret_cast<float *>(base + o.sc);
   s.mls = reinterpret_cast<float *>(base + o.mls);
   s.ored = reinterpret_cast<float *>(base + o.ored);
+  s.cred = reinterpret_cast<float *>(base + o.cred);
+  s.minv = reinterpret_cast<float *>(base + o.minv);
+  s.mlv = reinterpret_cast<float *>(base + o.mlv);
+  s.mli = reinterpret_cast<int *>(base + o.mli);
   return s;
 }
 
@@ -326,6 +388,37 @@ __device__ __forceinline__ Gemv gemv_of(const Params &p, int type, int layer, in
   return g;
 }
 
+// A projection task on tensor cores: its m-tiles [mt0, mt1) of the
+// fragment-ordered matrix are streamed as row blocks of mb m-tiles, each row
+// block as nkc ring stages of (up to) kcb k-blocks.  Every (m-tile, k-block)
+// is one 512-byte fragment block; stage (rb, kc) packs the blocks of its
+// m-tiles as [m-tile][k-block].
+struct MmaTile {
+  const uint16_t *w;  // the operator's matrix, fragment order
+  int KB;             // k-blocks per row (K / 16)
+  int mt0, mt1;       // m-tiles of this task
+  int mb, kcb, nkc, nrb;
+};
+
+__device__ __forceinline__ MmaTile mma_tile(const Params &p, int type, int layer, int idx) {
+  const Gemv g = gemv_of(p, type, layer, idx);
+  MmaTile m;
+  m.w = g.w;
+  m.KB = g.K >> 4;
+  m.mt0 = g.row0 >> 4;
+  m.mt1 = (g.row1 + 15) >> 4;  // the LM head's last m-tile may hold zero padding rows
+  switch (type) {
+    case 2: m.mb = p.mb_qkv; m.kcb = p.kcb_qkv; break;
+    case 5: m.mb = p.mb_o; m.kcb = p.kcb_o; break;
+    case 6: m.mb = p.mb_gu; m.kcb = p.kcb_gu; break;
+    case 7: m.mb = p.mb_down; m.kcb = p.kcb_down; break;
+    default: m.mb = p.mb_lm; m.kcb = p.kcb_lm; break;
+  }
+  m.nkc = (m.KB + m.kcb - 1) / m.kcb;
+  m.nrb = (m.mt1 - m.mt0 + m.mb - 1) / m.mb;
+  return m;
+}
+
 struct AttnSpan {
   int b, g, s, L;      // sequence, kv head, split, cached rows before the step
   int p0, cached_end;  // cached rows [p0, cached_end) of this split
@@ -359,11 +452,26 @@ struct Stream {
   uint32_t bytes, last_bytes;  // bytes of a full / of the last stage (per source)
   uint32_t stride;             // bytes between consecutive stages of one source
   int nst;                     // stages
+  // tensor-core projections: stage st = (row block st / nkc, k chunk st % nkc)
+  int nkc;                     // 0 for the plain streams above
+  int KB, mt0, mt1, mb, kcb;
 };
 
 __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t) {
-  Stream s{nullptr, nullptr, 0u, 0u, 0u, 0};
+  Stream s{nullptr, nullptr, 0u, 0u, 0u, 0, 0, 0, 0, 0, 0, 0};
   const int type = t.type;
+  if (p.mma && (type == 2 || (type >= 5 && type <= 8))) {
+    const MmaTile m = mma_tile(p, type, t.layer, (int)t.idx);
+    s.src0 = reinterpret_cast<const uint8_t *>(m.w);
+    s.nst = m.nrb * m.nkc;
+    s.nkc = m.nkc;
+    s.KB = m.KB;
+    s.mt0 = m.mt0;
+    s.mt1 = m.mt1;
+    s.mb = m.mb;
+    s.kcb = m.kcb;
+    return s;
+  }
   if (type == 3) {
     const AttnSpan a = attn_span(p, (int)t.idx);
     const int n = a.cached_end - a.p0;
@@ -385,6 +493,52 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
   return s;
 }
 
+// Bytes that stage st of stream s lands in the ring.
+__device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
+  if (s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int nm = min(s.mb, s.mt1 - (s.mt0 + rb * s.mb));
+    const int nkb = min(s.kcb, s.KB - kc * s.kcb);
+    return (uint32_t)(nm * nkb * 512);
+  }
+  const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
+  return s.src1 ? 2 * nb : nb;
+}
+
+// Issue the copies of stage st of stream s into ring slot dst (the full
+// barrier already expects stage_bytes_of(s, st) bytes).
+__device__ __forceinline__ void issue_stage(const Stream &s, int st, uint8_t *dst, int stage_bytes,
+                                            uint64_t *bar) {
+  if (s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
+    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
+    const uint32_t cb = (uint32_t)nkb * 512u;
+    for (int i = 0; i < nm; ++i)
+      bulk_g2s(dst + (size_t)i * cb, s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb, bar);
+    return;
+  }
+  const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
+  bulk_g2s(dst, s.src0 + (size_t)st * s.stride, nb, bar);
+  if (s.src1) bulk_g2s(dst + stage_bytes / 2, s.src1 + (size_t)st * s.stride, nb, bar);
+}
+
+// Prefetch stage st of stream s into L2; returns the bytes requested.
+__device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
+  if (s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
+    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
+    const uint32_t cb = (uint32_t)nkb * 512u;
+    for (int i = 0; i < nm; ++i) prefetch_l2(s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb);
+    return cb * (uint32_t)nm;
+  }
+  const uint32_t pb = st == s.nst - 1 ? s.last_bytes : s.bytes;
+  prefetch_l2(s.src0 + (size_t)st * s.stride, pb);
+  if (s.src1) prefetch_l2(s.src1 + (size_t)st * s.stride, pb);
+  return s.src1 ? 2 * pb : pb;
+}
+
 // ---------------------------------------------------------------------------
 // Producer: one thread streams every stage of the worker's queue.
 // ---------------------------------------------------------------------------
@@ -402,13 +556,13 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // up to l2_prefetch_bytes ahead of the ring.
   const long long dist = p.l2_prefetch_bytes;
   int pf_n = 0, pf_st = 0;
-  Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1};
+  Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1, 0, 0, 0, 0, 0, 0};
   uint32_t pf_k = 0;
   long long ahead = 0;
   for (int n = 0; n < q.count; ++n) {
     const Stream ts = task_stream(p, p.tasks[q.first + n * q.stride]);
     for (int st = 0; st < ts.nst; ++st) {
-      const uint32_t nb = st == ts.nst - 1 ? ts.last_bytes : ts.bytes;
+      const uint32_t nb = stage_bytes_of(ts, st);
       if (dist > 0) {
         // stages before k were issued without a prefetch: move the cursor on
         while (pf_k < k && pf_n < q.count) {
@@ -440,11 +594,9 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
               pf_st = 0;
               pfs.nst = -1;
             } else {
-              const uint32_t pb = pf_st == pfs.nst - 1 ? pfs.last_bytes : pfs.bytes;
-              prefetch_l2(pfs.src0 + (size_t)pf_st * pfs.stride, pb);
-              if (pfs.src1) prefetch_l2(pfs.src1 + (size_t)pf_st * pfs.stride, pb);
-              ahead += pfs.src1 ? 2 * pb : pb;
-              if (p.trace) sm.tmark[3] += pfs.src1 ? 2 * pb : pb;
+              const uint32_t pb = prefetch_stage(pfs, pf_st);
+              ahead += pb;
+              if (p.trace) sm.tmark[3] += pb;
               ++pf_st;
               ++pf_k;
             }
@@ -460,10 +612,9 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
         }
       }
       uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes;
-      mbar_arrive_expect_tx(&sm.full[slot], ts.src1 ? 2 * nb : nb);
-      bulk_g2s(dst, ts.src0 + (size_t)st * ts.stride, nb, &sm.full[slot]);
-      if (ts.src1) bulk_g2s(dst + p.stage_bytes / 2, ts.src1 + (size_t)st * ts.stride, nb, &sm.full[slot]);
-      if (dist > 0 && pf_k > k) ahead -= ts.src1 ? 2 * nb : nb;  // stage k was prefetched
+      mbar_arrive_expect_tx(&sm.full[slot], nb);
+      issue_stage(ts, st, dst, p.stage_bytes, &sm.full[slot]);
+      if (dist > 0 && pf_k > k) ahead -= nb;  // stage k was prefetched
       ++k;
     }
   }
@@ -770,6 +921,259 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 }
 
 // ---------------------------------------------------------------------------
+// Projection task on tensor cores (batch >= 2).
+// ---------------------------------------------------------------------------
+// B fragments of k-blocks kb0 + warp + 8 j (j < kpw) of the operand xb: the
+// activations are written earlier in this step by other SMs, so they are read
+// through L2 (never from a possibly stale L1 line).
+template <int NN>
+__device__ __forceinline__ void load_bfrag(uint4 (&bf)[kMmaMaxKPW][NN], const uint16_t *xb,
+                                           int kb0, int kpw, int warp, int lane) {
+#pragma unroll
+  for (int j = 0; j < kMmaMaxKPW; ++j) {
+    if (j < kpw) {
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+        bf[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
+                              xb + ((size_t)(kb0 + warp + 8 * j) * NN + n) * 256) + lane);
+    }
+  }
+}
+
+// Sum over the 16 lanes of a half warp (lanes that share a sequence column).
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// The batched projection y[b][r] = sum_k W[r][k] x̂[b][k] of one task on
+// mma.sync.  The input arrives as a hi/lo bf16 operand of x[b][k] * gain[k]
+// written by the producing task's epilogue, with per-16-row sums of squares;
+// the RMSNorm's per-sequence factor 1 / rms(x_b) is applied to the fp32
+// accumulators in the epilogue (it factors out of the sum over k).
+//
+// Work split: for each ring stage (row block x k chunk) warp w takes the
+// k-blocks w, w + 8, ... of the chunk for every m-tile of the row block, so
+// every B fragment is loaded by one warp, once per row block.  The warps'
+// partial sums of a row block are added in shared memory in a fixed order
+// (deterministic), PM m-tiles per pass, and the fused epilogue of the
+// operator runs on the sums: thread (row = tid % 16, sequence = tid / 16 % 8nn).
+template <int NN>
+__device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const DevTask &t,
+                                         uint32_t &k, int task_id, const DepWait &dep_wait) {
+  constexpr int NC = 8 * NN;          // operand columns (sequences, zero padded)
+  constexpr int PM = NN == 2 ? 2 : 4; // m-tiles per reduction pass
+  constexpr int CS = NC + 1;          // row stride of the reduction buffer (floats)
+  static_assert(kComputeWarps * PM * 16 * CS <= kMmaCredFloats, "reduction buffer");
+  const int type = t.type;
+  const int layer = t.layer;
+  const DevLayer *L = layer < p.Ly ? p.layers + layer : nullptr;
+  const MmaTile mt = mma_tile(p, type, layer, (int)t.idx);
+  const uint16_t *xb;
+  const float *ssp = nullptr;
+  switch (type) {
+    case 2: xb = L->xa; ssp = L->ssa; break;
+    case 5: xb = L->attb; break;
+    case 6: xb = L->xmb; ssp = L->ssm; break;
+    case 7: xb = L->hb; break;
+    default: xb = p.xfb; ssp = p.ssf; break;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = tid & 15;          // row of an m-tile this thread finishes
+  const int col = (tid >> 4) % NC;   // sequence this thread finishes
+  const bool col_ok = col < p.B;
+  const int N = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
+
+  if (!dep_wait()) return false;
+  uint4 bc[kMmaMaxKPW][NN];
+  load_bfrag<NN>(bc, xb, 0, min(mt.kcb, mt.KB) >> 3, warp, lane);
+  float inv = 1.f;
+  if (ssp) {
+    for (int b = warp; b < p.B; b += kComputeWarps) {
+      float s = 0.f;
+      for (int j = lane; j < p.n_parts; j += 32) s += __ldcg(ssp + (size_t)b * p.n_parts + j);
+      s = warp_sum(s);
+      if (lane == 0) sm.minv[b] = rsqrtf(s / (float)p.H + p.eps);
+    }
+    compute_sync();
+    inv = col_ok ? sm.minv[col] : 0.f;
+  }
+
+  float acc[kMmaMaxMB][NN][4];
+#pragma unroll
+  for (int m = 0; m < kMmaMaxMB; ++m)
+#pragma unroll
+    for (int n = 0; n < NN; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+  float best_v = -INFINITY;
+  int best_i = 0x7fffffff;
+  trace_mark(p, sm, 0);
+  const int nst = mt.nrb * mt.nkc;
+  for (int st = 0; st < nst; ++st) {
+    const int rb = st / mt.nkc, kc = st - rb * mt.nkc;
+    const int m0 = mt.mt0 + rb * mt.mb, nm = min(mt.mb, mt.mt1 - m0);
+    const int nkb = min(mt.kcb, mt.KB - kc * mt.kcb), kpw = nkb >> 3;
+    // the next stage's k chunk (the same chunks repeat for every row block):
+    // each B fragment register is refilled for it right after its last use
+    const int kn = kc + 1 == mt.nkc ? 0 : kc + 1;
+    const int kpw_n = st + 1 < nst ? min(mt.kcb, mt.KB - kn * mt.kcb) >> 3 : 0;
+    const uint16_t *xn = xb + ((size_t)(kn * mt.kcb + warp) * NN) * 256;
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (got) {
+      const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
+#pragma unroll
+      for (int j = 0; j < kMmaMaxKPW; ++j) {
+        if (j < kpw) {
+          const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
+#pragma unroll
+          for (int m = 0; m < kMmaMaxMB; ++m) {
+            if (m < nm) {
+              const uint4 a = *reinterpret_cast<const uint4 *>(blk + (size_t)m * nkb * 512);
+#pragma unroll
+              for (int n = 0; n < NN; ++n) {
+                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
+                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
+              }
+            }
+          }
+        }
+        if (j < kpw_n) {
+#pragma unroll
+          for (int n = 0; n < NN; ++n)
+            bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
+                                  xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+        }
+      }
+      release_stage(sm, p, k);
+      ++k;
+    }
+    if (kc + 1 < mt.nkc) continue;
+
+    // row block done: cross-warp sums and the fused epilogue, PM m-tiles per pass
+#pragma unroll
+    for (int q0 = 0; q0 < kMmaMaxMB; q0 += PM) {
+      if (q0 >= nm) break;  // uniform over the CTA
+      {
+        const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+        for (int ml = 0; ml < PM; ++ml) {
+          const int m = q0 + ml;
+          if (m < kMmaMaxMB && m < nm) {
+            float *cw = sm.cred + (size_t)(warp * PM + ml) * 16 * CS;
+#pragma unroll
+            for (int n = 0; n < NN; ++n) {
+              const int c = n * 8 + 2 * tq;
+              cw[g * CS + c] = acc[m][n][0];
+              cw[g * CS + c + 1] = acc[m][n][1];
+              cw[(g + 8) * CS + c] = acc[m][n][2];
+              cw[(g + 8) * CS + c + 1] = acc[m][n][3];
+            }
+          }
+        }
+      }
+      compute_sync();
+      if (!sm.ctl[kAbort]) {
+#pragma unroll
+        for (int it = 0; it < PM * NC / 16; ++it) {
+          const int ml = (tid + kComputeThreads * it) / (16 * NC);  // uniform per warp
+          const bool m_ok = q0 + ml < nm;
+          float v = 0.f;
+          if (m_ok) {
+#pragma unroll
+            for (int w = 0; w < kComputeWarps; ++w)
+              v += sm.cred[((size_t)(w * PM + ml) * 16 + row) * CS + col];
+          }
+          const int r = (m0 + q0 + ml) * 16 + row;  // row of the operator's output
+          const bool store = m_ok && col_ok && r < N;
+          const size_t bH = (size_t)col * p.H;
+          if (type == 2) {
+            if (store) L->qkv[(size_t)col * p.n_qkv + r] = v * inv;
+          } else if (type == 5 || type == 7) {
+            // residual add, next operand (gain of the following norm), 16-row ss
+            float x = 0.f;
+            if (store) {
+              x = __ldcg((type == 5 ? L->x_in : L->xm) + bH + r) + v;
+              (type == 5 ? L->xm : L->x_out)[bH + r] = x;
+              const uint16_t *gn = type == 5 ? L->mlp_norm : L->gain_next;
+              put_opnd(type == 5 ? L->xmb : L->xa_next, r, col, NN, x * bf2f(gn[r]));
+            }
+            const float s2 = half_warp_sum(x * x);
+            if (store && row == 0)
+              (type == 5 ? L->ssm : L->ssa_next)[(size_t)col * p.n_parts + (r >> 4)] = s2;
+          } else if (type == 6) {
+            // rows (2i, 2i + 1) = (gate_i, up_i) sit on neighbouring lanes
+            const float gv = v * inv;
+            const float uv = __shfl_xor_sync(0xffffffffu, gv, 1);
+            if (store && !(row & 1)) {
+              const int i = r >> 1;
+              const float hv = gv / (1.f + __expf(-gv)) * uv;
+              L->h[(size_t)col * p.F + i] = hv;
+              put_opnd(L->hb, i, col, NN, hv);
+            }
+          } else {
+            const float lv = v * inv;
+            if (store) {
+              if (p.logits) p.logits[(size_t)col * p.V + r] = lv;
+              if (lv > best_v || (lv == best_v && r < best_i)) {
+                best_v = lv;
+                best_i = r;
+              }
+            }
+          }
+        }
+      }
+      compute_sync();
+    }
+#pragma unroll
+    for (int m = 0; m < kMmaMaxMB; ++m)
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+  }
+  trace_mark(p, sm, 1);
+  if (sm.ctl[kAbort]) return false;
+  if (type == 8) {
+    // (max, lowest index) per sequence: the 16 lanes of a half warp share a
+    // column, then the 16 / NC half warps of each column
+    float bv = best_v;
+    int bi = best_i;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (row == 0) {
+      sm.mlv[tid >> 4] = bv;
+      sm.mli[tid >> 4] = bi;
+    }
+    compute_sync();
+    if (tid < p.B) {
+      bv = -INFINITY;
+      bi = 0x7fffffff;
+      for (int h = tid; h < 16; h += NC) {
+        const float ov = sm.mlv[h];
+        const int oi = sm.mli[h];
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (bi == 0x7fffffff) bi = mt.mt0 * 16;  // all values NaN: keep a valid index
+      p.lm_val[(size_t)tid * p.n_lm + t.idx] = bv;
+      p.lm_idx[(size_t)tid * p.n_lm + t.idx] = bi;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
 // Attention: one (sequence b, kv head g, split s).
 // ---------------------------------------------------------------------------
 // Split-KV attention: after writing its partial, a split arrives on the
@@ -829,10 +1233,15 @@ __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Sme
       }
       M = Mp;
     }
-    float *dst = L.att + (size_t)b * p.qdim + (g * rep + h) * D;
+    const int c0 = (g * rep + h) * D + d0;
+    float *dst = L.att + (size_t)b * p.qdim;
     const float inv = 1.f / den;
-    dst[d0] = n0 * inv;
-    dst[d0 + 32] = n1 * inv;
+    dst[c0] = n0 * inv;
+    dst[c0 + 32] = n1 * inv;
+    if (p.mma) {
+      put_opnd(L.attb, c0, b, p.nn, n0 * inv);
+      put_opnd(L.attb, c0 + 32, b, p.nn, n1 * inv);
+    }
   }
   return true;
 }
@@ -1095,6 +1504,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     const int head = a.g * rep + h;
     if (p.S == 1) {
       L.att[(size_t)a.b * p.qdim + head * D + d] = num / den;
+      if (p.mma) put_opnd(L.attb, head * D + d, a.b, p.nn, num / den);
     } else {
       float *dst = L.part + (((size_t)a.b * p.Hq + head) * p.S + a.s) * (D + 2);
       dst[d] = num;
@@ -1111,9 +1521,26 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
 // Online-softmax merge of the splits of one (sequence, kv head):
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
 __device__ void embed_task(const Params &p) {
+  if (!p.mma) {
+    for (int b = 0; b < p.B; ++b) {
+      const uint16_t *e = p.embed + (size_t)p.tokens_in[b] * p.H;
+      for (int i = threadIdx.x; i < p.H; i += kComputeThreads)
+        p.x0[(size_t)b * p.H + i] = bf2f(e[i]);
+    }
+    return;
+  }
+  // batch >= 2: also layer 0's QKV operand and its 16-row sums of squares
+  // (H is a multiple of 256, so every lane runs the same iterations)
+  const DevLayer &L0 = p.layers[0];
   for (int b = 0; b < p.B; ++b) {
     const uint16_t *e = p.embed + (size_t)p.tokens_in[b] * p.H;
-    for (int i = threadIdx.x; i < p.H; i += kComputeThreads) p.x0[(size_t)b * p.H + i] = bf2f(e[i]);
+    for (int i = threadIdx.x; i < p.H; i += kComputeThreads) {
+      const float x = bf2f(e[i]);
+      p.x0[(size_t)b * p.H + i] = x;
+      put_opnd(L0.xa, i, b, p.nn, x * bf2f(L0.attn_norm[i]));
+      const float s2 = half_warp_sum(x * x);
+      if ((threadIdx.x & 15) == 0) L0.ssa[(size_t)b * p.n_parts + (i >> 4)] = s2;
+    }
   }
 }
 
@@ -1140,6 +1567,10 @@ __device__ void argmax_task(const Params &p, uint32_t epoch) {
 // ---------------------------------------------------------------------------
 // The worker kernel
 // ---------------------------------------------------------------------------
+// kMma: projections on tensor cores (batch >= 2) instead of the CUDA-core
+// GEMV; the two modes are separate instantiations so that each gets its own
+// register allocation.
+template <bool kMma>
 __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const Smem sm = carve(smem_raw, p);
@@ -1202,16 +1633,21 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       switch (t.type) {
         case 1: ok = dw(); if (ok) embed_task(p); break;
         case 2: case 5: case 6: case 7: case 8: {
-          const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
-          const int nch = K >> 3;
-          const int cpt = nch <= kComputeThreads ? 1 : (nch + kComputeThreads - 1) / kComputeThreads;
-          const int rps = t.type == 2 ? p.rps_qkv : t.type == 5 ? p.rps_o : t.type == 6 ? p.rps_gu
-                        : t.type == 7 ? p.rps_down : p.rps_lm;
-          if (cpt == 1 && rps >= 8) ok = gemv_task<1, 8>(p, sm, t, k, id, dw);
-          else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id, dw);
-          else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id, dw);
-          else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id, dw);
-          else ok = gemv_task<kMaxCpt, 8>(p, sm, t, k, id, dw);
+          if constexpr (kMma) {
+            ok = p.nn == 2 ? mma_task<2>(p, sm, t, k, id, dw) : mma_task<1>(p, sm, t, k, id, dw);
+          } else {
+            const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
+            const int nch = K >> 3;
+            const int cpt =
+                nch <= kComputeThreads ? 1 : (nch + kComputeThreads - 1) / kComputeThreads;
+            const int rps = t.type == 2 ? p.rps_qkv : t.type == 5 ? p.rps_o
+                          : t.type == 6 ? p.rps_gu : t.type == 7 ? p.rps_down : p.rps_lm;
+            if (cpt == 1 && rps >= 8) ok = gemv_task<1, 8>(p, sm, t, k, id, dw);
+            else if (cpt == 2 && rps == 6) ok = gemv_task<2, 6>(p, sm, t, k, id, dw);
+            else if (cpt == 2 && rps >= 8) ok = gemv_task<2, 8>(p, sm, t, k, id, dw);
+            else if (cpt <= 6 && rps == 2) ok = gemv_task<6, 2>(p, sm, t, k, id, dw);
+            else ok = gemv_task<kMaxCpt, 8>(p, sm, t, k, id, dw);
+          }
           break;
         }
         case 3:
@@ -1259,31 +1695,78 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
   }
 }
 
+// Weight layout for the tensor-core path: a row-major [rows][K] bf16 matrix
+// to mma.sync A-fragment order.  Item (m-tile mt, k-block kb, lane) holds the
+// lane's 8 elements, so stage copies and fragment loads are 16 bytes per lane.
+// Rows >= rows (the last m-tile's padding) are zero.
+__global__ void frag_permute_kernel(uint4 *dst, const uint32_t *src, int rows, int K,
+                                    long long n_items) {
+  const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (item >= n_items) return;
+  const int lane = (int)(item & 31);
+  const long long blk = item >> 5;
+  const int KB = K >> 4;
+  const int mt = (int)(blk / KB), kb = (int)(blk - (long long)mt * KB);
+  const int r0 = mt * 16 + (lane >> 2), r1 = r0 + 8;
+  const int c = kb * 16 + 2 * (lane & 3);  // even: one 32-bit word holds (c, c + 1)
+  const size_t w = (size_t)K / 2;
+  uint4 o;
+  o.x = r0 < rows ? src[(size_t)r0 * w + c / 2] : 0u;
+  o.y = r1 < rows ? src[(size_t)r1 * w + c / 2] : 0u;
+  o.z = r0 < rows ? src[(size_t)r0 * w + c / 2 + 4] : 0u;
+  o.w = r1 < rows ? src[(size_t)r1 * w + c / 2 + 4] : 0u;
+  dst[item] = o;
+}
+
 }  // namespace
+
+// dst receives ceil(rows / 16) m-tiles of K / 16 fragment blocks (512 bytes each).
+cudaError_t permute_to_fragments(void *dst, const void *src, int rows, int K,
+                                 cudaStream_t stream) {
+  const long long n_items = (long long)((rows + 15) / 16) * (K / 16) * 32;
+  if (n_items == 0) return cudaSuccess;
+  const int threads = 256;
+  const long long blocks = (n_items + threads - 1) / threads;
+  frag_permute_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<uint4 *>(dst), static_cast<const uint32_t *>(src), rows, K, n_items);
+  return cudaGetLastError();
+}
 
 size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int rep_p) {
   return smem_offsets(stages, stage_bytes, pps, head_dim, rep_p).total;
 }
 
 cudaError_t worker_configure(size_t smem) {
-  return cudaFuncSetAttribute(mk_worker_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(mk_worker_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(mk_worker_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)smem);
 }
 
 cudaError_t worker_max_blocks(int *blocks, size_t smem) {
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, mk_worker_kernel, kThreads, smem);
+  int a = 0, b = 0;
+  cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, mk_worker_kernel<false>, kThreads, smem);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mk_worker_kernel<true>, kThreads, smem);
+  *blocks = a < b ? a : b;
+  return e;
 }
 
 // Persistent launch: one cooperative grid of `workers` CTAs.
 cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream) {
   void *args[] = {const_cast<Params *>(&p)};
-  return cudaLaunchCooperativeKernel((const void *)mk_worker_kernel, dim3(workers), dim3(kThreads),
-                                     args, smem, stream);
+  const void *fn = p.mma ? (const void *)mk_worker_kernel<true> : (const void *)mk_worker_kernel<false>;
+  return cudaLaunchCooperativeKernel(fn, dim3(workers), dim3(kThreads), args, smem, stream);
 }
 
 // Per-operator launch: one CTA per task of the operator.
 cudaError_t launch_tasks(const Params &p, int n_ctas, size_t smem, cudaStream_t stream) {
-  mk_worker_kernel<<<n_ctas, kThreads, smem, stream>>>(p);
+  if (p.mma)
+    mk_worker_kernel<true><<<n_ctas, kThreads, smem, stream>>>(p);
+  else
+    mk_worker_kernel<false><<<n_ctas, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,11 @@ constexpr int kRedRows = 256;          // GEMV rows whose warp partials shared m
 constexpr int kMaxRep = 8;             // q heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxBatch = 16;
+// Tensor-core projections (batch >= 2): mma.sync m16n8k16, bf16 in, fp32 out.
+constexpr int kMmaMaxMB = 6;    // 16-row m-tiles per row block (accumulators per warp)
+constexpr int kMmaMaxKPW = 3;   // 16-column k-blocks per warp and ring stage
+constexpr int kMmaMaxKCB = 8 * kMmaMaxKPW;  // k-blocks per ring stage
+constexpr int kMmaCredFloats = kComputeWarps * 4 * 16 * 9;  // cross-warp reduction buffer
 
 // Device status words: [0] status code, [1] task, [2] event, [3] block.
 enum DeviceStatus : int { kDevOk = 0, kDevTimeout = -6, kDevBadInput = -7 };
@@ -38,6 +43,8 @@ struct DevEvent {  // 16 bytes
 };
 
 // Per-layer device pointers: weight arena slices and activation buffers.
+// With batch >= 2 the four projection matrices are stored in mma.sync
+// A-fragment order (see frag_permute_kernel in the worker), not row-major.
 struct DevLayer {
   const uint16_t *w_qkv;   // [n_kv_heads * (rep + 2) * D][H], group-major rows
   const uint16_t *w_o;     // [H][Hq * D]
@@ -51,6 +58,19 @@ struct DevLayer {
   float *h;     // [B][F]  SiLU(gate) * up
   float *x_in;  // [B][H]  residual stream entering the layer
   float *x_out; // [B][H]  residual stream leaving the layer
+  // Batch >= 2 only: the projection inputs as two-term bf16 expansions
+  // (x = hi + lo) in mma.sync B-fragment order (see opnd_off in the worker),
+  // with the following RMSNorm's gain folded in, and per-16-row sums of
+  // squares [B][H / 16] of the streams that feed an RMSNorm.
+  uint16_t *xa;    // x_in * attn_norm   (QKV input)
+  float *ssa;      // sums of squares of x_in
+  uint16_t *attb;  // att                (O input)
+  uint16_t *xmb;   // xm * mlp_norm      (GATE_UP input)
+  float *ssm;      // sums of squares of xm
+  uint16_t *hb;    // h                  (DOWN input)
+  uint16_t *xa_next;  // DOWN epilogue targets: next layer's xa / ssa (or the
+  float *ssa_next;    // final hidden state's), with the gain of that norm
+  const uint16_t *gain_next;
 };
 
 struct Params {
@@ -86,6 +106,14 @@ struct Params {
   int qkv_rows, o_rows, gu_rows, down_rows, lm_rows, S, chunk, n_lm;
   int rps_qkv, rps_o, rps_gu, rps_down, rps_lm;  // GEMV rows per ring stage
   int pps;                                       // KV positions per ring stage
+  // tensor-core projections (batch >= 2)
+  int mma;      // 1: projections run on mma.sync with fragment-ordered weights
+  int nn;       // 8-sequence column tiles (1 or 2)
+  int n_parts;  // H / 16: sum-of-squares partials per sequence
+  int mb_qkv, mb_o, mb_gu, mb_down, mb_lm;        // m-tiles per row block
+  int kcb_qkv, kcb_o, kcb_gu, kcb_down, kcb_lm;   // k-blocks per ring stage
+  uint16_t *xfb;  // operand of the LM head: x_final * final_norm
+  float *ssf;     // sums of squares of x_final
   // ring
   int ring_stages, stage_bytes;
   int l2_prefetch_bytes;  // per worker: L2 prefetch distance ahead of the ring

@@ -3,29 +3,9 @@ import numpy as np
 import pytest
 
 import synth
-from gpu_helpers import Case, compare_step, torch
+from gpu_helpers import Case, compare_step, kv_rows_close, torch
 
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("built_libs")]
-
-
-def _kv_rows_close(case, ref_k, ref_v, lens, untouched=None):
-    """Rows appended at position lens[b]: the GPU's and the oracle's fp32 values
-    differ only in summation order, so after rounding to bf16 almost every
-    element is bit-identical and the rest differ by about one bf16 step of the
-    row's scale."""
-    gk = case.d_k.cpu().numpy().view(np.uint16)
-    gv = case.d_v.cpu().numpy().view(np.uint16)
-    for b in range(case.w.batch):
-        L = int(lens[b])
-        for arr_g, arr_r in ((gk, ref_k), (gv, ref_v)):
-            a = synth.bf16_to_f32(arr_g[:, b, :, L]).astype(np.float64)
-            r = synth.bf16_to_f32(arr_r[:, b, :, L]).astype(np.float64)
-            scale = np.max(np.abs(r), axis=-1, keepdims=True)
-            assert np.all(np.abs(a - r) <= 1e-2 * scale), "appended K/V row differs"
-            assert np.mean(arr_g[:, b, :, L] == arr_r[:, b, :, L]) > 0.9
-        # rows the steps never wrote are untouched
-        U = L if untouched is None else int(untouched[b])
-        np.testing.assert_array_equal(gk[:, b, :, :U], case.k[:, b, :, :U])
 
 
 @pytest.mark.parametrize("tied", [0, 1])
@@ -37,7 +17,7 @@ def test_tiny_step_matches_oracle(tied):
     ref = c.oracle_step(k=k, v=v, lens=lens)
     compare_step(ref, got, w, "tiny")
     np.testing.assert_array_equal(got["kv_len"], c.lens + 1)
-    _kv_rows_close(c, k, v, c.lens)
+    kv_rows_close(c, k, v, c.lens)
 
 
 def test_tiny_long_cache_uses_split_attention_and_merge():
@@ -100,7 +80,7 @@ def test_qwen3_06b_step_matches_oracle():
         ref = c.oracle_step(tokens=tok, k=k, v=v, lens=lens)
         compare_step(ref, got, w, f"0.6b step{step}")
         tok = ref["tokens"].copy()
-    _kv_rows_close(c, k, v, c.lens + 1, untouched=c.lens)
+    kv_rows_close(c, k, v, c.lens + 1, untouched=c.lens)
 
 
 def test_bad_inputs_are_rejected_and_write_nothing():
@@ -162,4 +142,4 @@ def test_qwen3_8b_bs1_full_size_step_matches_oracle():
     got = c.gpu_step()
     ref = c.oracle_step(k=k, v=v, lens=lens)
     compare_step(ref, got, w, "8b")
-    _kv_rows_close(c, k, v, c.lens)
+    kv_rows_close(c, k, v, c.lens)

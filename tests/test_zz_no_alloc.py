@@ -31,8 +31,9 @@ def _two_steps(case, fn):
     return out, case.d_k.cpu().numpy().copy(), case.d_v.cpu().numpy().copy()
 
 
-@pytest.mark.parametrize("w", [synth.TINY.with_(kv_len=300), synth.Q06B],
-                         ids=["tiny-split", "qwen3-0.6b"])
+@pytest.mark.parametrize("w", [synth.TINY.with_(kv_len=300), synth.Q06B,
+                               synth.TINY.with_(batch=5, kv_len=None, kv_len_range=(0, 300))],
+                         ids=["tiny-split", "qwen3-0.6b", "tiny-batch5"])
 def test_noalloc_step_matches_decode_step_twice(w):
     c = Case(w, seed=21, extra_cap=4)
     ref, ref_k, ref_v = _two_steps(c, c.mk.decode_step)
