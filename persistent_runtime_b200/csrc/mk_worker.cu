@@ -551,9 +551,11 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
   // L2 prefetch cursor (task pf_n, stage pf_st, global stage index pf_k) in
-  // the worker's stream of stages, across task boundaries.  While the
-  // producer is blocked on a full ring it prefetches the next stages into L2,
-  // up to l2_prefetch_bytes ahead of the ring.
+  // the worker's stream of stages, across task boundaries.  While the ring is
+  // full of landed stages that the compute warps have not consumed yet (they
+  // wait on an event or run a compute-heavy body, so HBM has spare capacity)
+  // the producer prefetches the next stages into L2, up to
+  // l2_prefetch_bytes ahead of the ring.
   const long long dist = p.l2_prefetch_bytes;
   int pf_n = 0, pf_st = 0;
   Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1, 0, 0, 0, 0, 0, 0};
@@ -587,7 +589,12 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
         while (!mbar_test(&sm.empty[slot], par)) {
           if (sm.ctl[kAbort]) goto out;
           ++spins;
-          if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count) {
+          // prefetch only while the consumer, not HBM, holds the ring back:
+          // the oldest stage in flight (this slot's previous use) has landed
+          // but is not released yet (the compute warps wait on an event or
+          // are busy with a compute-heavy body)
+          if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count &&
+              mbar_test(&sm.full[slot], par)) {
             if (pfs.nst < 0) pfs = task_stream(p, p.tasks[q.first + pf_n * q.stride]);
             if (pf_st >= pfs.nst) {
               ++pf_n;
@@ -1522,10 +1529,17 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
 __device__ void embed_task(const Params &p) {
   if (!p.mma) {
+    // 8 elements per 16-byte load (H is a multiple of 256: H / 2048 loads
+    // per thread)
+    const int nch = p.H >> 3;
     for (int b = 0; b < p.B; ++b) {
-      const uint16_t *e = p.embed + (size_t)p.tokens_in[b] * p.H;
-      for (int i = threadIdx.x; i < p.H; i += kComputeThreads)
-        p.x0[(size_t)b * p.H + i] = bf2f(e[i]);
+      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + (size_t)p.tokens_in[b] * p.H);
+      float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H);
+      for (int c = threadIdx.x; c < nch; c += kComputeThreads) {
+        const uint4 w = __ldg(e + c);
+        dst[2 * c] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+        dst[2 * c + 1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+      }
     }
     return;
   }
@@ -1544,22 +1558,42 @@ __device__ void embed_task(const Params &p) {
   }
 }
 
-__device__ void argmax_task(const Params &p, uint32_t epoch) {
-  const int b = threadIdx.x;
-  if (b < p.B) {
-    float bv = -INFINITY;
-    int bi = 0;
-    bool any = false;
-    for (int j = 0; j < p.n_lm; ++j) {
+// (value, index) a beats b: larger value, lower index on ties; NaN never
+// beats a number (all-NaN partials give the lowest index).
+__device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
+  if (av > bv) return true;
+  if (av == bv) return ai < bi;
+  return isnan(bv) && (!isnan(av) || ai < bi);
+}
+
+// One warp per sequence: lanes scan the LM-head partials (task order), then a
+// shuffle reduction with the same total order.
+__device__ __noinline__ void argmax_task(const Params &p, uint32_t epoch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int b = warp; b < p.B; b += kComputeWarps) {
+    float bv = NAN;
+    int bi = 0x7fffffff;
+    for (int j = lane; j < p.n_lm; j += 32) {
       const float v = __ldcg(p.lm_val + (size_t)b * p.n_lm + j);
-      if (!any || v > bv) {
+      const int i = __ldcg(p.lm_idx + (size_t)b * p.n_lm + j);
+      if (beats(v, i, bv, bi)) {
         bv = v;
-        bi = __ldcg(p.lm_idx + (size_t)b * p.n_lm + j);
-        any = true;
+        bi = i;
       }
     }
-    p.tokens_out[b] = bi;
-    p.kv_len[b] = p.kv_len[b] + 1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (beats(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      p.tokens_out[b] = bi;
+      p.kv_len[b] = p.kv_len[b] + 1;
+    }
   }
   if (threadIdx.x == 0 && p.persistent) *p.epoch = epoch;
 }
