@@ -96,6 +96,10 @@ typedef struct {
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring (0 = off) */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
+  int l2_stream_policy;      /* L2 policy of streamed weights and cached K/V: 0 or 1 =
+                                evict-first (default: they are read once per step and
+                                must not displace code, activations and counters),
+                                -1 = the normal policy */
 } mk_tuning;
 
 /* Weights: device pointers, bf16, row-major [out][in].  Per-layer arrays are

@@ -48,7 +48,7 @@ class Tuning(ctypes.Structure):
                 ("attn_tasks_per_worker", ctypes.c_int), ("attn_min_chunk", ctypes.c_int),
                 ("use_mma", ctypes.c_int), ("ring_stages", ctypes.c_int),
                 ("ring_stage_bytes", ctypes.c_int), ("l2_prefetch_bytes", ctypes.c_int),
-                ("wait_timeout_us", ctypes.c_uint)]
+                ("wait_timeout_us", ctypes.c_uint), ("l2_stream_policy", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)

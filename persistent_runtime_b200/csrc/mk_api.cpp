@@ -407,6 +407,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.ring_stages = t.ring_stages;
   p.stage_bytes = t.ring_stage_bytes;
   p.l2_prefetch_bytes = t.l2_prefetch_bytes;
+  p.evict_first = t.l2_stream_policy >= 0 ? 1 : 0;
   p.timeout_ns = (unsigned long long)t.wait_timeout_us * 1000ull;
   p.trace = nullptr;
   *out = h;

@@ -62,13 +62,25 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Global -> shared bulk copy completing on an mbarrier, with an L2 cache
+// policy (createpolicy) for the source lines.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar) {
+                                         uint64_t *bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// L2 policy for data read once per step: evict first (or the normal policy).
+__device__ __forceinline__ uint64_t stream_policy(bool evict_first) {
+  uint64_t pol;
+  if (evict_first)
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
@@ -231,7 +243,8 @@ struct Smem {
   uint8_t *ring;
   uint64_t *full, *empty;
   volatile int *ctl;
-  unsigned long long *tmark;  // [4] trace marks: prologue done, streaming done, ready
+  unsigned long long *tmark;  // [8] trace marks: prologue done, streaming done, ready,
+                              // L2 prefetch bytes, first ring stage available
   // GEMV scratch
   float *red;   // [kRedRows][kComputeWarps] warp partial sums of tile rows
   float *ss;    // [kComputeWarps]
@@ -269,7 +282,7 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   p += 4 * kCtlWords;
   p = align_to(p, 16);
   o.tmark = p;
-  p += 32;
+  p += 64;
   // GEMV scratch
   size_t g = p;
   o.red = g;
@@ -508,19 +521,20 @@ __device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
 // Issue the copies of stage st of stream s into ring slot dst (the full
 // barrier already expects stage_bytes_of(s, st) bytes).
 __device__ __forceinline__ void issue_stage(const Stream &s, int st, uint8_t *dst, int stage_bytes,
-                                            uint64_t *bar) {
+                                            uint64_t *bar, uint64_t pol) {
   if (s.nkc > 0) {
     const int rb = st / s.nkc, kc = st - rb * s.nkc;
     const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
     const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
     const uint32_t cb = (uint32_t)nkb * 512u;
     for (int i = 0; i < nm; ++i)
-      bulk_g2s(dst + (size_t)i * cb, s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb, bar);
+      bulk_g2s(dst + (size_t)i * cb, s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb, bar,
+               pol);
     return;
   }
   const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
-  bulk_g2s(dst, s.src0 + (size_t)st * s.stride, nb, bar);
-  if (s.src1) bulk_g2s(dst + stage_bytes / 2, s.src1 + (size_t)st * s.stride, nb, bar);
+  bulk_g2s(dst, s.src0 + (size_t)st * s.stride, nb, bar, pol);
+  if (s.src1) bulk_g2s(dst + stage_bytes / 2, s.src1 + (size_t)st * s.stride, nb, bar, pol);
 }
 
 // Prefetch stage st of stream s into L2; returns the bytes requested.
@@ -557,6 +571,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // the producer prefetches the next stages into L2, up to
   // l2_prefetch_bytes ahead of the ring.
   const long long dist = p.l2_prefetch_bytes;
+  const uint64_t pol = stream_policy(p.evict_first != 0);
   int pf_n = 0, pf_st = 0;
   Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1, 0, 0, 0, 0, 0, 0};
   uint32_t pf_k = 0;
@@ -620,7 +635,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       }
       uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes;
       mbar_arrive_expect_tx(&sm.full[slot], nb);
-      issue_stage(ts, st, dst, p.stage_bytes, &sm.full[slot]);
+      issue_stage(ts, st, dst, p.stage_bytes, &sm.full[slot], pol);
       if (dist > 0 && pf_k > k) ahead -= nb;  // stage k was prefetched
       ++k;
     }
@@ -652,6 +667,11 @@ __device__ __forceinline__ bool wait_full(const Params &p, const Smem &sm, uint3
     }
   }
   return true;
+}
+
+// Trace mark 4: the running task's first ring stage is available.
+__device__ __forceinline__ void trace_first_stage(const Params &p, const Smem &sm, int st) {
+  if (p.trace && st == 0 && threadIdx.x == 0) sm.tmark[4] = global_timer();
 }
 
 __device__ __forceinline__ void release_stage(const Smem &sm, const Params &p, uint32_t k) {
@@ -835,6 +855,7 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
     }
     const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
     if (got) {
+      trace_first_stage(p, sm, st);
       const uint16_t *ws =
           reinterpret_cast<const uint16_t *>(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
       if (active) {
@@ -1029,6 +1050,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
     const uint16_t *xn = xb + ((size_t)(kn * mt.kcb + warp) * NN) * 256;
     const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
     if (got) {
+      trace_first_stage(p, sm, st);
       const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
 #pragma unroll
       for (int j = 0; j < kMmaMaxKPW; ++j) {
@@ -1431,6 +1453,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     const int n = min(p.pps, cached - st * p.pps);
     const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
     if (!got) continue;
+    trace_first_stage(p, sm, st);
     const uint16_t *Ks =
         reinterpret_cast<const uint16_t *>(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
     const uint16_t *Vs = Ks + p.stage_bytes / 4;  // second half of the stage
@@ -1660,7 +1683,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       uint64_t t_wait = 0;
       if (p.trace && tid == 0) {
         t_wait = global_timer();
-        sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = 0;  // tmark[3] accumulates
+        sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = sm.tmark[4] = 0;  // tmark[3] accumulates
       }
       const DepWait dw{p, sm, t.dep, epoch, id};
       bool ok = true;
@@ -1709,6 +1732,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           tr[4] = sm.tmark[0];
           tr[5] = sm.tmark[1];
           tr[6] = sm.tmark[3];  // bytes this worker has prefetched into L2 so far
+          tr[7] = sm.tmark[4];  // the task's first ring stage was available
         }
       }
     }

@@ -117,6 +117,7 @@ struct Params {
   // ring
   int ring_stages, stage_bytes;
   int l2_prefetch_bytes;  // per worker: L2 prefetch distance ahead of the ring
+  int evict_first;        // 1: ring copies carry an L2 evict-first cache hint
   unsigned long long timeout_ns;
   // optional task trace: per task id {wait begin, ready, end, worker} (%globaltimer ns)
   unsigned long long *trace;

@@ -1,8 +1,9 @@
 """Per-task trace of the persistent kernel (see mk_set_trace in include/mk.h).
 
 Each task writes eight words: {wait begin, ready, end, (smid << 32) | worker,
-prologue done, streaming done, 0, 0} in %globaltimer nanoseconds (the two
-phase marks are 0 for tasks without those phases).  `summarize` reports where
+prologue done, streaming done, L2 prefetch bytes so far, first ring stage
+available} in %globaltimer nanoseconds (the phase marks are 0 for tasks
+without those phases).  `summarize` reports where
 worker time goes (waiting on events vs. prologue / streaming / epilogue of the
 task bodies) per task type; `to_chrome` writes the Chrome trace-event JSON
 format (one row per worker) for chrome://tracing or Perfetto.
@@ -24,12 +25,12 @@ def _fields(trace: np.ndarray):
     worker = t[:, 3] & 0xFFFFFFFF
     smid = t[:, 3] >> 32
     pro, loop = t[:, 4], t[:, 5]
-    return wait0, ready, end, worker, smid, pro, loop
+    return wait0, ready, end, worker, smid, pro, loop, t[:, 7]
 
 
 def summarize(trace: np.ndarray, graph) -> dict:
     """Wait / busy split of one traced step (all times in microseconds)."""
-    wait0, ready, end, worker, _, pro, loop = _fields(trace)
+    wait0, ready, end, worker, _, pro, loop, first = _fields(trace)
     ran = end > 0
     origin = int(wait0[ran].min())
     span = (int(end[ran].max()) - origin) / 1e3
@@ -51,6 +52,11 @@ def summarize(trace: np.ndarray, graph) -> dict:
             ent["prologue_us_mean"] = float(((pro - ready)[selh] / 1e3).mean())
             ent["stream_us_mean"] = float(((loop - pro)[selh] / 1e3).mean())
             ent["epilogue_us_mean"] = float(((end - loop)[selh] / 1e3).mean())
+        self_ = sel & (first > 0) & (pro > 0)
+        if self_.any():
+            # > 0: the first ring stage arrived after the prologue (HBM wait)
+            ent["first_stage_after_prologue_us_mean"] = float(
+                (np.maximum(first - pro, 0)[self_] / 1e3).mean())
         per_type[TASK_NAMES.get(int(ty), str(ty))] = ent
     ops = np.asarray(graph.task_op)[ran]
     r, e = ready[ran], end[ran]
@@ -70,7 +76,7 @@ def summarize(trace: np.ndarray, graph) -> dict:
 
 
 def to_chrome(trace: np.ndarray, graph, path: str) -> None:
-    wait0, ready, end, worker, smid, pro, loop = _fields(trace)
+    wait0, ready, end, worker, smid, pro, loop, first = _fields(trace)
     ran = end > 0
     origin = int(wait0[ran].min())
     ev = []
@@ -86,6 +92,7 @@ def to_chrome(trace: np.ndarray, graph, path: str) -> None:
                    "args": {"task": int(i), "layer": int(graph.task_layer[i]),
                             "idx": int(graph.task_idx[i]), "sm": int(smid[i]),
                             "prologue_us": float((pro[i] - ready[i]) / 1e3) if pro[i] else None,
-                            "stream_us": float((loop[i] - pro[i]) / 1e3) if loop[i] else None}})
+                            "stream_us": float((loop[i] - pro[i]) / 1e3) if loop[i] else None,
+                            "first_stage_us": float((first[i] - ready[i]) / 1e3) if first[i] else None}})
     with open(path, "w") as f:
         json.dump({"traceEvents": ev, "displayTimeUnit": "ns"}, f)
