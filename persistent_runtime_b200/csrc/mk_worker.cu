@@ -1215,7 +1215,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
 // loads at once; passes combine online.
 __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Smem &sm, int layer,
                                                       int b, int g) {
-  constexpr int kPass = 16;
+  constexpr int kPass = 24;  // splits merged per round trip
   compute_sync();  // every thread's partial stores precede the arrival
   uint32_t *ctr = p.arrivals + ((size_t)layer * p.B + b) * p.Hkv + g;
   if (threadIdx.x == 0) {
@@ -1236,27 +1236,30 @@ __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Sme
     const float *src = L.part + (((size_t)b * p.Hq + g * rep + h) * p.S) * (D + 2);
     float M = -INFINITY, den = 0.f, n0 = 0.f, n1 = 0.f;
     for (int s0 = 0; s0 < ns; s0 += kPass) {
-      float m[kPass], l[kPass], o0[kPass], o1[kPass];
+      // every load of the pass is issued before any is used: lane i holds
+      // split s0 + i's running max and sum, every lane its two dims of
+      // each split
+      const bool mine = lane < kPass && s0 + lane < ns;
+      const float *pl = src + (size_t)(s0 + lane) * (D + 2);
+      const float ml = mine ? __ldcg(pl + D) : -INFINITY;
+      const float ll = mine ? __ldcg(pl + D + 1) : 0.f;
+      float o0[kPass], o1[kPass];
 #pragma unroll
       for (int i = 0; i < kPass; ++i) {
         const bool ok = s0 + i < ns;
         const float *ps = src + (size_t)(s0 + i) * (D + 2);
-        m[i] = ok ? __ldcg(ps + D) : -INFINITY;
-        l[i] = ok ? __ldcg(ps + D + 1) : 0.f;
         o0[i] = ok ? __ldcg(ps + d0) : 0.f;
         o1[i] = ok ? __ldcg(ps + d0 + 32) : 0.f;
       }
-      float Mp = M;
-#pragma unroll
-      for (int i = 0; i < kPass; ++i) Mp = fmaxf(Mp, m[i]);
+      const float Mp = fmaxf(M, warp_max(ml));
       const float r = M == -INFINITY ? 0.f : __expf(M - Mp);
-      den *= r;
+      const float wl = ml == -INFINITY ? 0.f : __expf(ml - Mp);
+      den = den * r + warp_sum(wl * ll);
       n0 *= r;
       n1 *= r;
 #pragma unroll
       for (int i = 0; i < kPass; ++i) {
-        const float w = m[i] == -INFINITY ? 0.f : __expf(m[i] - Mp);
-        den = fmaf(w, l[i], den);
+        const float w = __shfl_sync(0xffffffffu, wl, i);
         n0 = fmaf(w, o0[i], n0);
         n1 = fmaf(w, o1[i], n1);
       }
