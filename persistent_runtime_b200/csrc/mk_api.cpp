@@ -2,11 +2,13 @@
 #include "mk.h"
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -40,10 +42,9 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   if (d.col_align <= 0) d.col_align = 16;
   if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 4;
   if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
-  // the same bytes in flight per SM; the tensor-core tiles of batch >= 2 use
-  // more, smaller stages (at most 24 k-blocks per stage)
-  if (d.ring_stages <= 0) d.ring_stages = batch > 1 ? 8 : 4;
-  if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = (batch > 1 ? 24 : 48) * 1024;
+  (void)batch;
+  if (d.ring_stages <= 0) d.ring_stages = 4;
+  if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
   if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
   return d;
@@ -162,6 +163,10 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   mk_tuning &t = h->tune;
   const mk_model_config &c = *cfg;
   const int D = c.head_dim;
+  if (t.ring_stages > 16) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "at most 16 ring stages");
+  }
   if (t.ring_stage_bytes % 1024) {
     delete h;
     return fail(nullptr, MK_ERR_ARG, "ring_stage_bytes must be a multiple of 1024");
@@ -175,7 +180,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   // shared memory: shrink the stage size until the CTA fits
   size_t smem = 0;
   for (;;) {
-    const int pps = t.ring_stage_bytes / (4 * D);
+    const int pps = std::min(256, t.ring_stage_bytes / (4 * D) / 8 * 8);
     smem = mk::worker_smem_bytes(t.ring_stages, t.ring_stage_bytes, pps, D, rep_p);
     if ((int)smem <= smem_optin) break;
     t.ring_stage_bytes -= 1024;
@@ -376,7 +381,14 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.rps_gu = std::max(2, rps(H) & ~1);
   p.rps_down = rps(F);
   p.rps_lm = rps(H);
-  p.pps = t.ring_stage_bytes / (4 * D);
+  // KV positions per stage: K and V of pps rows each, a multiple of 8 (whole
+  // 1024-byte swizzle atoms), at most 256 (the TMA box height limit) and at
+  // most one split (a multiple of 64), so a short split is one exact box
+  p.pps = std::min(std::min(256, T.attn_chunk), t.ring_stage_bytes / (4 * D) / 8 * 8);
+  if (p.pps < 8) {
+    mk_destroy(h);
+    return fail(nullptr, MK_ERR_ARG, "ring stage smaller than 8 K/V rows");
+  }
   if (mma) {
     // m-tiles per row block: the task's rows up to the accumulator limit;
     // k-blocks per stage: what the stage holds for that many m-tiles, a
@@ -571,6 +583,50 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
   return MK_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+}  // namespace
+
+std::string mk::encode_kv_maps(const mk_handle *h, const void *kc, const void *vc, Params *p) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return "cuTensorMapEncodeTiled is not available from the driver";
+  const mk_model_config &c = h->cfg;
+  if ((reinterpret_cast<uintptr_t>(kc) | reinterpret_cast<uintptr_t>(vc)) & 15)
+    return "K/V caches must be 16-byte aligned";
+  const cuuint64_t rows = (cuuint64_t)c.n_layers * c.batch * c.n_kv_heads * c.kv_capacity;
+  const cuuint64_t dims[2] = {(cuuint64_t)c.head_dim, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)h->base.pps};
+  const cuuint32_t estride[2] = {1u, 1u};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = enc(i == 0 ? &p->tmap_k : &p->tmap_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(i == 0 ? kc : vc), dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")";
+  }
+  return "";
+}
+
+extern "C" {
+
 static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int32_t *kvl,
                            void *kc, void *vc, Params *p) {
   if (!h) return fail(nullptr, MK_ERR_ARG, "null handle");
@@ -583,6 +639,10 @@ static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int3
   p->kv_len = kvl;
   p->k_cache = static_cast<uint16_t *>(kc);
   p->v_cache = static_cast<uint16_t *>(vc);
+  if (h->base.mma) {  // only the batched kernel reads K/V through tensor maps
+    const std::string e = mk::encode_kv_maps(h, kc, vc, p);
+    if (!e.empty()) return fail(h, MK_ERR_ARG, e);
+  }
   return MK_OK;
 }
 

@@ -21,6 +21,14 @@ cudaError_t permute_to_fragments(void *dst, const void *src, int rows, int K,
                                  cudaStream_t stream);
 }  // namespace mk
 
+struct mk_handle;
+namespace mk {
+// Encodes p->tmap_k / p->tmap_v for the caches of one step; returns "" or
+// the reason it failed.
+std::string encode_kv_maps(const mk_handle *h, const void *k_cache, const void *v_cache,
+                           Params *p);
+}  // namespace mk
+
 struct mk_handle {
   mk_model_config cfg{};
   mk_tuning tune{};

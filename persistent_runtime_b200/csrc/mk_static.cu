@@ -205,6 +205,11 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
   p.kv_len = d_kv_len;
   p.k_cache = static_cast<uint16_t *>(d_k_cache);
   p.v_cache = static_cast<uint16_t *>(d_v_cache);
+  const std::string me = p.mma ? mk::encode_kv_maps(h, d_k_cache, d_v_cache, &p) : "";
+  if (!me.empty()) {
+    h->err = me;
+    return MK_ERR_ARG;
+  }
   p.logits = d_logits;
   p.persistent = 1;
   e = mk::launch_persistent(p, h->tune.num_workers, h->smem, st);

@@ -73,6 +73,17 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// 2-D tiled TMA load of the box at (x, y) of a tensor map (kernel parameter
+// space) into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // L2 policy for data read once per step: evict first (or the normal policy).
 __device__ __forceinline__ uint64_t stream_policy(bool evict_first) {
   uint64_t pol;
@@ -209,6 +220,39 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, const ui
       "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y));
+}
+
+// m16n8k8 variant (A 16 x 8: two registers, B 8 x 8: one register).
+__device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5}, {%6}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b));
+}
+
+// m16n8k16 with the A rows g + 8 zero (a1 = a3 = 0).
+__device__ __forceinline__ void mma_bf16_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                             uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// Four 8 x 8 b16 matrices from shared memory; lanes 8i..8i+7 give the row
+// addresses of matrix i.  Plain: thread l receives row l / 4, columns
+// 2 (l % 4) and 2 (l % 4) + 1; .trans: rows 2 (l % 4), 2 (l % 4) + 1 of
+// column l / 4.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
 // Activation operands are two-term bf16 expansions x = hi + lo, hi = bf16(x),
@@ -461,19 +505,24 @@ __device__ __forceinline__ size_t kv_row(const Params &p, int layer, int b, int 
 // Everything the producer needs to stream one task, computed once per task so
 // that issuing a stage is pure address arithmetic (no dependent loads).
 struct Stream {
-  const uint8_t *src0, *src1;  // stage 0 sources (src1: V rows of attention, else null)
-  uint32_t bytes, last_bytes;  // bytes of a full / of the last stage (per source)
-  uint32_t stride;             // bytes between consecutive stages of one source
-  int nst;                     // stages
+  const uint8_t *src0 = nullptr;  // stage 0 source (weights)
+  uint32_t bytes = 0, last_bytes = 0;  // bytes of a full / of the last stage
+  uint32_t stride = 0;            // bytes between consecutive stages
+  int nst = 0;                    // stages
   // tensor-core projections: stage st = (row block st / nkc, k chunk st % nkc)
-  int nkc;                     // 0 for the plain streams above
-  int KB, mt0, mt1, mb, kcb;
+  int nkc = 0;                    // 0 for the other streams
+  int KB = 0, mt0 = 0, mt1 = 0, mb = 0, kcb = 0;
+  // attention: K/V rows y0 + st * pps .. of the 2-D cache tensor maps
+  int kv = 0;
+  int y0 = 0;
 };
 
+// kMma: the batched kernel (tensor-core tiles, swizzled TMA K/V boxes).
+template <bool kMma>
 __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t) {
-  Stream s{nullptr, nullptr, 0u, 0u, 0u, 0, 0, 0, 0, 0, 0, 0};
+  Stream s{};
   const int type = t.type;
-  if (p.mma && (type == 2 || (type >= 5 && type <= 8))) {
+  if (kMma && (type == 2 || (type >= 5 && type <= 8))) {
     const MmaTile m = mma_tile(p, type, t.layer, (int)t.idx);
     s.src0 = reinterpret_cast<const uint8_t *>(m.w);
     s.nst = m.nrb * m.nkc;
@@ -486,15 +535,16 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
     return s;
   }
   if (type == 3) {
+    // whole boxes of pps rows (the last stage reads past the split: masked)
     const AttnSpan a = attn_span(p, (int)t.idx);
     const int n = a.cached_end - a.p0;
     if (n <= 0) return s;
     s.nst = (n + p.pps - 1) / p.pps;
-    const size_t off = kv_row(p, t.layer, a.b, a.g, a.p0);
-    s.src0 = reinterpret_cast<const uint8_t *>(p.k_cache + off);
-    s.src1 = reinterpret_cast<const uint8_t *>(p.v_cache + off);
-    s.stride = s.bytes = (uint32_t)(p.pps * p.D * 2);
-    s.last_bytes = (uint32_t)((n - (s.nst - 1) * p.pps) * p.D * 2);
+    s.kv = 1;
+    s.y0 = (int)(kv_row(p, t.layer, a.b, a.g, a.p0) / p.D);
+    s.bytes = s.last_bytes = (uint32_t)(p.pps * p.D * 2);
+    // batch 1: plain row copies of exactly the cached rows
+    if (!kMma) s.last_bytes = (uint32_t)((n - (s.nst - 1) * p.pps) * p.D * 2);
   } else if (type == 2 || (type >= 5 && type <= 8)) {
     const Gemv g = gemv_of(p, type, t.layer, (int)t.idx);
     const int rows = g.row1 - g.row0;
@@ -507,22 +557,40 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
 }
 
 // Bytes that stage st of stream s lands in the ring.
+template <bool kMma>
 __device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
-  if (s.nkc > 0) {
+  if (kMma && s.nkc > 0) {
     const int rb = st / s.nkc, kc = st - rb * s.nkc;
     const int nm = min(s.mb, s.mt1 - (s.mt0 + rb * s.mb));
     const int nkb = min(s.kcb, s.KB - kc * s.kcb);
     return (uint32_t)(nm * nkb * 512);
   }
-  const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
-  return s.src1 ? 2 * nb : nb;
+  if (s.kv) return 2 * (st == s.nst - 1 ? s.last_bytes : s.bytes);  // K and V
+  return st == s.nst - 1 ? s.last_bytes : s.bytes;
 }
 
 // Issue the copies of stage st of stream s into ring slot dst (the full
 // barrier already expects stage_bytes_of(s, st) bytes).
-__device__ __forceinline__ void issue_stage(const Stream &s, int st, uint8_t *dst, int stage_bytes,
+template <bool kMma>
+__device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, int st, uint8_t *dst,
                                             uint64_t *bar, uint64_t pol) {
-  if (s.nkc > 0) {
+  if (s.kv) {
+    const int y = s.y0 + st * p.pps;
+    if (!kMma) {  // plain rows: K at dst, V pps rows further
+      const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
+      bulk_g2s(dst, p.k_cache + (size_t)y * p.D, nb, bar, pol);
+      bulk_g2s(dst + s.bytes, p.v_cache + (size_t)y * p.D, nb, bar, pol);
+      return;
+    }
+    // K boxes (64 dims x pps rows, 128-byte swizzle) at dst, V boxes after them
+    const uint32_t box = (uint32_t)p.pps * 128u;
+    for (int h = 0; h < (p.D >> 6); ++h) {
+      tma_load_2d(dst + h * box, &p.tmap_k, 64 * h, y, bar, pol);
+      tma_load_2d(dst + s.bytes + h * box, &p.tmap_v, 64 * h, y, bar, pol);
+    }
+    return;
+  }
+  if (kMma && s.nkc > 0) {
     const int rb = st / s.nkc, kc = st - rb * s.nkc;
     const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
     const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
@@ -534,12 +602,12 @@ __device__ __forceinline__ void issue_stage(const Stream &s, int st, uint8_t *ds
   }
   const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
   bulk_g2s(dst, s.src0 + (size_t)st * s.stride, nb, bar, pol);
-  if (s.src1) bulk_g2s(dst + stage_bytes / 2, s.src1 + (size_t)st * s.stride, nb, bar, pol);
 }
 
 // Prefetch stage st of stream s into L2; returns the bytes requested.
+template <bool kMma>
 __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
-  if (s.nkc > 0) {
+  if (kMma && s.nkc > 0) {
     const int rb = st / s.nkc, kc = st - rb * s.nkc;
     const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
     const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
@@ -547,10 +615,10 @@ __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
     for (int i = 0; i < nm; ++i) prefetch_l2(s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb);
     return cb * (uint32_t)nm;
   }
+  if (s.kv) return 0u;  // K/V tiles are not prefetched
   const uint32_t pb = st == s.nst - 1 ? s.last_bytes : s.bytes;
   prefetch_l2(s.src0 + (size_t)st * s.stride, pb);
-  if (s.src1) prefetch_l2(s.src1 + (size_t)st * s.stride, pb);
-  return s.src1 ? 2 * pb : pb;
+  return pb;
 }
 
 // ---------------------------------------------------------------------------
@@ -560,6 +628,7 @@ struct Queue {
   int first, stride, count;  // tasks first, first + stride, ... (count of them)
 };
 
+template <bool kMma>
 __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const int NS = p.ring_stages;
   uint32_t k = 0;
@@ -573,17 +642,18 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const long long dist = p.l2_prefetch_bytes;
   const uint64_t pol = stream_policy(p.evict_first != 0);
   int pf_n = 0, pf_st = 0;
-  Stream pfs{nullptr, nullptr, 0u, 0u, 0u, -1, 0, 0, 0, 0, 0, 0};
+  Stream pfs{};
+  pfs.nst = -1;
   uint32_t pf_k = 0;
   long long ahead = 0;
   for (int n = 0; n < q.count; ++n) {
-    const Stream ts = task_stream(p, p.tasks[q.first + n * q.stride]);
+    const Stream ts = task_stream<kMma>(p, p.tasks[q.first + n * q.stride]);
     for (int st = 0; st < ts.nst; ++st) {
-      const uint32_t nb = stage_bytes_of(ts, st);
+      const uint32_t nb = stage_bytes_of<kMma>(ts, st);
       if (dist > 0) {
         // stages before k were issued without a prefetch: move the cursor on
         while (pf_k < k && pf_n < q.count) {
-          if (pfs.nst < 0) pfs = task_stream(p, p.tasks[q.first + pf_n * q.stride]);
+          if (pfs.nst < 0) pfs = task_stream<kMma>(p, p.tasks[q.first + pf_n * q.stride]);
           if (pf_st >= pfs.nst) {
             ++pf_n;
             pf_st = 0;
@@ -610,13 +680,13 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
           // are busy with a compute-heavy body)
           if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count &&
               mbar_test(&sm.full[slot], par)) {
-            if (pfs.nst < 0) pfs = task_stream(p, p.tasks[q.first + pf_n * q.stride]);
+            if (pfs.nst < 0) pfs = task_stream<kMma>(p, p.tasks[q.first + pf_n * q.stride]);
             if (pf_st >= pfs.nst) {
               ++pf_n;
               pf_st = 0;
               pfs.nst = -1;
             } else {
-              const uint32_t pb = prefetch_stage(pfs, pf_st);
+              const uint32_t pb = prefetch_stage<kMma>(pfs, pf_st);
               ahead += pb;
               if (p.trace) sm.tmark[3] += pb;
               ++pf_st;
@@ -635,7 +705,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       }
       uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes;
       mbar_arrive_expect_tx(&sm.full[slot], nb);
-      issue_stage(ts, st, dst, p.stage_bytes, &sm.full[slot], pol);
+      issue_stage<kMma>(p, ts, st, dst, &sm.full[slot], pol);
       if (dist > 0 && pf_k > k) ahead -= nb;  // stage k was prefetched
       ++k;
     }
@@ -1278,6 +1348,262 @@ __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Sme
   return true;
 }
 
+// bf16 pair (lo element in the low half) and its rounding remainder pair:
+// x = hi + lo to about 16 significant bits (see opnd_off).
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const uint16_t h0 = f2bf(x0), h1 = f2bf(x1);
+  hi = (uint32_t)h0 | ((uint32_t)h1 << 16);
+  lo = (uint32_t)f2bf(x0 - bf2f(h0)) | ((uint32_t)f2bf(x1 - bf2f(h1)) << 16);
+}
+
+// One block of 8 positions [j0, j0 + 8) of a K/V tile (rows of D bf16) for
+// one warp, on tensor cores.  Query heads are the rows of the MMA (up to 8,
+// zero padded to 16), positions its columns:
+//   S  = Q K^T        m16n8k16, K fragments by ldmatrix from the row-major tile
+//   P  = exp(S - m)   online softmax on the accumulator fragments: head g's 8
+//                     scores sit in the 4 lanes of quad g (2 each)
+//   O^T += V^T P^T    m16n8k8, V fragments by ldmatrix.trans; the B fragment
+//                     of P^T is the lane's own pair of probabilities
+// Q and P enter as hi/lo bf16 pairs (two MMAs each); K and V are exact bf16.
+// Positions >= n are masked; their rows are read from position n - 1 so
+// every value stays finite.  Lane (g, t) keeps head g's running max and sum
+// (m_run, l_run) and o[j] = O^T rows (16 j + g, 16 j + g + 8), heads
+// (2 t, 2 t + 1).
+// Byte offset of (row r, 16-byte chunk c16 of the head dims) in a K or V
+// tile.  SWZ: D / 64 TMA boxes of 64 dims x `rows` rows with the 128-byte
+// swizzle (chunk c of row r stored at chunk c ^ (r mod 8) of its 128-byte
+// line; conflict-free for 8 consecutive rows); else plain row-major rows.
+template <int D, bool SWZ>
+__device__ __forceinline__ uint32_t kv_off(int r, int c16, int rows) {
+  if (!SWZ) return (uint32_t)(r * D * 2 + c16 * 16);
+  return (uint32_t)((c16 >> 3) * rows * 128 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
+}
+
+template <int D, bool SWZ>
+__device__ __forceinline__ void attn_block_mma(uint32_t kbase, uint32_t vbase, int rows, int j0,
+                                               int n, const uint32_t (&qh)[D / 16][2],
+                                               const uint32_t (&ql)[D / 16][2], float &m_run,
+                                               float &l_run, float (&o)[D / 16][4]) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  // ldmatrix rows: 8 consecutive positions (distinct r mod 8: no bank conflicts)
+  const int pos = min(j0 + (lane & 7), n - 1);
+  const int mat = lane >> 3;  // the 8 x 8 matrix this lane addresses
+  // four independent accumulation chains (hi/lo x even/odd k-step), summed
+  float sa[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sa[i][0] = sa[i][1] = sa[i][2] = sa[i][3] = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {  // 32 dims (two k-steps) per ldmatrix.x4
+    uint32_t b[4];
+    ldmatrix_x4(b, kbase + kv_off<D, SWZ>(pos, 4 * c + mat, rows));
+    mma_bf16_top(sa[0], qh[2 * c][0], qh[2 * c][1], b[0], b[1]);
+    mma_bf16_top(sa[1], ql[2 * c][0], ql[2 * c][1], b[0], b[1]);
+    mma_bf16_top(sa[2], qh[2 * c + 1][0], qh[2 * c + 1][1], b[2], b[3]);
+    mma_bf16_top(sa[3], ql[2 * c + 1][0], ql[2 * c + 1][1], b[2], b[3]);
+  }
+  float s[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) s[i] = (sa[0][i] + sa[2][i]) + (sa[1][i] + sa[3][i]);
+  const bool v0 = j0 + 2 * t < n, v1 = j0 + 2 * t + 1 < n;
+  const float s0 = v0 ? s[0] : -INFINITY, s1 = v1 ? s[1] : -INFINITY;
+  float mx = fmaxf(s0, s1);
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float m_new = fmaxf(m_run, mx);  // finite: position j0 < n is valid
+  const float alpha = m_run == -INFINITY ? 0.f : __expf(m_run - m_new);
+  const float p0 = v0 ? __expf(s0 - m_new) : 0.f, p1 = v1 ? __expf(s1 - m_new) : 0.f;
+  float sum = p0 + p1;
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  l_run = l_run * alpha + sum;
+  m_run = m_new;
+  uint32_t ph, pl;
+  split_pair(p0, p1, ph, pl);
+  // rescale factors of the heads 2t, 2t + 1 this lane accumulates
+  const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * t);
+  const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
+#pragma unroll
+  for (int j = 0; j < D / 16; ++j) {
+    o[j][0] *= a0;
+    o[j][1] *= a1;
+    o[j][2] *= a0;
+    o[j][3] *= a1;
+  }
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {  // two 16-dim m-tiles per ldmatrix.x4.trans
+    uint32_t v[4];
+    ldmatrix_x4_trans(v, vbase + kv_off<D, SWZ>(pos, 4 * c + mat, rows));
+    mma_bf16_k8(o[2 * c], v[0], v[1], ph);
+    mma_bf16_k8(o[2 * c], v[0], v[1], pl);
+    mma_bf16_k8(o[2 * c + 1], v[2], v[3], ph);
+    mma_bf16_k8(o[2 * c + 1], v[2], v[3], pl);
+  }
+}
+
+// Decode attention for one (sequence b, kv head g, split s): q/k RMSNorm and
+// RoPE prologue, K/V append, then every warp runs flash-decoding style over
+// its own 8-position blocks on tensor cores (no CTA barrier inside the loop)
+// and the warps' states are merged once at the end.  D: head dim (64, 128);
+// SWZ: the K/V tiles arrive as swizzled TMA boxes (else as plain rows).
+template <int D, bool SWZ>
+__device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
+                                          uint32_t &k, int task_id, const DepWait &dep_wait) {
+  constexpr int NP = 8;  // positions per warp block
+  const AttnSpan a = attn_span(p, (int)t.idx);
+  if (!a.active) {  // the split starts past the new row: it only arrives
+    if (!dep_wait()) return false;
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rep = p.rep;
+  constexpr int dpl = D >> 5;
+  const DevLayer &L = p.layers[t.layer];
+  const float *qkv = L.qkv + (size_t)a.b * p.n_qkv + (size_t)a.g * p.grp;
+  const float *rope = p.rope + (size_t)a.L * D;  // [D/2][2]
+  // gains and RoPE factors of this lane's dims: independent of the step's
+  // results, so loaded before the wait
+  float gq[4], gk[4], rc[2], rs[2];
+  for (int i = 0; i < dpl; ++i) {
+    gq[i] = bf2f(L.q_norm[lane + 32 * i]);
+    gk[i] = bf2f(L.k_norm[lane + 32 * i]);
+  }
+  for (int i = 0; i < (dpl >> 1); ++i) {
+    rc[i] = rope[2 * (lane + 32 * i)];
+    rs[i] = rope[2 * (lane + 32 * i) + 1];
+  }
+  if (!dep_wait()) return false;
+
+  // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
+  // holds position L; v is only rounded)
+  for (int row = warp; row < rep + 2; row += kComputeWarps) {
+    if (row >= rep && !a.has_new) continue;
+    float v[4];
+    for (int i = 0; i < dpl; ++i) v[i] = __ldcg(qkv + row * D + lane + 32 * i);
+    if (row <= rep) {  // q heads and k
+      float ss = 0.f;
+      for (int i = 0; i < dpl; ++i) ss = fmaf(v[i], v[i], ss);
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss / (float)D + p.eps);
+      for (int i = 0; i < dpl; ++i) v[i] = v[i] * inv * (row < rep ? gq[i] : gk[i]);
+      const int hp = dpl >> 1;  // dims lane + 32 i pair with lane + 32 (i + hp)
+      for (int i = 0; i < hp; ++i) {
+        const float c = rc[i], s = rs[i];
+        const float x0 = v[i], x1 = v[i + hp];
+        v[i] = x0 * c - x1 * s;
+        v[i + hp] = x1 * c + x0 * s;
+      }
+    }
+    if (row < rep) {
+      for (int i = 0; i < dpl; ++i) sm.q[row * kMaxHeadDim + lane + 32 * i] = v[i] * p.attn_scale;
+    } else {
+      uint16_t *cache = row == rep ? p.k_cache : p.v_cache;
+      uint16_t *dst = row == rep ? sm.knew : sm.vnew;
+      const size_t off = kv_row(p, t.layer, a.b, a.g, a.L);
+      for (int i = 0; i < dpl; ++i) {
+        const uint16_t hb = f2bf(v[i]);
+        cache[off + lane + 32 * i] = hb;
+        dst[lane + 32 * i] = hb;
+      }
+    }
+  }
+  compute_sync();
+  // Q fragments (rows = heads, zero from rep on) as hi/lo bf16 pairs
+  const int gq_row = lane >> 2, tq = lane & 3;
+  uint32_t qh[D / 16][2], ql[D / 16][2];
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c = 16 * kk + 2 * tq + 8 * half;
+      const bool ok = gq_row < rep;
+      const float x0 = ok ? sm.q[gq_row * kMaxHeadDim + c] : 0.f;
+      const float x1 = ok ? sm.q[gq_row * kMaxHeadDim + c + 1] : 0.f;
+      split_pair(x0, x1, qh[kk][half], ql[kk][half]);
+    }
+  }
+  float o[D / 16][4];
+#pragma unroll
+  for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  trace_mark(p, sm, 0);
+
+  const int cached = a.cached_end - a.p0;
+  const int nst = cached > 0 ? (cached + p.pps - 1) / p.pps : 0;
+  for (int st = 0; st < nst; ++st) {
+    const int n = min(p.pps, cached - st * p.pps);
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (!got) continue;
+    trace_first_stage(p, sm, st);
+    const uint32_t kb = smem_u32(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
+    const uint32_t vb = kb + (uint32_t)(p.pps * D * 2);  // V boxes follow the K boxes
+    for (int j0 = warp * NP; j0 < n; j0 += kComputeWarps * NP)
+      attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, qh, ql, m_run, l_run, o);
+    release_stage(sm, p, k);
+    ++k;
+  }
+  // the new row: one more block, on the warp after the last cached block
+  if (a.has_new && warp == ((cached + NP - 1) / NP) % kComputeWarps)
+    attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, qh, ql, m_run, l_run, o);
+
+  trace_mark(p, sm, 1);
+  // every warp's state to shared memory: o (heads 2 tq, 2 tq + 1), then the
+  // running max and sum of head gq_row
+  static_assert(kStateSlots == kComputeWarps, "one state slot per warp");
+  const int stride = D + 2;
+  {
+    float *st_w = sm.ored + (size_t)warp * p.rep_p * stride;
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      const int d = 16 * j + gq_row;
+      if (h0 < rep) {
+        st_w[h0 * stride + d] = o[j][0];
+        st_w[h0 * stride + d + 8] = o[j][2];
+      }
+      if (h1 < rep) {
+        st_w[h1 * stride + d] = o[j][1];
+        st_w[h1 * stride + d + 8] = o[j][3];
+      }
+    }
+    if (tq == 0 && gq_row < rep) {
+      st_w[gq_row * stride + D] = m_run;
+      st_w[gq_row * stride + D + 1] = l_run;
+    }
+  }
+  compute_sync();
+  if (sm.ctl[kAbort]) return false;
+  for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
+    const int h = oi / D, d = oi - h * D;
+    float M = -INFINITY;
+    for (int w = 0; w < kStateSlots; ++w)
+      M = fmaxf(M, sm.ored[((size_t)w * p.rep_p + h) * stride + D]);
+    float num = 0.f, den = 0.f;
+    for (int w = 0; w < kStateSlots; ++w) {
+      const float *sw = sm.ored + ((size_t)w * p.rep_p + h) * stride;
+      const float mw = sw[D];
+      const float e = mw == -INFINITY ? 0.f : __expf(mw - M);
+      den = fmaf(e, sw[D + 1], den);
+      num = fmaf(e, sw[d], num);
+    }
+    const int head = a.g * rep + h;
+    if (p.S == 1) {
+      L.att[(size_t)a.b * p.qdim + head * D + d] = num / den;
+      if (p.mma) put_opnd(L.attb, head * D + d, a.b, p.nn, num / den);
+    } else {
+      float *dst = L.part + (((size_t)a.b * p.Hq + head) * p.S + a.s) * (D + 2);
+      dst[d] = num;
+      if (d == 0) {
+        dst[D] = M;
+        dst[D + 1] = den;
+      }
+    }
+  }
+  if (p.S == 1) return true;
+  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+}
+
 // One block of up to NP = 32 / RP positions for one warp: scores, online
 // softmax update of the warp's running state, and PV.  RP = q heads per kv head
 // rounded up to a power of two (heads >= rep are padding).  Lane l covers dims
@@ -1369,12 +1695,14 @@ __device__ __forceinline__ void attn_block(const Params &p, float *pw, float *aw
   __syncwarp();
 }
 
-// Decode attention for one (sequence b, kv head g, split s): q/k RMSNorm and
-// RoPE prologue, K/V append, then every warp runs flash-decoding style over
-// its own positions (no CTA barrier inside the loop) and the warps' states
-// are merged once at the end.
+// Decode attention for one (sequence b, kv head g, split s) on CUDA cores
+// (the batch-1 kernel): q/k RMSNorm and RoPE prologue, K/V append, then every
+// warp runs flash-decoding style over its own positions (no CTA barrier
+// inside the loop) and the warps' states are merged once at the end.  At
+// batch 1 a split is one 8-position block per warp and the step is bound by
+// the weight stream; this body keeps the batch-1 kernel's register budget.
 template <int RP>
-__device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
+__device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, const DevTask &t,
                                           uint32_t &k, int task_id, const DepWait &dep_wait) {
   constexpr int NP = 32 / RP;
   const AttnSpan a = attn_span(p, (int)t.idx);
@@ -1459,7 +1787,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     trace_first_stage(p, sm, st);
     const uint16_t *Ks =
         reinterpret_cast<const uint16_t *>(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
-    const uint16_t *Vs = Ks + p.stage_bytes / 4;  // second half of the stage
+    const uint16_t *Vs = Ks + (size_t)p.pps * p.D;  // V rows follow the pps K rows
     for (int j0 = warp * NP; j0 < n; j0 += kComputeWarps * NP)
       attn_block<RP>(p, pw, aw, Ks, Vs, j0, n, qr, m_run, l_run, o);
     release_stage(sm, p, k);
@@ -1674,12 +2002,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
   if (sm.ctl[kAbort]) return;  // nothing issued yet
 
   if (warp == kComputeWarps) {
-    if ((tid & 31) == 0) producer_loop(p, sm, q);
+    if ((tid & 31) == 0) producer_loop<kMma>(p, sm, q);
     __syncwarp();
   } else {
     const uint32_t epoch = (uint32_t)sm.ctl[kEpoch];
     uint32_t k = 0;
-    const int rp = p.rep_p;
     for (int n = 0; n < q.count; ++n) {
       const int id = q.first + n * q.stride;
       const DevTask t = p.tasks[id];
@@ -1711,9 +2038,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           break;
         }
         case 3:
-          ok = rp <= 2 ? attn_task<2>(p, sm, t, k, id, dw)
-             : rp == 4 ? attn_task<4>(p, sm, t, k, id, dw)
-                       : attn_task<8>(p, sm, t, k, id, dw);
+          if constexpr (kMma) {
+            ok = p.D == 128 ? attn_task<128, true>(p, sm, t, k, id, dw)
+                            : attn_task<64, true>(p, sm, t, k, id, dw);
+          } else {
+            const int rp = p.rep_p;
+            ok = rp <= 2 ? attn_task_cc<2>(p, sm, t, k, id, dw)
+               : rp == 4 ? attn_task_cc<4>(p, sm, t, k, id, dw)
+                         : attn_task_cc<8>(p, sm, t, k, id, dw);
+          }
           break;
         case 9: ok = dw(); if (ok) argmax_task(p, epoch); break;
         default: ok = dw(); break;  // empty task

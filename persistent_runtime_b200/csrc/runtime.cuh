@@ -3,6 +3,8 @@
 // without nvcc.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (a plain 128-byte descriptor type)
+
 #include <cstdint>
 
 namespace mk {
@@ -74,6 +76,11 @@ struct DevLayer {
 };
 
 struct Params {
+  // 2-D tensor maps of the K and V caches seen as [Ly * B * Hkv * Lcap][D]
+  // bf16 rows: boxes of 64 dims x pps rows, 128-byte swizzle (encoded on the
+  // host for every step, since the caches are step arguments)
+  alignas(64) CUtensorMap tmap_k;
+  alignas(64) CUtensorMap tmap_v;
   // graph
   const DevTask *tasks;
   const DevEvent *events;
@@ -105,7 +112,7 @@ struct Params {
   // tiling
   int qkv_rows, o_rows, gu_rows, down_rows, lm_rows, S, chunk, n_lm;
   int rps_qkv, rps_o, rps_gu, rps_down, rps_lm;  // GEMV rows per ring stage
-  int pps;                                       // KV positions per ring stage
+  int pps;  // KV positions per ring stage (multiple of 8): K then V, D / 64 swizzled boxes each
   // tensor-core projections (batch >= 2)
   int mma;      // 1: projections run on mma.sync with fragment-ordered weights
   int nn;       // 8-sequence column tiles (1 or 2)
