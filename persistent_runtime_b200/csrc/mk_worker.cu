@@ -1881,8 +1881,9 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
 
 // Online-softmax merge of the splits of one (sequence, kv head):
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
+template <bool kMma>
 __device__ void embed_task(const Params &p) {
-  if (!p.mma) {
+  if (!kMma) {
     // 8 elements per 16-byte load (H is a multiple of 256: H / 2048 loads
     // per thread)
     const int nch = p.H >> 3;
@@ -1897,18 +1898,46 @@ __device__ void embed_task(const Params &p) {
     }
     return;
   }
-  // batch >= 2: also layer 0's QKV operand and its 16-row sums of squares
-  // (H is a multiple of 256, so every lane runs the same iterations)
+  // batch >= 2: the fp32 rows (coalesced 16-byte loads and stores), then
+  // layer 0's QKV operand one 16-byte lane unit per item: unit (k-block kb,
+  // column tile nt, lane (g, t)) holds sequence 8 nt + g, elements
+  // 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} as hi, then lo, pairs.  The 16-row
+  // sum of squares of (kb, b) is the sum over the quad's 4 lanes.
   const DevLayer &L0 = p.layers[0];
-  for (int b = 0; b < p.B; ++b) {
-    const uint16_t *e = p.embed + (size_t)p.tokens_in[b] * p.H;
-    for (int i = threadIdx.x; i < p.H; i += kComputeThreads) {
-      const float x = bf2f(e[i]);
-      p.x0[(size_t)b * p.H + i] = x;
-      put_opnd(L0.xa, i, b, p.nn, x * bf2f(L0.attn_norm[i]));
-      const float s2 = half_warp_sum(x * x);
-      if ((threadIdx.x & 15) == 0) L0.ssa[(size_t)b * p.n_parts + (i >> 4)] = s2;
+  const int nch = p.H >> 3;
+  for (int it = threadIdx.x; it < p.B * nch; it += kComputeThreads) {
+    const int b = it / nch, c = it - b * nch;
+    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)p.tokens_in[b] * p.H) + c);
+    float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H) + 2 * c;
+    dst[0] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+    dst[1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+  }
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int units = (p.H >> 4) * p.nn * 32;  // a multiple of 256: whole warps
+  for (int u = threadIdx.x; u < units; u += kComputeThreads) {
+    const int blk = u >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
+    float s2 = 0.f;
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (b < p.B) {
+      const uint32_t *e = reinterpret_cast<const uint32_t *>(p.embed + (size_t)p.tokens_in[b] * p.H);
+      const uint32_t *gm = reinterpret_cast<const uint32_t *>(L0.attn_norm);
+      const int c0 = (16 * kb + 2 * t) >> 1;  // 32-bit word of elements (2t, 2t + 1)
+      const uint32_t e01 = __ldg(e + c0), e89 = __ldg(e + c0 + 4);
+      const uint32_t g01 = __ldg(gm + c0), g89 = __ldg(gm + c0 + 4);
+      const float x0 = bf_lo(e01), x1 = bf_hi(e01), x8 = bf_lo(e89), x9 = bf_hi(e89);
+      s2 = fmaf(x0, x0, fmaf(x1, x1, fmaf(x8, x8, x9 * x9)));
+      const float y0 = x0 * bf_lo(g01), y1 = x1 * bf_hi(g01);
+      const float y8 = x8 * bf_lo(g89), y9 = x9 * bf_hi(g89);
+      const uint16_t h0 = f2bf(y0), h1 = f2bf(y1), h8 = f2bf(y8), h9 = f2bf(y9);
+      o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
+      o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
+      o.z = (uint32_t)f2bf(y0 - bf2f(h0)) | ((uint32_t)f2bf(y1 - bf2f(h1)) << 16);
+      o.w = (uint32_t)f2bf(y8 - bf2f(h8)) | ((uint32_t)f2bf(y9 - bf2f(h9)) << 16);
     }
+    reinterpret_cast<uint4 *>(L0.xa)[u] = o;
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+    if (t == 0 && b < p.B) L0.ssa[(size_t)b * p.n_parts + kb] = s2;
   }
 }
 
@@ -2018,7 +2047,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       const DepWait dw{p, sm, t.dep, epoch, id};
       bool ok = true;
       switch (t.type) {
-        case 1: ok = dw(); if (ok) embed_task(p); break;
+        case 1: ok = dw(); if (ok) embed_task<kMma>(p); break;
         case 2: case 5: case 6: case 7: case 8: {
           if constexpr (kMma) {
             ok = p.nn == 2 ? mma_task<2>(p, sm, t, k, id, dw) : mma_task<1>(p, sm, t, k, id, dw);
