@@ -162,14 +162,15 @@ def upload(torch, a):
 # ----------------------------------------------------------------------------
 # CPU oracle timing
 # ----------------------------------------------------------------------------
-def oracle_time_step(w, weights, lens, tokens, k, v, cap, layers_run=-1, vocab_run=-1):
+def oracle_time_step(w, weights, lens, tokens, k, v, cap, layers_run=-1, vocab_run=-1,
+                     seq_mask=None):
     import oracle
     oracle.build() if not os.path.exists(os.path.join(ROOT, "oracle", "libmk_oracle.so")) else None
     m = oracle.Model(w, weights, cap)
     kl = lens.copy()
     t0 = time.perf_counter()
     m.step(tokens, kl, k, v, want_logits=False, want_hidden=False, layers_run=layers_run,
-           vocab_run=vocab_run)
+           vocab_run=vocab_run, seq_mask=seq_mask)
     return time.perf_counter() - t0
 
 
@@ -422,10 +423,21 @@ def main():
     if trace_summary is not None:
         result["trace"] = trace_summary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t = oracle_time_step(w, weights, lens, tokens, k_host, v_host, cap)
+        if w.batch == 1:
+            t = oracle_time_step(w, weights, lens, tokens, k_host, v_host, cap)
+            sample = "one full decode step of the same workload, single-threaded fp32 oracle"
+        else:
+            # the oracle advances each sequence on its own: time sequence 0's
+            # full step and scale by the batch (the step's bytes per sequence
+            # are the same weights plus that sequence's cache)
+            mask = np.zeros(w.batch, dtype=np.uint8)
+            mask[0] = 1
+            t = w.batch * oracle_time_step(w, weights, lens, tokens, k_host, v_host, cap,
+                                           seq_mask=mask)
+            sample = (f"sequence 0's full decode step (kv {int(lens[0])}), single-threaded fp32 "
+                      f"oracle, times {w.batch} sequences")
         result["cpu_baseline"] = {"value": 1e6 * t, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                  "sample": "one full decode step of the same workload, "
-                                            "single-threaded fp32 oracle"}
+                                  "sample": sample}
     mk.close()
     if world > 1:
         dist.destroy_process_group()

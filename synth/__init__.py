@@ -117,8 +117,11 @@ Q8B_B16 = Workload("qwen3-8b-b16", 36, 4096, 32, 8, 128, 12288, 151936, 0, 16, 8
 # Profiling case: the 8B layer shapes with 4 layers (2.7 GB of weights), small
 # enough for multi-pass counter captures.
 Q8B_4L = Q8B.with_(name="qwen3-8b-4layer", n_layers=4)
+# Profiling case of the batched kernel: 4 of the 8B layers at batch 16, 1024
+# cached rows per sequence (about 4.5 GB on the device).
+Q8B_B16_4L = Q8B_B16.with_(name="qwen3-8b-b16-4layer", n_layers=4, kv_len=1024)
 
-WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16, Q8B_4L)}
+WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16, Q8B_4L, Q8B_B16_4L)}
 
 # ----------------------------------------------------------------------------
 # Stream ids (one counter stream per tensor)
