@@ -91,7 +91,7 @@ typedef struct {
   int col_align;             /* rows per GEMV task rounded up to this (16) */
   int attn_tasks_per_worker; /* target attention tasks per worker (4) */
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
-  int use_mma;               /* reserved: tensor-core projections for batch >= 2 */
+  int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
   int ring_stages;           /* shared-memory weight ring depth (4) */
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring (0 = off) */
@@ -166,7 +166,11 @@ mk_status mk_graph_from_edges(int n_tasks, const int32_t *task_op, const int32_t
  * mk_build_graph - plan the graph for `device` (W = its SM count unless
  * tuning->num_workers is set), upload the task/event tables, and allocate the
  * event counters, the step epoch, the status word and the activation buffers
- * (all owned by the handle).  Errors: MK_ERR_ARG, MK_ERR_CUDA, MK_ERR_OOM.
+ * (all owned by the handle).  batch 1 runs the CUDA-core worker kernel;
+ * batch 2..16 the tensor-core one (projections on mma.sync with the batch as
+ * the N dimension, attention on mma.sync over TMA K/V tiles), which needs
+ * col_align to be a multiple of 16.  Errors: MK_ERR_ARG, MK_ERR_CUDA,
+ * MK_ERR_OOM.
  */
 mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, int device,
                          mk_handle **out);
@@ -175,9 +179,14 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
  * mk_load_weights - copy the caller's weights into a library-owned arena laid
  * out in task-stream order: QKV rows group-major (per kv head: its q heads,
  * then k, then v), gate and up rows interleaved, every task's weight tile one
- * contiguous range.  Copies are ordered on `stream`; the caller may free its
- * tensors once the stream has passed this call.  May be called again to
- * replace the weights.  Errors: MK_ERR_ARG, MK_ERR_OOM, MK_ERR_CUDA.
+ * contiguous range.  For batch >= 2 handles the projection matrices are then
+ * permuted on the device into mma.sync A-fragment order (512-byte blocks per
+ * 16-row x 16-column tile) and the LM head is padded to whole 16-row tiles
+ * (a separate copy even when tied); this uses a temporary device staging
+ * buffer of the largest layer matrix and synchronises `stream`.  Copies are
+ * ordered on `stream`; the caller may free its tensors once the stream has
+ * passed this call.  May be called again to replace the weights.  Errors:
+ * MK_ERR_ARG, MK_ERR_OOM, MK_ERR_CUDA.
  */
 mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream);
 
@@ -190,8 +199,9 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream);
  *   d_kv_len[b].
  * Buffers (caller owned, device): d_tokens_in/out int32 [batch] (may be the
  * same buffer); d_kv_len int32 [batch]; d_k_cache, d_v_cache bf16
- * [n_layers][batch][n_kv_heads][kv_capacity][head_dim]; d_logits fp32
- * [batch][vocab] or NULL (then logits are not stored).
+ * [n_layers][batch][n_kv_heads][kv_capacity][head_dim], 16-byte aligned (for
+ * batch >= 2 the call encodes two TMA tensor maps of them on the host);
+ * d_logits fp32 [batch][vocab] or NULL (then logits are not stored).
  * Device-side failures (kv_len[b] + 1 > kv_capacity or a token out of range:
  * the step writes nothing; an event wait that times out) are recorded in the
  * handle's status word, make later steps no-ops, and are returned by
