@@ -88,7 +88,8 @@ typedef struct {
 /* Tuning knobs; pass NULL for defaults.  A zero field also means "default". */
 typedef struct {
   int num_workers;           /* worker CTAs W; 0 = one per SM of the device */
-  int col_align;             /* rows per GEMV task rounded up to this (16) */
+  int col_align;             /* rows per GEMV task rounded up to this (4 at batch 1, else 16;
+                                batch >= 2 needs a multiple of 16) */
   int attn_tasks_per_worker; /* target attention tasks per worker (4) */
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
   int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
@@ -202,6 +203,7 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream);
  * [n_layers][batch][n_kv_heads][kv_capacity][head_dim], 16-byte aligned (for
  * batch >= 2 the call encodes two TMA tensor maps of them on the host);
  * d_logits fp32 [batch][vocab] or NULL (then logits are not stored).
+ * Misaligned caches are rejected with MK_ERR_ARG before any launch.
  * Device-side failures (kv_len[b] + 1 > kv_capacity or a token out of range:
  * the step writes nothing; an event wait that times out) are recorded in the
  * handle's status word, make later steps no-ops, and are returned by

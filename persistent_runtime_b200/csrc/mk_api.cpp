@@ -39,10 +39,12 @@ mk_status cuda_fail(mk_handle *h, cudaError_t e, const char *what) {
 mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   mk_tuning d{};
   if (t) d = *t;
-  if (d.col_align <= 0) d.col_align = 16;
+  // batch 1: 4-row alignment gives every SM a tile of the row operators (e.g.
+  // 147 x 28 rows of a 4096-row matrix on 148 SMs instead of 128 x 32);
+  // the tensor-core tiles of batch >= 2 need whole 16-row m-tiles
+  if (d.col_align <= 0) d.col_align = batch > 1 ? 16 : 4;
   if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 4;
   if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
-  (void)batch;
   if (d.ring_stages <= 0) d.ring_stages = 4;
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
@@ -633,6 +635,9 @@ static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int3
   if (h->host_only) return fail(h, MK_ERR_ARG, "handle was made by mk_plan_graph");
   if (!h->loaded) return fail(h, MK_ERR_NOT_LOADED, "mk_load_weights has not been called");
   if (!tin || !tout || !kvl || !kc || !vc) return fail(h, MK_ERR_ARG, "null buffer");
+  // K/V rows are moved by bulk / tensor copies, which need 16-byte alignment
+  if ((reinterpret_cast<uintptr_t>(kc) | reinterpret_cast<uintptr_t>(vc)) & 15)
+    return fail(h, MK_ERR_ARG, "K/V caches must be 16-byte aligned");
   *p = h->base;
   p->tokens_in = tin;
   p->tokens_out = tout;

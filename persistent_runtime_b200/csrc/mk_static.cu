@@ -135,6 +135,10 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
     h->err = "null buffer";
     return MK_ERR_ARG;
   }
+  if ((reinterpret_cast<uintptr_t>(d_k_cache) | reinterpret_cast<uintptr_t>(d_v_cache)) & 15) {
+    h->err = "K/V caches must be 16-byte aligned";
+    return MK_ERR_ARG;
+  }
   void *base_v = nullptr;
   cudaError_t e = scratch_address(h->device, &base_v);
   if (e != cudaSuccess) {

@@ -143,3 +143,17 @@ def test_qwen3_8b_bs1_full_size_step_matches_oracle():
     ref = c.oracle_step(k=k, v=v, lens=lens)
     compare_step(ref, got, w, "8b")
     kv_rows_close(c, k, v, c.lens)
+
+
+def test_misaligned_caches_are_rejected_on_the_host():
+    # The host checks the cache pointers before any launch (bulk and tensor
+    # copies need 16-byte alignment), so nothing runs on the GPU.
+    import persistent_runtime_b200 as prb
+    w = synth.TINY
+    c = Case(w, seed=8)
+    k_off = c.d_k.view(-1)[1:]  # 2 bytes past an aligned start
+    with pytest.raises(prb.MkError) as ei:
+        c.mk.decode_step(c.d_tok, c.d_out, c.d_len, k_off, c.d_v, c.d_logits)
+    assert ei.value.status == prb.MK_ERR_ARG and "aligned" in str(ei.value)
+    got = c.gpu_step()  # the handle is still usable
+    assert (got["kv_len"] == c.lens + 1).all()

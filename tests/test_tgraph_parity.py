@@ -15,11 +15,22 @@ CONFIGS = [(synth.TINY, 148), (synth.TINY, 1), (synth.TINY, 2), (synth.TINY, 7),
            (synth.Q8B_B8, 148), (synth.Q8B_B16, 148)]
 
 
+def default_col_align(w):
+    # the library's default tile alignment: 4 rows at batch 1 (every SM gets a
+    # tile of the row operators), 16 for the tensor-core path of batch >= 2
+    return 4 if w.batch == 1 else 16
+
+
 @pytest.mark.parametrize("w,W", CONFIGS, ids=[f"{w.name}-W{W}" for w, W in CONFIGS])
-def test_decode_graph_bit_exact_with_oracle(w, W):
+@pytest.mark.parametrize("align", [16, None], ids=["align16", "default"])
+def test_decode_graph_bit_exact_with_oracle(w, W, align):
     cap = w.kv_capacity(0)
-    mine = prb.plan_graph(w, cap, W)
-    ref = oracle.tgraph_decode(w, cap, W)
+    if align is None:  # the library's defaults against the oracle at the same alignment
+        mine = prb.plan_graph(w, cap, W)
+        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w))
+    else:
+        mine = prb.plan_graph(w, cap, W, col_align=align)
+        ref = oracle.tgraph_decode(w, cap, W, align)
     gc.assert_graphs_equal(mine, ref)
     np.testing.assert_array_equal(mine.edge_src, ref.edge_src)
     np.testing.assert_array_equal(mine.edge_dst, ref.edge_dst)
