@@ -214,6 +214,17 @@ def run_reference(args):
     return 0
 
 
+def reduce_max(x: float, world: int, dist=None, device: str = "cuda") -> float:
+    """The largest x over the ranks (every rank calls it; world 1 needs no
+    process group)."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_config(w, lens, n):
     return {"workload": f"{w.name} bs{w.batch} kv{int(np.max(lens))}",
             "model": f"{w.name}-shaped decoder, {w.n_layers} layers, hidden {w.hidden}, "
@@ -307,11 +318,7 @@ def main():
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dist, "cuda")
 
     def timed(fn, k):
         reset()
