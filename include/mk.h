@@ -90,7 +90,8 @@ typedef struct {
   int num_workers;           /* worker CTAs W; 0 = one per SM of the device */
   int col_align;             /* rows per GEMV task rounded up to this (4 at batch 1, else 16;
                                 batch >= 2 needs a multiple of 16) */
-  int attn_tasks_per_worker; /* target attention tasks per worker (4) */
+  int attn_tasks_per_worker; /* at most this many attention tasks per worker (1 at batch 1,
+                                else 4) */
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
   int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
   int ring_stages;           /* shared-memory weight ring depth (4) */
@@ -213,6 +214,24 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream);
 mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_tokens_out,
                          int32_t *d_kv_len, void *d_k_cache, void *d_v_cache, float *d_logits,
                          void *stream);
+
+/*
+ * mk_decode_steps - n_steps decode steps in ONE persistent launch, with the
+ * greedy token fed back on the device ("Mirage Persistent Kernel (MPK)" page,
+ * section 5.3: one call runs the decode).  Step 0 reads d_tokens_in; step s
+ * writes d_tokens_out[s * batch + b] and step s + 1 reads it; every step
+ * appends one K/V row per (layer, sequence, kv head) and increments
+ * d_kv_len[b].  d_logits [batch][vocab] (or NULL) receives the last step's
+ * logits.  Results are bitwise those of n_steps calls of mk_decode_step.
+ * Weight streams run ahead across step boundaries; K/V rows of a step are
+ * read only after the previous step has completed.  Requires
+ * kv_len[b] + n_steps <= kv_capacity (else the launch writes nothing and the
+ * status word reports MK_ERR_DEVICE).  n_steps must be >= 1.  Errors as for
+ * mk_decode_step.
+ */
+mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
+                          int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
+                          void *d_v_cache, float *d_logits, void *stream);
 
 /*
  * mk_decode_step_perop - the comparison path: the same task bodies, launched

@@ -17,7 +17,8 @@
 //               QKV: the smallest multiple of col_align that divides one kv
 //               group's rows G = (Hq/Hkv + 2) * D and gives ceil(N/n) <= W
 //               (else n = G), so no task spans two kv groups.
-//               ATTN: S' = ceil(apw * W / (B * Hkv)),
+//               ATTN: S' = max(1, floor(apw * W / (B * Hkv))) (at most
+//               apw tasks per worker),
 //               chunk = max(min_chunk, align_up(ceil(Lcap / S'), 64)),
 //               S = ceil(Lcap / chunk).  Every split writes its partial
 //               and may write the merged head block: the split of (b, g) that
@@ -407,7 +408,7 @@ Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_
       break;
     }
   }
-  int sp = ceil_div((long)apw * W, (long)B * Hkv);
+  int sp = (int)std::max(1L, (long)apw * W / ((long)B * Hkv));
   int chunk = std::max(min_chunk, align_up(ceil_div(Lcap, sp), 64));
   int S = ceil_div(Lcap, chunk);
   L.qkv_rows = qkv_rows;

@@ -23,7 +23,7 @@ TASK_NAMES = {0: "GENERIC", 1: "EMBED", 2: "QKV", 3: "ATTN", 4: "MERGE", 5: "OPR
 
 # Every symbol declared in include/mk.h.
 EXPORTS = ("mk_plan_graph", "mk_graph_from_edges", "mk_build_graph", "mk_load_weights",
-           "mk_decode_step", "mk_decode_step_perop", "mk_decode_step_noalloc",
+           "mk_decode_step", "mk_decode_steps", "mk_decode_step_perop", "mk_decode_step_noalloc",
            "mk_sync_status", "mk_reset",
            "mk_graph_export", "mk_get_info", "mk_final_hidden", "mk_debug_set_event_count",
            "mk_set_trace", "mk_set_timeout_us", "mk_last_error", "mk_destroy")
@@ -102,6 +102,7 @@ def lib():
         "mk_load_weights": ([vp, ctypes.POINTER(Weights), vp], st),
         "mk_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_decode_step_perop": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
+        "mk_decode_steps": ([vp, i32, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_decode_step_noalloc": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_sync_status": ([vp, vp, vp], st),
         "mk_reset": ([vp, vp], st),
@@ -272,6 +273,13 @@ class Megakernel:
         _check(lib().mk_decode_step(self._h, _ptr(tokens_in), _ptr(tokens_out), _ptr(kv_len),
                                     _ptr(k_cache), _ptr(v_cache), _ptr(logits),
                                     _stream_ptr(stream)), self._h)
+
+    def decode_steps(self, n_steps, tokens_in, tokens_out, kv_len, k_cache, v_cache, logits=None,
+                     stream=None):
+        """n_steps steps in one launch; tokens_out holds n_steps x batch tokens."""
+        _check(lib().mk_decode_steps(self._h, n_steps, _ptr(tokens_in), _ptr(tokens_out),
+                                     _ptr(kv_len), _ptr(k_cache), _ptr(v_cache), _ptr(logits),
+                                     _stream_ptr(stream)), self._h)
 
     def decode_step_perop(self, tokens_in, tokens_out, kv_len, k_cache, v_cache, logits=None,
                           stream=None):

@@ -43,7 +43,9 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   // 147 x 28 rows of a 4096-row matrix on 148 SMs instead of 128 x 32);
   // the tensor-core tiles of batch >= 2 need whole 16-row m-tiles
   if (d.col_align <= 0) d.col_align = batch > 1 ? 16 : 4;
-  if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 4;
+  // batch 1: one round of attention tasks (a second round costs a whole task
+  // latency); batches: up to 4 per worker for balance over many (b, g) pairs
+  if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = batch > 1 ? 4 : 1;
   if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
   if (d.ring_stages <= 0) d.ring_stages = 4;
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
@@ -424,6 +426,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.evict_first = t.l2_stream_policy >= 0 ? 1 : 0;
   p.timeout_ns = (unsigned long long)t.wait_timeout_us * 1000ull;
   p.trace = nullptr;
+  p.n_steps = 1;
   *out = h;
   return MK_OK;
 }
@@ -659,6 +662,22 @@ mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_to
   if (s != MK_OK) return s;
   p.logits = d_logits;
   p.persistent = 1;
+  cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
+  return MK_OK;
+}
+
+mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
+                          int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
+                          void *d_v_cache, float *d_logits, void *stream) {
+  if (n_steps < 1) return fail(h, MK_ERR_ARG, "n_steps must be >= 1");
+  Params p;
+  mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache, &p);
+  if (s != MK_OK) return s;
+  p.logits = d_logits;
+  p.persistent = 1;
+  p.n_steps = n_steps;
   cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");

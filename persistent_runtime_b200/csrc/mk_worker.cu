@@ -46,6 +46,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
+// Order this thread's earlier (acquire-synchronised) view of global memory
+// before its later async-proxy (bulk / tensor copy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -115,6 +121,10 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v) {
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
                : "memory");
   return old;
+}
+
+__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
@@ -281,7 +291,7 @@ __device__ __forceinline__ void put_opnd(uint16_t *buf, int k, int b, int nn, fl
 // ---------------------------------------------------------------------------
 // Shared memory layout (identical computation on host: see smem_bytes()).
 // ---------------------------------------------------------------------------
-enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kCtlWords = 16 };
+enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kLogits = 5, kCtlWords = 16 };
 
 struct Smem {
   uint8_t *ring;
@@ -489,7 +499,7 @@ __device__ __forceinline__ AttnSpan attn_span(const Params &p, int idx) {
   int bg = idx / p.S;
   a.g = bg % p.Hkv;
   a.b = bg / p.Hkv;
-  a.L = p.kv_len[a.b];
+  a.L = __ldcg(p.kv_len + a.b);  // updated by every step's ARGMAX: read through L2
   a.p0 = a.s * p.chunk;
   int end = a.p0 + p.chunk;
   a.cached_end = min(end, a.L);
@@ -646,8 +656,29 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   pfs.nst = -1;
   uint32_t pf_k = 0;
   long long ahead = 0;
+  const uint32_t epoch0 = (uint32_t)sm.ctl[kEpoch];
+  for (int s = 0; s < p.n_steps; ++s) {
+  // K/V rows of step s > 0 include the rows step s - 1 appended (possibly on
+  // another SM), and the stream's extent depends on kv_len: the first K/V
+  // stream of a step waits until the previous step has completed.  Weight
+  // streams are never gated, so they run ahead across the step boundary.
+  bool kv_open = s == 0;
   for (int n = 0; n < q.count; ++n) {
-    const Stream ts = task_stream<kMma>(p, p.tasks[q.first + n * q.stride]);
+    const DevTask tk = p.tasks[q.first + n * q.stride];
+    if (tk.type == 3 && !kv_open) {
+      const uint64_t t0 = global_timer();
+      uint32_t spins = 0;
+      while ((int32_t)(ld_acquire(p.epoch) - (epoch0 + (uint32_t)s - 1u)) < 0) {
+        if (sm.ctl[kAbort]) goto out;
+        if ((++spins & 63u) == 0 && global_timer() - t0 > budget) {
+          record_error(p, kDevTimeout, q.first + n * q.stride, -1);
+          goto out;
+        }
+      }
+      fence_proxy_async_global();  // the appended rows are read by bulk / tensor copies
+      kv_open = true;
+    }
+    const Stream ts = task_stream<kMma>(p, tk);
     for (int st = 0; st < ts.nst; ++st) {
       const uint32_t nb = stage_bytes_of<kMma>(ts, st);
       if (dist > 0) {
@@ -710,6 +741,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       ++k;
     }
   }
+  }
 out:
   sm.ctl[kIssued] = (int)k;
 }
@@ -766,6 +798,20 @@ __device__ bool wait_event(const Params &p, int e, uint32_t epoch, int task) {
   }
 }
 
+// Thread 0: wait (bounded) until the device step epoch reached `target`.
+__device__ bool wait_epoch(const Params &p, uint32_t target, int task) {
+  const uint64_t t0 = global_timer();
+  uint32_t spins = 0;
+  while ((int32_t)(ld_acquire(p.epoch) - target) < 0) {
+    if (++spins > 64) __nanosleep(32);
+    if ((spins & 63u) == 0 && global_timer() - t0 > p.timeout_ns) {
+      record_error(p, kDevTimeout, task, -1);
+      return false;
+    }
+  }
+  return true;
+}
+
 // The wait for a task's dependency event.  Task bodies first issue the loads
 // that do not depend on this step's results (gains, RoPE factors), then call
 // this; every compute thread calls it exactly once per task.
@@ -816,7 +862,7 @@ __device__ __forceinline__ void gemv_finish(const Params &p, const Smem &sm, int
     } else if (type == 7) {
       L->x_out[r] = (f == tid ? res : __ldcg(L->xm + r)) + v;
     } else {
-      if (p.logits) p.logits[r] = v;
+      if (p.logits && sm.ctl[kLogits]) p.logits[r] = v;
       if (v > best_v || (v == best_v && r < best_i)) {
         best_v = v;
         best_i = r;
@@ -1214,7 +1260,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
           } else {
             const float lv = v * inv;
             if (store) {
-              if (p.logits) p.logits[(size_t)col * p.V + r] = lv;
+              if (p.logits && sm.ctl[kLogits]) p.logits[(size_t)col * p.V + r] = lv;
               if (lv > best_v || (lv == best_v && r < best_i)) {
                 best_v = lv;
                 best_i = r;
@@ -1296,7 +1342,7 @@ __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Sme
   if (!sm.ctl[kLast]) return true;
   if (threadIdx.x == 0) *ctr = 0u;  // every split of this step has arrived
   const DevLayer &L = p.layers[layer];
-  const int ns = min(p.S, p.kv_len[b] / p.chunk + 1);  // splits that hold any position
+  const int ns = min(p.S, __ldcg(p.kv_len + b) / p.chunk + 1);  // splits that hold any position
   const int D = p.D, rep = p.rep;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per_head = D / 64;  // warps per head (64 dims each, 2 per lane)
@@ -1449,29 +1495,37 @@ template <int D, bool SWZ>
 __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
                                           uint32_t &k, int task_id, const DepWait &dep_wait) {
   constexpr int NP = 8;  // positions per warp block
-  const AttnSpan a = attn_span(p, (int)t.idx);
-  if (!a.active) {  // the split starts past the new row: it only arrives
-    if (!dep_wait()) return false;
-    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
-  }
+  // the span read before the wait is exact when the launch runs one step
+  // (kv_len is fixed during it); a multi-step launch re-reads it after the wait
+  const AttnSpan a0 = attn_span(p, (int)t.idx);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rep = p.rep;
   constexpr int dpl = D >> 5;
   const DevLayer &L = p.layers[t.layer];
-  const float *qkv = L.qkv + (size_t)a.b * p.n_qkv + (size_t)a.g * p.grp;
-  const float *rope = p.rope + (size_t)a.L * D;  // [D/2][2]
-  // gains and RoPE factors of this lane's dims: independent of the step's
-  // results, so loaded before the wait
+  const float *qkv = L.qkv + (size_t)a0.b * p.n_qkv + (size_t)a0.g * p.grp;
+  // gains and RoPE factors of this lane's dims (the RoPE position is the
+  // speculative one above): loaded before the wait
   float gq[4], gk[4], rc[2], rs[2];
   for (int i = 0; i < dpl; ++i) {
     gq[i] = bf2f(L.q_norm[lane + 32 * i]);
     gk[i] = bf2f(L.k_norm[lane + 32 * i]);
   }
-  for (int i = 0; i < (dpl >> 1); ++i) {
-    rc[i] = rope[2 * (lane + 32 * i)];
-    rs[i] = rope[2 * (lane + 32 * i) + 1];
-  }
+  auto load_rope = [&](int pos) {  // [D/2][2] cos, sin of position pos
+    const float *rope = p.rope + (size_t)pos * D;
+    for (int i = 0; i < (dpl >> 1); ++i) {
+      rc[i] = rope[2 * (lane + 32 * i)];
+      rs[i] = rope[2 * (lane + 32 * i) + 1];
+    }
+  };
+  load_rope(a0.L);
   if (!dep_wait()) return false;
+  AttnSpan a = a0;
+  if (p.n_steps > 1) {  // kv_len advanced by the previous step of this launch
+    a = attn_span(p, (int)t.idx);
+    if (a.L != a0.L) load_rope(a.L);
+  }
+  if (!a.active)  // the split starts past the new row: it only arrives
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
 
   // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
   // holds position L; v is only rounded)
@@ -1705,28 +1759,36 @@ template <int RP>
 __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, const DevTask &t,
                                           uint32_t &k, int task_id, const DepWait &dep_wait) {
   constexpr int NP = 32 / RP;
-  const AttnSpan a = attn_span(p, (int)t.idx);
-  if (!a.active) {  // the split starts past the new row: it only arrives
-    if (!dep_wait()) return false;
-    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
-  }
+  // the span read before the wait is exact when the launch runs one step
+  // (kv_len is fixed during it); a multi-step launch re-reads it after the wait
+  const AttnSpan a0 = attn_span(p, (int)t.idx);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int D = p.D, rep = p.rep, dpl = D >> 5;
   const DevLayer &L = p.layers[t.layer];
-  const float *qkv = L.qkv + (size_t)a.b * p.n_qkv + (size_t)a.g * p.grp;
-  const float *rope = p.rope + (size_t)a.L * D;  // [D/2][2]
-  // gains and RoPE factors of this lane's dims: independent of the step's
-  // results, so loaded before the wait
+  const float *qkv = L.qkv + (size_t)a0.b * p.n_qkv + (size_t)a0.g * p.grp;
+  // gains and RoPE factors of this lane's dims (the RoPE position is the
+  // speculative one above): loaded before the wait
   float gq[4], gk[4], rc[2], rs[2];
   for (int i = 0; i < dpl; ++i) {
     gq[i] = bf2f(L.q_norm[lane + 32 * i]);
     gk[i] = bf2f(L.k_norm[lane + 32 * i]);
   }
-  for (int i = 0; i < (dpl >> 1); ++i) {
-    rc[i] = rope[2 * (lane + 32 * i)];
-    rs[i] = rope[2 * (lane + 32 * i) + 1];
-  }
+  auto load_rope = [&](int pos) {  // [D/2][2] cos, sin of position pos
+    const float *rope = p.rope + (size_t)pos * D;
+    for (int i = 0; i < (dpl >> 1); ++i) {
+      rc[i] = rope[2 * (lane + 32 * i)];
+      rs[i] = rope[2 * (lane + 32 * i) + 1];
+    }
+  };
+  load_rope(a0.L);
   if (!dep_wait()) return false;
+  AttnSpan a = a0;
+  if (p.n_steps > 1) {  // kv_len advanced by the previous step of this launch
+    a = attn_span(p, (int)t.idx);
+    if (a.L != a0.L) load_rope(a.L);
+  }
+  if (!a.active)  // the split starts past the new row: it only arrives
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
 
   // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
   // holds position L; v is only rounded)
@@ -1881,14 +1943,16 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
 
 // Online-softmax merge of the splits of one (sequence, kv head):
 //   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
+// tok: this step's input tokens (read through L2: the previous step of the
+// same launch may have written them).
 template <bool kMma>
-__device__ void embed_task(const Params &p) {
+__device__ void embed_task(const Params &p, const int32_t *tok) {
   if (!kMma) {
     // 8 elements per 16-byte load (H is a multiple of 256: H / 2048 loads
     // per thread)
     const int nch = p.H >> 3;
     for (int b = 0; b < p.B; ++b) {
-      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + (size_t)p.tokens_in[b] * p.H);
+      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
       float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H);
       for (int c = threadIdx.x; c < nch; c += kComputeThreads) {
         const uint4 w = __ldg(e + c);
@@ -1907,7 +1971,8 @@ __device__ void embed_task(const Params &p) {
   const int nch = p.H >> 3;
   for (int it = threadIdx.x; it < p.B * nch; it += kComputeThreads) {
     const int b = it / nch, c = it - b * nch;
-    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)p.tokens_in[b] * p.H) + c);
+    const uint4 w =
+        __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H) + c);
     float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H) + 2 * c;
     dst[0] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
     dst[1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
@@ -1919,7 +1984,8 @@ __device__ void embed_task(const Params &p) {
     float s2 = 0.f;
     uint4 o = make_uint4(0u, 0u, 0u, 0u);
     if (b < p.B) {
-      const uint32_t *e = reinterpret_cast<const uint32_t *>(p.embed + (size_t)p.tokens_in[b] * p.H);
+      const uint32_t *e =
+          reinterpret_cast<const uint32_t *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
       const uint32_t *gm = reinterpret_cast<const uint32_t *>(L0.attn_norm);
       const int c0 = (16 * kb + 2 * t) >> 1;  // 32-bit word of elements (2t, 2t + 1)
       const uint32_t e01 = __ldg(e + c0), e89 = __ldg(e + c0 + 4);
@@ -1951,7 +2017,8 @@ __device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
 
 // One warp per sequence: lanes scan the LM-head partials (task order), then a
 // shuffle reduction with the same total order.
-__device__ __noinline__ void argmax_task(const Params &p, uint32_t epoch) {
+// tok_out: this step's output tokens.
+__device__ __noinline__ void argmax_task(const Params &p, int32_t *tok_out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int b = warp; b < p.B; b += kComputeWarps) {
     float bv = NAN;
@@ -1974,11 +2041,10 @@ __device__ __noinline__ void argmax_task(const Params &p, uint32_t epoch) {
       }
     }
     if (lane == 0) {
-      p.tokens_out[b] = bi;
-      p.kv_len[b] = p.kv_len[b] + 1;
+      tok_out[b] = bi;
+      p.kv_len[b] = __ldcg(p.kv_len + b) + 1;
     }
   }
-  if (threadIdx.x == 0 && p.persistent) *p.epoch = epoch;
 }
 
 // ---------------------------------------------------------------------------
@@ -2016,7 +2082,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     if (*(volatile int32_t *)p.status != 0) bad = 1;  // an earlier step failed: no-op
     for (int b = 0; b < p.B && !bad; ++b) {
       const int L = p.kv_len[b], tok = p.tokens_in[b];
-      if (L < 0 || L + 1 > p.Lcap || tok < 0 || tok >= p.V) {
+      if (L < 0 || L + p.n_steps > p.Lcap || tok < 0 || tok >= p.V) {
         record_error(p, kDevBadInput, -1, b);
         bad = 1;
       }
@@ -2034,8 +2100,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     if ((tid & 31) == 0) producer_loop<kMma>(p, sm, q);
     __syncwarp();
   } else {
-    const uint32_t epoch = (uint32_t)sm.ctl[kEpoch];
+    const uint32_t epoch0 = (uint32_t)sm.ctl[kEpoch];  // step 0's epoch
     uint32_t k = 0;
+    bool run = true;
+    for (int s = 0; s < p.n_steps && run; ++s) {
+    const uint32_t epoch = epoch0 + (uint32_t)s;
+    if (tid == 0) sm.ctl[kLogits] = s == p.n_steps - 1;  // seen after the next barrier
     for (int n = 0; n < q.count; ++n) {
       const int id = q.first + n * q.stride;
       const DevTask t = p.tasks[id];
@@ -2047,7 +2117,18 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       const DepWait dw{p, sm, t.dep, epoch, id};
       bool ok = true;
       switch (t.type) {
-        case 1: ok = dw(); if (ok) embed_task<kMma>(p); break;
+        case 1:
+          ok = dw();
+          // step s > 0 reads the tokens step s - 1 wrote: wait until that
+          // step's ARGMAX has published its epoch (every task of step s
+          // descends from this EMBED)
+          if (ok && s > 0) {
+            if (tid == 0 && !wait_epoch(p, epoch - 1u, id)) sm.ctl[kAbort] = 1;
+            compute_sync();
+            ok = !sm.ctl[kAbort];
+          }
+          if (ok) embed_task<kMma>(p, s == 0 ? p.tokens_in : p.tokens_out + (size_t)(s - 1) * p.B);
+          break;
         case 2: case 5: case 6: case 7: case 8: {
           if constexpr (kMma) {
             ok = p.nn == 2 ? mma_task<2>(p, sm, t, k, id, dw) : mma_task<1>(p, sm, t, k, id, dw);
@@ -2077,15 +2158,20 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
                          : attn_task_cc<8>(p, sm, t, k, id, dw);
           }
           break;
-        case 9: ok = dw(); if (ok) argmax_task(p, epoch); break;
+        case 9: ok = dw(); if (ok) argmax_task(p, p.tokens_out + (size_t)s * p.B); break;
         default: ok = dw(); break;  // empty task
       }
-      if (!ok) break;
+      if (!ok) {
+        run = false;
+        break;
+      }
       compute_sync();
       if (tid == 0) {
         // bar.sync above orders every compute thread's stores before this
         // release, which is cumulative at gpu scope
         if (p.persistent && t.trig >= 0) red_release_add(p.counters + t.trig, 1u);
+        // the step is complete once its ARGMAX has run: publish the epoch
+        if (p.persistent && t.type == 9) st_release(p.epoch, epoch);
         if (p.trace) {
           uint32_t smid;
           asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
@@ -2100,6 +2186,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           tr[7] = sm.tmark[4];  // the task's first ring stage was available
         }
       }
+    }
     }
     if (tid == 0) sm.ctl[kConsumed] = (int)k;
   }

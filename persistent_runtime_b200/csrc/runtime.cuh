@@ -99,11 +99,13 @@ struct Params {
   int32_t *lm_idx;         // [B][n_lm] partial argmax indices
   const float *rope;       // [kv_capacity][D/2][2] cos, sin
   // step arguments
+  int n_steps;  // steps run by this launch (persistent mode): step s reads the
+                // tokens step s - 1 wrote and writes tokens_out[s][B]
   const int32_t *tokens_in;
   int32_t *tokens_out;
   int32_t *kv_len;
   uint16_t *k_cache, *v_cache;  // [Ly][B][Hkv][Lcap][D]
-  float *logits;                // [B][V] or null
+  float *logits;                // [B][V] of the last step, or null
   // shapes
   int B, H, Hq, Hkv, D, F, V, Ly, Lcap, rep, grp, n_qkv, qdim;
   int rep_p;  // rep rounded up to a power of two (1, 2, 4 or 8)

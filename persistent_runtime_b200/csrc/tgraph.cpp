@@ -94,7 +94,8 @@ std::string lower(const ModelShape &m, const GraphTuning &t, Lowering *L) {
   T.n_gu = (int)cdiv(m.ffn, T.gu_rows);
   T.n_down = (int)cdiv(m.hidden, T.down_rows);
   T.n_lm = (int)cdiv(m.vocab, T.lm_rows);
-  long target = cdiv((long)t.attn_tasks_per_worker * W, (long)m.batch * m.n_kv_heads);
+  // splits per (sequence, kv head): at most attn_tasks_per_worker tasks per worker
+  long target = std::max(1L, (long)t.attn_tasks_per_worker * W / ((long)m.batch * m.n_kv_heads));
   long chunk = cdiv(cdiv(m.kv_capacity, target), 64) * 64;
   if (chunk < t.attn_min_chunk) chunk = t.attn_min_chunk;
   T.attn_chunk = (int)chunk;

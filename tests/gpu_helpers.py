@@ -66,10 +66,14 @@ class Case:
         fn(self.d_tok, self.d_out, self.d_len, self.d_k, self.d_v, self.d_logits)
         rc, detail = self.mk.sync_status()
         assert rc == 0, (rc, detail)
+        return {"tokens": self.d_out.cpu().numpy(), "logits": self.d_logits.cpu().numpy(),
+                "hidden": self.gpu_hidden(), "kv_len": self.d_len.cpu().numpy()}
+
+    def gpu_hidden(self):
+        """fp32 [batch][hidden] residual stream after the last layer of the latest step."""
         n = self.w.batch * self.w.hidden
         hidden = _wrap_device_f32(self.mk.final_hidden_ptr(), n).view(self.w.batch, -1).clone()
-        return {"tokens": self.d_out.cpu().numpy(), "logits": self.d_logits.cpu().numpy(),
-                "hidden": hidden.cpu().numpy(), "kv_len": self.d_len.cpu().numpy()}
+        return hidden.cpu().numpy()
 
     def oracle_step(self, tokens=None, k=None, v=None, lens=None):
         k = self.k if k is None else k

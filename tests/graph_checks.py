@@ -159,7 +159,7 @@ def closed_form_counts(w, kv_capacity, W, col_align=16, apw=4, min_chunk=64):
     m = next((m for m in range(col_align, G + 1, col_align) if G % m == 0 and cdiv(Nqkv, m) <= W), G)
     t_qkv = cdiv(Nqkv, m)
     tiles = lambda N: cdiv(N, aup(cdiv(N, W), col_align))
-    sp = cdiv(apw * W, w.batch * w.n_kv_heads)
+    sp = max(1, apw * W // (w.batch * w.n_kv_heads))
     chunk = max(min_chunk, aup(cdiv(kv_capacity, sp), 64))
     S = cdiv(kv_capacity, chunk)
     n_attn = w.batch * w.n_kv_heads * S

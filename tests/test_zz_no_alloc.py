@@ -53,12 +53,13 @@ def test_noalloc_step_matches_decode_step_twice(w):
 
 def test_noalloc_rejects_steps_beyond_the_static_region():
     import persistent_runtime_b200 as prb
-    # 36 8B-shaped layers with a 60000-row cache: the attention partials alone
-    # need about 43 MiB, more than the 16 MiB region; the size is checked
-    # before anything else, so no weights are needed
+    # 36 8B-shaped layers with a 60000-row cache and 4 attention tasks per
+    # worker (73 splits per head): the split partials alone need about 43 MiB,
+    # more than the 16 MiB region; the size is checked before anything else,
+    # so no weights are needed
     w = synth.Q8B.with_(kv_len=60000)
     t = torch()
-    mk = prb.Megakernel(w, 60004, 0)
+    mk = prb.Megakernel(w, 60004, 0, attn_tasks_per_worker=4)
     buf = t.zeros(8, dtype=t.int32, device="cuda")
     with pytest.raises(prb.MkError) as ei:
         mk.decode_step_noalloc(buf, buf, buf, buf, buf)
