@@ -393,6 +393,15 @@ def main():
             baselines["perop_graph_error"] = str(e)[:200]
         baselines["perop_launches_per_step"] = n_ops
 
+    # the same K steps as ONE launch (mk_decode_steps: tokens fed back on the
+    # device); reported beside the one-launch-per-step loop above
+    multi_out = torch.zeros((args.steps, w.batch), dtype=torch.int32, device="cuda")
+    multi = lambda: mk.decode_steps(args.steps, d_tok, multi_out, d_len, d_k, d_v, d_logits)  # noqa
+    reset()
+    mk.decode_steps(args.warmup, d_tok, multi_out, d_len, d_k, d_v, d_logits)
+    check()
+    multi_us = 1000.0 * timed(multi, 1) / args.steps
+
     trace_summary = None
     if args.trace:
         from persistent_runtime_b200 import trace as mktrace
@@ -423,6 +432,8 @@ def main():
                      "traffic": None if traffic is None else traffic["dram_bytes_per_launch"]},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": 4 * w.batch,
                 "d2h_bytes_per_step": 4 * w.batch},
+        "multistep": {"value": multi_us, "unit": UNIT, "steps_per_launch": args.steps,
+                      "note": "the same steps in one mk_decode_steps launch"},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
         "baselines": baselines,
