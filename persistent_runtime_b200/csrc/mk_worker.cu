@@ -1592,7 +1592,13 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     trace_first_stage(p, sm, st);
     const uint32_t kb = smem_u32(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
     const uint32_t vb = kb + (uint32_t)(p.pps * D * 2);  // V boxes follow the K boxes
-    for (int j0 = warp * NP; j0 < n; j0 += kComputeWarps * NP)
+    // blocks are numbered across the split's stages and dealt round-robin
+    // (warp w takes global blocks w, w + 8, ...), so a stage whose block
+    // count is not a multiple of 8 does not leave the same warps idle every
+    // time; warps drift apart by at most the ring depth
+    const int base = st * (p.pps / NP);
+    for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * NP; j0 < n;
+         j0 += kComputeWarps * NP)
       attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, qh, ql, m_run, l_run, o);
     release_stage(sm, p, k);
     ++k;
