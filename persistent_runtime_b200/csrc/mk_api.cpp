@@ -180,7 +180,9 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     return fail(nullptr, MK_ERR_ARG, "batch > 1 needs col_align to be a multiple of 16");
   }
   const int rep0 = c.n_q_heads / c.n_kv_heads;
-  const int rep_p = rep0 <= 1 ? 1 : rep0 <= 2 ? 2 : rep0 <= 4 ? 4 : 8;
+  // q heads per kv head padded to the attention instantiations (2, 4, 8):
+  // the per-warp state scratch is sized by it
+  const int rep_p = rep0 <= 2 ? 2 : rep0 <= 4 ? 4 : 8;
   // shared memory: shrink the stage size until the CTA fits
   size_t smem = 0;
   for (;;) {

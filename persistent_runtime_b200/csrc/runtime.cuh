@@ -108,7 +108,7 @@ struct Params {
   float *logits;                // [B][V] of the last step, or null
   // shapes
   int B, H, Hq, Hkv, D, F, V, Ly, Lcap, rep, grp, n_qkv, qdim;
-  int rep_p;  // rep rounded up to a power of two (1, 2, 4 or 8)
+  int rep_p;  // rep rounded up to 2, 4 or 8 (the attention instantiations)
   float eps;
   float attn_scale;  // 1 / sqrt(D)
   // tiling
