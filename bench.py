@@ -155,6 +155,22 @@ def gen_inputs(w, seed, cap):
     return weights, lens, tokens, k, v
 
 
+def paged_pools(cache, P, seed):
+    """[Ly][B][Hkv][cap][D] rows -> pool [n_pages][Ly][Hkv][P][D] with the pages of
+    every sequence scattered by a seeded permutation, and the page table
+    [B][ceil(cap / P)]."""
+    Ly, B, Hkv, cap, D = cache.shape
+    mp = -(-cap // P)
+    n_pages = B * mp
+    table = np.random.default_rng(seed).permutation(n_pages).astype(np.int32).reshape(B, mp)
+    pool = np.zeros((n_pages, Ly, Hkv, P, D), dtype=np.uint16)
+    for b in range(B):
+        for j in range(mp):
+            rows = cache[:, b, :, j * P:(j + 1) * P, :]
+            pool[table[b, j], :, :, :rows.shape[2], :] = rows
+    return pool, table, n_pages
+
+
 def upload(torch, a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
@@ -249,6 +265,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true", help="skip the per-operator arms")
     ap.add_argument("--tuning", default="", help="k=v,... passed to mk_tuning")
+    ap.add_argument("--kv-page-size", type=int, default=0,
+                    help="run on paged K/V pools with this many positions per page")
     ap.add_argument("--trace", default="", help="write a Chrome trace of one step to this path")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -283,6 +301,8 @@ def main():
     tokens = synth.make_tokens(w, args.seed)
     keep_host = rank == 0 and world == 1 and not args.no_cpu_baseline
     weights = synth.make_weights(w, args.seed)
+    if args.kv_page_size:
+        tuning["kv_page_size"] = args.kv_page_size
     mk = prb.Megakernel(w, cap, dev, **tuning)
     dw = {"embed": upload(torch, weights["embed"]), "final_norm": upload(torch, weights["final_norm"]),
           "lm_head": None if weights["lm_head"] is None else upload(torch, weights["lm_head"]),
@@ -294,7 +314,15 @@ def main():
         weights = None
     torch.cuda.empty_cache()
     k_host, v_host = synth.make_kv(w, lens, cap, args.seed)
-    d_k, d_v = upload(torch, k_host), upload(torch, v_host)
+    if args.kv_page_size:
+        # the same rows in pages scattered over the pools by a seeded permutation
+        kp, table, n_pages = paged_pools(k_host, args.kv_page_size, args.seed)
+        vp, _, _ = paged_pools(v_host, args.kv_page_size, args.seed)
+        d_k, d_v = upload(torch, kp), upload(torch, vp)
+        d_table = torch.from_numpy(table).cuda()
+        del kp, vp
+    else:
+        d_k, d_v = upload(torch, k_host), upload(torch, v_host)
     if not keep_host:
         k_host = v_host = None
     d_len = torch.from_numpy(lens.copy()).cuda()
@@ -332,7 +360,13 @@ def main():
         check()
         return max_over_ranks(e0.elapsed_time(e1))
 
-    step = lambda: mk.decode_step(d_tok, d_tok, d_len, d_k, d_v, d_logits)  # noqa: E731
+    def run_steps(n, out):
+        if args.kv_page_size:
+            mk.decode_steps_paged(n, d_tok, out, d_len, d_k, d_v, n_pages, d_table, d_logits)
+        else:
+            mk.decode_steps(n, d_tok, out, d_len, d_k, d_v, d_logits)
+
+    step = lambda: run_steps(1, d_tok)  # noqa: E731
 
     # warm-up
     reset()
@@ -354,7 +388,7 @@ def main():
 
     def e2e_step():
         d_tok.copy_(h_tok, non_blocking=True)
-        mk.decode_step(d_tok, d_tok, d_len, d_k, d_v, d_logits)
+        run_steps(1, d_tok)
         h_out.copy_(d_tok, non_blocking=True)
         stream.synchronize()
         h_tok.copy_(h_out)
@@ -365,7 +399,7 @@ def main():
 
     baselines = {}
     n_ops = mk.info().n_ops
-    if not args.no_baselines:
+    if not args.no_baselines and not args.kv_page_size:  # the per-operator arms take no page table
         perop = lambda: mk.decode_step_perop(d_tok, d_tok, d_len, d_k, d_v, d_logits)  # noqa
         reset()
         for _ in range(args.warmup):
@@ -396,9 +430,9 @@ def main():
     # the same K steps as ONE launch (mk_decode_steps: tokens fed back on the
     # device); reported beside the one-launch-per-step loop above
     multi_out = torch.zeros((args.steps, w.batch), dtype=torch.int32, device="cuda")
-    multi = lambda: mk.decode_steps(args.steps, d_tok, multi_out, d_len, d_k, d_v, d_logits)  # noqa
+    multi = lambda: run_steps(args.steps, multi_out)  # noqa: E731
     reset()
-    mk.decode_steps(args.warmup, d_tok, multi_out, d_len, d_k, d_v, d_logits)
+    run_steps(args.warmup, multi_out)
     check()
     multi_us = 1000.0 * timed(multi, 1) / args.steps
 
@@ -423,7 +457,8 @@ def main():
         "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us_step / 1000.0, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, lens, world),
+        "config": dict(workload_config(w, lens, world),
+                       **({"kv_page_size": args.kv_page_size} if args.kv_page_size else {})),
         "tokens_per_s": tok_s, "hbm_gbs": gbs, "frac_of_8tbs": gbs / HBM_NOMINAL_GBS,
         "bytes_per_step": bytes_k / args.steps,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",

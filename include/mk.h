@@ -98,6 +98,8 @@ typedef struct {
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring (0 = off) */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
+  int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the
+                                paged pools (a multiple of 64), see mk_decode_steps_paged */
   int l2_stream_policy;      /* L2 policy of streamed weights and cached K/V: 0 or 1 =
                                 evict-first (default: they are read once per step and
                                 must not displace code, activations and counters),
@@ -232,6 +234,27 @@ mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_to
 mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
                           int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
                           void *d_v_cache, float *d_logits, void *stream);
+
+/*
+ * mk_decode_steps_paged - mk_decode_steps with the K/V caches as pools of
+ * pages (MPK review, zhaifeiyue, paradigm-positioning paragraph on adoption:
+ * paged attention and page allocation have to run inside the megakernel
+ * runtime for it to replace a serving stack).  The handle must
+ * have been built with tuning->kv_page_size = P > 0 (a multiple of 64).
+ * d_k_pool, d_v_pool: bf16 [n_pages][n_layers][n_kv_heads][P][head_dim],
+ * 16-byte aligned.  d_page_table: int32 [batch][ceil(kv_capacity / P)];
+ * position pos of sequence b is row pos % P of page
+ * d_page_table[b][pos / P].  Pages of one sequence may be anywhere in the
+ * pool; two sequences must not share a page they write.  Entries for
+ * positions [0, kv_len[b] + n_steps) must lie in [0, n_pages), else the
+ * launch writes nothing and the status word reports MK_ERR_DEVICE.  All
+ * other semantics and errors as mk_decode_steps; results are bitwise those
+ * of the contiguous layout.
+ */
+mk_status mk_decode_steps_paged(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
+                                int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_pool,
+                                void *d_v_pool, int n_pages, const int32_t *d_page_table,
+                                float *d_logits, void *stream);
 
 /*
  * mk_decode_step_perop - the comparison path: the same task bodies, launched

@@ -23,7 +23,8 @@ TASK_NAMES = {0: "GENERIC", 1: "EMBED", 2: "QKV", 3: "ATTN", 4: "MERGE", 5: "OPR
 
 # Every symbol declared in include/mk.h.
 EXPORTS = ("mk_plan_graph", "mk_graph_from_edges", "mk_build_graph", "mk_load_weights",
-           "mk_decode_step", "mk_decode_steps", "mk_decode_step_perop", "mk_decode_step_noalloc",
+           "mk_decode_step", "mk_decode_steps", "mk_decode_steps_paged", "mk_decode_step_perop",
+           "mk_decode_step_noalloc",
            "mk_sync_status", "mk_reset",
            "mk_graph_export", "mk_get_info", "mk_final_hidden", "mk_debug_set_event_count",
            "mk_set_trace", "mk_set_timeout_us", "mk_last_error", "mk_destroy")
@@ -48,7 +49,8 @@ class Tuning(ctypes.Structure):
                 ("attn_tasks_per_worker", ctypes.c_int), ("attn_min_chunk", ctypes.c_int),
                 ("use_mma", ctypes.c_int), ("ring_stages", ctypes.c_int),
                 ("ring_stage_bytes", ctypes.c_int), ("l2_prefetch_bytes", ctypes.c_int),
-                ("wait_timeout_us", ctypes.c_uint), ("l2_stream_policy", ctypes.c_int)]
+                ("wait_timeout_us", ctypes.c_uint), ("kv_page_size", ctypes.c_int),
+                ("l2_stream_policy", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -103,6 +105,7 @@ def lib():
         "mk_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_decode_step_perop": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_decode_steps": ([vp, i32, vp, vp, vp, vp, vp, vp, vp], st),
+        "mk_decode_steps_paged": ([vp, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp], st),
         "mk_decode_step_noalloc": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         "mk_sync_status": ([vp, vp, vp], st),
         "mk_reset": ([vp, vp], st),
@@ -280,6 +283,15 @@ class Megakernel:
         _check(lib().mk_decode_steps(self._h, n_steps, _ptr(tokens_in), _ptr(tokens_out),
                                      _ptr(kv_len), _ptr(k_cache), _ptr(v_cache), _ptr(logits),
                                      _stream_ptr(stream)), self._h)
+
+    def decode_steps_paged(self, n_steps, tokens_in, tokens_out, kv_len, k_pool, v_pool,
+                           n_pages, page_table, logits=None, stream=None):
+        """n_steps steps on paged K/V pools [n_pages][Ly][Hkv][P][D] with a page table
+        [batch][ceil(kv_capacity / P)] (handle built with kv_page_size = P)."""
+        _check(lib().mk_decode_steps_paged(self._h, n_steps, _ptr(tokens_in), _ptr(tokens_out),
+                                           _ptr(kv_len), _ptr(k_pool), _ptr(v_pool), n_pages,
+                                           _ptr(page_table), _ptr(logits), _stream_ptr(stream)),
+               self._h)
 
     def decode_step_perop(self, tokens_in, tokens_out, kv_len, k_cache, v_cache, logits=None,
                           stream=None):

@@ -179,6 +179,10 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     delete h;
     return fail(nullptr, MK_ERR_ARG, "batch > 1 needs col_align to be a multiple of 16");
   }
+  if (t.kv_page_size < 0 || t.kv_page_size % 64) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "kv_page_size must be 0 or a multiple of 64");
+  }
   const int rep0 = c.n_q_heads / c.n_kv_heads;
   // q heads per kv head padded to the attention instantiations (2, 4, 8):
   // the per-warp state scratch is sized by it
@@ -391,6 +395,16 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   // 1024-byte swizzle atoms), at most 256 (the TMA box height limit) and at
   // most one split (a multiple of 64), so a short split is one exact box
   p.pps = std::min(std::min(256, T.attn_chunk), t.ring_stage_bytes / (4 * D) / 8 * 8);
+  if (t.kv_page_size > 0) {
+    // paged pools: a stage must stay inside one page; splits start at
+    // multiples of 64 and pages hold multiples of 64 rows, so a stage of a
+    // divisor of 64 rows never crosses a page
+    int q = 64;
+    while (q > p.pps) q >>= 1;
+    p.pps = q;
+    p.page_size = t.kv_page_size;
+    p.max_pages = (c.kv_capacity + t.kv_page_size - 1) / t.kv_page_size;
+  }
   if (p.pps < 8) {
     mk_destroy(h);
     return fail(nullptr, MK_ERR_ARG, "ring stage smaller than 8 K/V rows");
@@ -616,7 +630,10 @@ std::string mk::encode_kv_maps(const mk_handle *h, const void *kc, const void *v
   const mk_model_config &c = h->cfg;
   if ((reinterpret_cast<uintptr_t>(kc) | reinterpret_cast<uintptr_t>(vc)) & 15)
     return "K/V caches must be 16-byte aligned";
-  const cuuint64_t rows = (cuuint64_t)c.n_layers * c.batch * c.n_kv_heads * c.kv_capacity;
+  const cuuint64_t rows =
+      p->page_size > 0
+          ? (cuuint64_t)p->n_pages * c.n_layers * c.n_kv_heads * p->page_size
+          : (cuuint64_t)c.n_layers * c.batch * c.n_kv_heads * c.kv_capacity;
   const cuuint64_t dims[2] = {(cuuint64_t)c.head_dim, rows};
   const cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
   const cuuint32_t box[2] = {64u, (cuuint32_t)h->base.pps};
@@ -635,8 +652,13 @@ std::string mk::encode_kv_maps(const mk_handle *h, const void *kc, const void *v
 extern "C" {
 
 static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int32_t *kvl,
-                           void *kc, void *vc, Params *p) {
+                           void *kc, void *vc, Params *p, int n_pages = 0,
+                           const int32_t *page_table = nullptr) {
   if (!h) return fail(nullptr, MK_ERR_ARG, "null handle");
+  if (!h->host_only && (h->base.page_size > 0) != (page_table != nullptr))
+    return fail(h, MK_ERR_ARG,
+                h->base.page_size > 0 ? "the handle was built for paged K/V: use mk_decode_steps_paged"
+                                      : "the handle was built for contiguous K/V caches");
   if (h->host_only) return fail(h, MK_ERR_ARG, "handle was made by mk_plan_graph");
   if (!h->loaded) return fail(h, MK_ERR_NOT_LOADED, "mk_load_weights has not been called");
   if (!tin || !tout || !kvl || !kc || !vc) return fail(h, MK_ERR_ARG, "null buffer");
@@ -649,6 +671,11 @@ static mk_status step_args(mk_handle *h, const int32_t *tin, int32_t *tout, int3
   p->kv_len = kvl;
   p->k_cache = static_cast<uint16_t *>(kc);
   p->v_cache = static_cast<uint16_t *>(vc);
+  if (page_table) {
+    if (n_pages < 1) return fail(h, MK_ERR_ARG, "n_pages must be >= 1");
+    p->page_table = page_table;
+    p->n_pages = n_pages;
+  }
   if (h->base.mma) {  // only the batched kernel reads K/V through tensor maps
     const std::string e = mk::encode_kv_maps(h, kc, vc, p);
     if (!e.empty()) return fail(h, MK_ERR_ARG, e);
@@ -676,6 +703,25 @@ mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
   if (n_steps < 1) return fail(h, MK_ERR_ARG, "n_steps must be >= 1");
   Params p;
   mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache, &p);
+  if (s != MK_OK) return s;
+  p.logits = d_logits;
+  p.persistent = 1;
+  p.n_steps = n_steps;
+  cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
+  return MK_OK;
+}
+
+mk_status mk_decode_steps_paged(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
+                                int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_pool,
+                                void *d_v_pool, int n_pages, const int32_t *d_page_table,
+                                float *d_logits, void *stream) {
+  if (n_steps < 1) return fail(h, MK_ERR_ARG, "n_steps must be >= 1");
+  if (!d_page_table) return fail(h, MK_ERR_ARG, "null page table");
+  Params p;
+  mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_pool, d_v_pool, &p,
+                          n_pages, d_page_table);
   if (s != MK_OK) return s;
   p.logits = d_logits;
   p.persistent = 1;

@@ -508,7 +508,13 @@ __device__ __forceinline__ AttnSpan attn_span(const Params &p, int idx) {
   return a;
 }
 
+// Element offset of cache row `row` of (layer, sequence b, kv head g): the
+// contiguous layout, or row % P of the sequence's page of the paged pools.
 __device__ __forceinline__ size_t kv_row(const Params &p, int layer, int b, int g, int row) {
+  if (p.page_size > 0) {
+    const int page = __ldg(p.page_table + (size_t)b * p.max_pages + row / p.page_size);
+    return ((((size_t)page * p.Ly + layer) * p.Hkv + g) * p.page_size + row % p.page_size) * p.D;
+  }
   return ((((size_t)layer * p.B + b) * p.Hkv + g) * p.Lcap + row) * p.D;
 }
 
@@ -522,10 +528,19 @@ struct Stream {
   // tensor-core projections: stage st = (row block st / nkc, k chunk st % nkc)
   int nkc = 0;                    // 0 for the other streams
   int KB = 0, mt0 = 0, mt1 = 0, mb = 0, kcb = 0;
-  // attention: K/V rows y0 + st * pps .. of the 2-D cache tensor maps
+  // attention: K/V rows y0 + st * pps .. of the 2-D cache tensor maps (paged
+  // pools: stage st starts at position kv_p0 + st * pps of (layer, b, g);
+  // a stage never crosses a page)
   int kv = 0;
   int y0 = 0;
+  int kv_l = 0, kv_b = 0, kv_g = 0, kv_p0 = 0;
 };
+
+// First cache row (in rows of D elements) of K/V stage st of stream s.
+__device__ __forceinline__ int kv_stage_row(const Params &p, const Stream &s, int st) {
+  if (p.page_size > 0) return (int)(kv_row(p, s.kv_l, s.kv_b, s.kv_g, s.kv_p0 + st * p.pps) / p.D);
+  return s.y0 + st * p.pps;
+}
 
 // kMma: the batched kernel (tensor-core tiles, swizzled TMA K/V boxes).
 template <bool kMma>
@@ -551,6 +566,10 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
     if (n <= 0) return s;
     s.nst = (n + p.pps - 1) / p.pps;
     s.kv = 1;
+    s.kv_l = t.layer;
+    s.kv_b = a.b;
+    s.kv_g = a.g;
+    s.kv_p0 = a.p0;
     s.y0 = (int)(kv_row(p, t.layer, a.b, a.g, a.p0) / p.D);
     s.bytes = s.last_bytes = (uint32_t)(p.pps * p.D * 2);
     // batch 1: plain row copies of exactly the cached rows
@@ -585,7 +604,7 @@ template <bool kMma>
 __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, int st, uint8_t *dst,
                                             uint64_t *bar, uint64_t pol) {
   if (s.kv) {
-    const int y = s.y0 + st * p.pps;
+    const int y = kv_stage_row(p, s, st);
     if (!kMma) {  // plain rows: K at dst, V pps rows further
       const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
       bulk_g2s(dst, p.k_cache + (size_t)y * p.D, nb, bar, pol);
@@ -2100,6 +2119,22 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     sm.tmark[3] = 0;
   }
   __syncthreads();
+  if (p.page_size > 0 && !sm.ctl[kAbort]) {
+    // every page a sequence touches in this launch must be in the pools
+    int badp = 0;
+    for (int i = tid; i < p.B * p.max_pages; i += kThreads) {
+      const int b = i / p.max_pages, j = i - b * p.max_pages;
+      const int rows = min(p.kv_len[b] + p.n_steps, p.Lcap);
+      if (j * p.page_size < rows) {
+        const int pg = p.page_table[i];
+        if (pg < 0 || pg >= p.n_pages) badp = 1;
+      }
+    }
+    if (__syncthreads_or(badp)) {
+      if (tid == 0) record_error(p, kDevBadInput, -1, -1);
+      return;  // nothing issued yet
+    }
+  }
   if (sm.ctl[kAbort]) return;  // nothing issued yet
 
   if (warp == kComputeWarps) {

@@ -104,7 +104,11 @@ struct Params {
   const int32_t *tokens_in;
   int32_t *tokens_out;
   int32_t *kv_len;
-  uint16_t *k_cache, *v_cache;  // [Ly][B][Hkv][Lcap][D]
+  uint16_t *k_cache, *v_cache;  // [Ly][B][Hkv][Lcap][D], or paged pools (below)
+  // paged KV (page_size > 0): pools [n_pages][Ly][Hkv][page_size][D]; position
+  // pos of sequence b is row pos % page_size of page page_table[b][pos / page_size]
+  const int32_t *page_table;    // [B][max_pages]
+  int page_size, max_pages, n_pages;
   float *logits;                // [B][V] of the last step, or null
   // shapes
   int B, H, Hq, Hkv, D, F, V, Ly, Lcap, rep, grp, n_qkv, qdim;
