@@ -90,8 +90,7 @@ typedef struct {
   int num_workers;           /* worker CTAs W; 0 = one per SM of the device */
   int col_align;             /* rows per GEMV task rounded up to this (4 at batch 1, else 16;
                                 batch >= 2 needs a multiple of 16) */
-  int attn_tasks_per_worker; /* at most this many attention tasks per worker (1 at batch 1,
-                                else 4) */
+  int attn_tasks_per_worker; /* at most this many attention tasks per worker (1) */
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
   int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
   int ring_stages;           /* shared-memory weight ring depth (4) */

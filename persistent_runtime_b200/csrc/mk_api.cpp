@@ -43,9 +43,10 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   // 147 x 28 rows of a 4096-row matrix on 148 SMs instead of 128 x 32);
   // the tensor-core tiles of batch >= 2 need whole 16-row m-tiles
   if (d.col_align <= 0) d.col_align = batch > 1 ? 16 : 4;
-  // batch 1: one round of attention tasks (a second round costs a whole task
-  // latency); batches: up to 4 per worker for balance over many (b, g) pairs
-  if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = batch > 1 ? 4 : 1;
+  // one round of attention tasks: a second round costs a whole task latency,
+  // and more splits mean more partials to merge (measured on Qwen3-8B: bs16
+  // 12.65 ms at 4 per worker, 11.36 ms at 1; bs8 7.23 -> 6.38 ms)
+  if (d.attn_tasks_per_worker <= 0) d.attn_tasks_per_worker = 1;
   if (d.attn_min_chunk <= 0) d.attn_min_chunk = 64;
   if (d.ring_stages <= 0) d.ring_stages = 4;
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;

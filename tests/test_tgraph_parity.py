@@ -18,7 +18,7 @@ CONFIGS = [(synth.TINY, 148), (synth.TINY, 1), (synth.TINY, 2), (synth.TINY, 7),
 def default_col_align(w):
     # the library's default tile alignment: 4 rows at batch 1 (every SM gets a
     # tile of the row operators), 16 for the tensor-core path of batch >= 2;
-    # its default attention tasks per worker: 1 at batch 1, 4 otherwise
+    # its default attention tasks per worker is 1
     return 4 if w.batch == 1 else 16
 
 
@@ -28,11 +28,10 @@ def test_decode_graph_bit_exact_with_oracle(w, W, align):
     cap = w.kv_capacity(0)
     if align is None:  # the library's defaults against the oracle with the same values
         mine = prb.plan_graph(w, cap, W)
-        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w),
-                                   1 if w.batch == 1 else 4)
+        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w), 1)
     else:
-        mine = prb.plan_graph(w, cap, W, col_align=align)
-        ref = oracle.tgraph_decode(w, cap, W, align)
+        mine = prb.plan_graph(w, cap, W, col_align=align, attn_tasks_per_worker=4)
+        ref = oracle.tgraph_decode(w, cap, W, align, 4)
     gc.assert_graphs_equal(mine, ref)
     np.testing.assert_array_equal(mine.edge_src, ref.edge_src)
     np.testing.assert_array_equal(mine.edge_dst, ref.edge_dst)
