@@ -1103,6 +1103,34 @@ __device__ __forceinline__ void load_bfrag(uint4 (&bf)[kMmaMaxKPW][NN], const ui
   }
 }
 
+// One full ring stage of a projection with compile-time tile counts (MBF
+// m-tiles, KPWF k-blocks per warp) and the refill of every B fragment for the
+// next stage: the common case, with no per-tile guards, so the A fragments of
+// a k-block are loaded before its MMAs.
+template <int NN, int MBF, int KPWF>
+__device__ __forceinline__ void mma_stage_full(float (&acc)[kMmaMaxMB][NN][4],
+                                               uint4 (&bc)[kMmaMaxKPW][NN], const uint8_t *slot,
+                                               const uint16_t *xn, int warp, int lane) {
+  constexpr int NKB = 8 * KPWF;
+#pragma unroll
+  for (int j = 0; j < KPWF; ++j) {
+    const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
+    uint4 a[MBF];
+#pragma unroll
+    for (int m = 0; m < MBF; ++m) a[m] = *reinterpret_cast<const uint4 *>(blk + m * NKB * 512);
+#pragma unroll
+    for (int m = 0; m < MBF; ++m)
+#pragma unroll
+      for (int n = 0; n < NN; ++n) {
+        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
+        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
+      }
+#pragma unroll
+    for (int n = 0; n < NN; ++n)
+      bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+  }
+}
+
 // Sum over the 16 lanes of a half warp (lanes that share a sequence column).
 __device__ __forceinline__ float half_warp_sum(float v) {
 #pragma unroll
@@ -1187,6 +1215,14 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
     if (got) {
       trace_first_stage(p, sm, st);
       const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
+      const bool full_next = kpw_n == kpw;
+      if (full_next && kpw == 3 && nm == 2) {
+        mma_stage_full<NN, 2, 3>(acc, bc, slot, xn, warp, lane);
+      } else if (full_next && kpw == 3 && nm == 3) {
+        mma_stage_full<NN, 3, 3>(acc, bc, slot, xn, warp, lane);
+      } else if (full_next && kpw == 2 && nm == 6) {
+        mma_stage_full<NN, 6, 2>(acc, bc, slot, xn, warp, lane);
+      } else {
 #pragma unroll
       for (int j = 0; j < kMmaMaxKPW; ++j) {
         if (j < kpw) {
@@ -1209,6 +1245,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
             bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
                                   xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
         }
+      }
       }
       release_stage(sm, p, k);
       ++k;
@@ -1966,69 +2003,103 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
   return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
 }
 
-// Online-softmax merge of the splits of one (sequence, kv head):
-//   M = max_s m_s,  w_s = exp(m_s - M),  o = sum_s w_s o_s / sum_s w_s l_s.
+// Batch >= 2 EMBED: kept out of line so its load batches do not raise the
+// register demand of the worker loop.
 // tok: this step's input tokens (read through L2: the previous step of the
 // same launch may have written them).
-template <bool kMma>
-__device__ void embed_task(const Params &p, const int32_t *tok) {
-  if (!kMma) {
-    // 8 elements per 16-byte load (H is a multiple of 256: H / 2048 loads
-    // per thread)
-    const int nch = p.H >> 3;
-    for (int b = 0; b < p.B; ++b) {
-      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
-      float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H);
-      for (int c = threadIdx.x; c < nch; c += kComputeThreads) {
-        const uint4 w = __ldg(e + c);
-        dst[2 * c] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-        dst[2 * c + 1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
-      }
-    }
-    return;
-  }
-  // batch >= 2: the fp32 rows (coalesced 16-byte loads and stores), then
+__device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
+  // The fp32 rows (coalesced 16-byte loads and stores), then
   // layer 0's QKV operand one 16-byte lane unit per item: unit (k-block kb,
   // column tile nt, lane (g, t)) holds sequence 8 nt + g, elements
   // 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} as hi, then lo, pairs.  The 16-row
-  // sum of squares of (kb, b) is the sum over the quad's 4 lanes.
+  // sum of squares of (kb, b) is the sum over the quad's 4 lanes.  One CTA
+  // does it all, so each thread keeps 4 items' loads in flight before it
+  // uses any (the loop bounds are multiples of 4 x 256: H is a multiple of
+  // 256, units a multiple of 512 per column tile).
+  constexpr int kU = 4;
   const DevLayer &L0 = p.layers[0];
-  const int nch = p.H >> 3;
-  for (int it = threadIdx.x; it < p.B * nch; it += kComputeThreads) {
-    const int b = it / nch, c = it - b * nch;
-    const uint4 w =
-        __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H) + c);
-    float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H) + 2 * c;
-    dst[0] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-    dst[1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+  const int nch = p.H >> 3, items = p.B * nch;
+  for (int i0 = threadIdx.x; i0 < items; i0 += kU * kComputeThreads) {
+    uint4 w[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int it = i0 + u * kComputeThreads;
+      if (it < items) {
+        const int b = it / nch, c = it - b * nch;
+        w[u] = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H) + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int it = i0 + u * kComputeThreads;
+      if (it < items) {
+        const int b = it / nch, c = it - b * nch;
+        float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H) + 2 * c;
+        dst[0] = make_float4(bf_lo(w[u].x), bf_hi(w[u].x), bf_lo(w[u].y), bf_hi(w[u].y));
+        dst[1] = make_float4(bf_lo(w[u].z), bf_hi(w[u].z), bf_lo(w[u].w), bf_hi(w[u].w));
+      }
+    }
   }
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int units = (p.H >> 4) * p.nn * 32;  // a multiple of 256: whole warps
-  for (int u = threadIdx.x; u < units; u += kComputeThreads) {
-    const int blk = u >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
-    float s2 = 0.f;
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (b < p.B) {
-      const uint32_t *e =
-          reinterpret_cast<const uint32_t *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
-      const uint32_t *gm = reinterpret_cast<const uint32_t *>(L0.attn_norm);
+  const int units = (p.H >> 4) * p.nn * 32;  // a multiple of 512: whole warps
+  const uint32_t *gm = reinterpret_cast<const uint32_t *>(L0.attn_norm);
+  for (int u0 = threadIdx.x; u0 < units; u0 += kU * kComputeThreads) {
+    uint32_t e01[kU], e89[kU], g01[kU], g89[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int un = u0 + u * kComputeThreads;
+      const int blk = un >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
       const int c0 = (16 * kb + 2 * t) >> 1;  // 32-bit word of elements (2t, 2t + 1)
-      const uint32_t e01 = __ldg(e + c0), e89 = __ldg(e + c0 + 4);
-      const uint32_t g01 = __ldg(gm + c0), g89 = __ldg(gm + c0 + 4);
-      const float x0 = bf_lo(e01), x1 = bf_hi(e01), x8 = bf_lo(e89), x9 = bf_hi(e89);
-      s2 = fmaf(x0, x0, fmaf(x1, x1, fmaf(x8, x8, x9 * x9)));
-      const float y0 = x0 * bf_lo(g01), y1 = x1 * bf_hi(g01);
-      const float y8 = x8 * bf_lo(g89), y9 = x9 * bf_hi(g89);
+      e01[u] = e89[u] = g01[u] = g89[u] = 0u;
+      if (un < units && b < p.B) {
+        const uint32_t *e =
+            reinterpret_cast<const uint32_t *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
+        e01[u] = __ldg(e + c0);
+        e89[u] = __ldg(e + c0 + 4);
+        g01[u] = __ldg(gm + c0);
+        g89[u] = __ldg(gm + c0 + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int un = u0 + u * kComputeThreads;
+      if (un >= units) break;  // uniform per warp
+      const int blk = un >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
+      const float x0 = bf_lo(e01[u]), x1 = bf_hi(e01[u]), x8 = bf_lo(e89[u]), x9 = bf_hi(e89[u]);
+      float s2 = fmaf(x0, x0, fmaf(x1, x1, fmaf(x8, x8, x9 * x9)));
+      const float y0 = x0 * bf_lo(g01[u]), y1 = x1 * bf_hi(g01[u]);
+      const float y8 = x8 * bf_lo(g89[u]), y9 = x9 * bf_hi(g89[u]);
       const uint16_t h0 = f2bf(y0), h1 = f2bf(y1), h8 = f2bf(y8), h9 = f2bf(y9);
+      uint4 o;
       o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
       o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
       o.z = (uint32_t)f2bf(y0 - bf2f(h0)) | ((uint32_t)f2bf(y1 - bf2f(h1)) << 16);
       o.w = (uint32_t)f2bf(y8 - bf2f(h8)) | ((uint32_t)f2bf(y9 - bf2f(h9)) << 16);
+      reinterpret_cast<uint4 *>(L0.xa)[un] = o;  // zeros for padded sequences
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+      if (t == 0 && b < p.B) L0.ssa[(size_t)b * p.n_parts + kb] = s2;
     }
-    reinterpret_cast<uint4 *>(L0.xa)[u] = o;
-    s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
-    s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
-    if (t == 0 && b < p.B) L0.ssa[(size_t)b * p.n_parts + kb] = s2;
+  }
+}
+
+template <bool kMma>
+__device__ void embed_task(const Params &p, const int32_t *tok) {
+  if (kMma) {
+    embed_batch(p, tok);
+    return;
+  }
+  // 8 elements per 16-byte load (H is a multiple of 256: H / 2048 loads
+  // per thread)
+  const int nch = p.H >> 3;
+  for (int b = 0; b < p.B; ++b) {
+    const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
+    float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H);
+    for (int c = threadIdx.x; c < nch; c += kComputeThreads) {
+      const uint4 w = __ldg(e + c);
+      dst[2 * c] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+      dst[2 * c + 1] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+    }
   }
 }
 
