@@ -1103,14 +1103,14 @@ __device__ __forceinline__ void load_bfrag(uint4 (&bf)[kMmaMaxKPW][NN], const ui
   }
 }
 
-// One full ring stage of a projection with compile-time tile counts (MBF
-// m-tiles, KPWF k-blocks per warp) and the refill of every B fragment for the
-// next stage: the common case, with no per-tile guards, so the A fragments of
-// a k-block are loaded before its MMAs.
-template <int NN, int MBF, int KPWF>
-__device__ __forceinline__ void mma_stage_full(float (&acc)[kMmaMaxMB][NN][4],
-                                               uint4 (&bc)[kMmaMaxKPW][NN], const uint8_t *slot,
-                                               const uint16_t *xn, int warp, int lane) {
+// One ring stage of a projection with compile-time tile counts (MBF m-tiles,
+// KPWF k-blocks per warp): the common cases, with no per-tile guards, so the
+// A fragments of a k-block are loaded before its MMAs.  The B fragments of
+// the next stage's first kpw_n k-blocks are refilled after their last use.
+template <int NN, int MBF, int KPWF, bool kGuard>
+__device__ __forceinline__ void mma_stage_fixed(float (&acc)[kMmaMaxMB][NN][4],
+                                                uint4 (&bc)[kMmaMaxKPW][NN], const uint8_t *slot,
+                                                const uint16_t *xn, int kpw_n, int warp, int lane) {
   constexpr int NKB = 8 * KPWF;
 #pragma unroll
   for (int j = 0; j < KPWF; ++j) {
@@ -1125,9 +1125,20 @@ __device__ __forceinline__ void mma_stage_full(float (&acc)[kMmaMaxMB][NN][4],
         mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
         mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
       }
+    if (!kGuard || j < kpw_n) {
 #pragma unroll
-    for (int n = 0; n < NN; ++n)
-      bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+      for (int n = 0; n < NN; ++n)
+        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+    }
+  }
+  // a next stage with more k-blocks (the first chunk after a short last one)
+#pragma unroll
+  for (int j = KPWF; j < (kGuard ? kMmaMaxKPW : 0); ++j) {
+    if (j < kpw_n) {
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+    }
   }
 }
 
@@ -1215,13 +1226,21 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
     if (got) {
       trace_first_stage(p, sm, st);
       const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
-      const bool full_next = kpw_n == kpw;
-      if (full_next && kpw == 3 && nm == 2) {
-        mma_stage_full<NN, 2, 3>(acc, bc, slot, xn, warp, lane);
-      } else if (full_next && kpw == 3 && nm == 3) {
-        mma_stage_full<NN, 3, 3>(acc, bc, slot, xn, warp, lane);
-      } else if (full_next && kpw == 2 && nm == 6) {
-        mma_stage_full<NN, 6, 2>(acc, bc, slot, xn, warp, lane);
+      const bool same = kpw_n == kpw;  // the next stage refills every fragment
+      if (same && kpw == 3 && nm == 2) {
+        mma_stage_fixed<NN, 2, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 3 && nm == 3) {
+        mma_stage_fixed<NN, 3, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 2 && nm == 6) {
+        mma_stage_fixed<NN, 6, 2, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 3 && nm == 2) {
+        mma_stage_fixed<NN, 2, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 3 && nm == 3) {
+        mma_stage_fixed<NN, 3, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 2 && nm == 2) {
+        mma_stage_fixed<NN, 2, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 2 && nm == 3) {
+        mma_stage_fixed<NN, 3, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
       } else {
 #pragma unroll
       for (int j = 0; j < kMmaMaxKPW; ++j) {
@@ -2008,77 +2027,72 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
 // tok: this step's input tokens (read through L2: the previous step of the
 // same launch may have written them).
 __device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
-  // The fp32 rows (coalesced 16-byte loads and stores), then
-  // layer 0's QKV operand one 16-byte lane unit per item: unit (k-block kb,
-  // column tile nt, lane (g, t)) holds sequence 8 nt + g, elements
-  // 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} as hi, then lo, pairs.  The 16-row
-  // sum of squares of (kb, b) is the sum over the quad's 4 lanes.  One CTA
-  // does it all, so each thread keeps 4 items' loads in flight before it
-  // uses any (the loop bounds are multiples of 4 x 256: H is a multiple of
-  // 256, units a multiple of 512 per column tile).
+  // One item per (k-block kb, sequence b < 8 nn): its 16 embedding elements
+  // 16 kb .. 16 kb + 15 (two 16-byte loads) become the fp32 row slice, the
+  // sum of squares of the 16-row part, and the 4 lane units of layer 0's
+  // QKV operand: unit (kb, column tile b / 8, lane (b % 8, t)) holds
+  // elements 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} times the attention-norm
+  // gains as hi, then lo, bf16 pairs (zeros for padded sequences).  One CTA
+  // does it all, so each thread keeps kU items' loads in flight before it
+  // uses any.
   constexpr int kU = 4;
   const DevLayer &L0 = p.layers[0];
-  const int nch = p.H >> 3, items = p.B * nch;
+  const int nb8 = 8 * p.nn, items = (p.H >> 4) * nb8;
+  const uint4 *gn = reinterpret_cast<const uint4 *>(L0.attn_norm);
+  uint4 *xa = reinterpret_cast<uint4 *>(L0.xa);
   for (int i0 = threadIdx.x; i0 < items; i0 += kU * kComputeThreads) {
-    uint4 w[kU];
+    uint4 e[kU][2], gw[kU][2];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int it = i0 + u * kComputeThreads;
-      if (it < items) {
-        const int b = it / nch, c = it - b * nch;
-        w[u] = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H) + c);
+      const int kb = it / nb8, b = it - kb * nb8;
+      e[u][0] = e[u][1] = gw[u][0] = gw[u][1] = make_uint4(0u, 0u, 0u, 0u);
+      if (it < items && b < p.B) {
+        const uint4 *er = reinterpret_cast<const uint4 *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
+        e[u][0] = __ldg(er + 2 * kb);
+        e[u][1] = __ldg(er + 2 * kb + 1);
+        gw[u][0] = __ldg(gn + 2 * kb);
+        gw[u][1] = __ldg(gn + 2 * kb + 1);
       }
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int it = i0 + u * kComputeThreads;
-      if (it < items) {
-        const int b = it / nch, c = it - b * nch;
-        float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H) + 2 * c;
-        dst[0] = make_float4(bf_lo(w[u].x), bf_hi(w[u].x), bf_lo(w[u].y), bf_hi(w[u].y));
-        dst[1] = make_float4(bf_lo(w[u].z), bf_hi(w[u].z), bf_lo(w[u].w), bf_hi(w[u].w));
-      }
-    }
-  }
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int units = (p.H >> 4) * p.nn * 32;  // a multiple of 512: whole warps
-  const uint32_t *gm = reinterpret_cast<const uint32_t *>(L0.attn_norm);
-  for (int u0 = threadIdx.x; u0 < units; u0 += kU * kComputeThreads) {
-    uint32_t e01[kU], e89[kU], g01[kU], g89[kU];
+      if (it >= items) break;
+      const int kb = it / nb8, b = it - kb * nb8;
+      const uint32_t ew[8] = {e[u][0].x, e[u][0].y, e[u][0].z, e[u][0].w,
+                              e[u][1].x, e[u][1].y, e[u][1].z, e[u][1].w};
+      const uint32_t gv[8] = {gw[u][0].x, gw[u][0].y, gw[u][0].z, gw[u][0].w,
+                              gw[u][1].x, gw[u][1].y, gw[u][1].z, gw[u][1].w};
+      float x[16], y[16];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int un = u0 + u * kComputeThreads;
-      const int blk = un >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
-      const int c0 = (16 * kb + 2 * t) >> 1;  // 32-bit word of elements (2t, 2t + 1)
-      e01[u] = e89[u] = g01[u] = g89[u] = 0u;
-      if (un < units && b < p.B) {
-        const uint32_t *e =
-            reinterpret_cast<const uint32_t *>(p.embed + (size_t)__ldcg(tok + b) * p.H);
-        e01[u] = __ldg(e + c0);
-        e89[u] = __ldg(e + c0 + 4);
-        g01[u] = __ldg(gm + c0);
-        g89[u] = __ldg(gm + c0 + 4);
+      for (int i = 0; i < 8; ++i) {
+        x[2 * i] = bf_lo(ew[i]);
+        x[2 * i + 1] = bf_hi(ew[i]);
+        y[2 * i] = x[2 * i] * bf_lo(gv[i]);
+        y[2 * i + 1] = x[2 * i + 1] * bf_hi(gv[i]);
       }
-    }
+      float st[4];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int un = u0 + u * kComputeThreads;
-      if (un >= units) break;  // uniform per warp
-      const int blk = un >> 5, kb = blk / p.nn, b = (blk - kb * p.nn) * 8 + g;
-      const float x0 = bf_lo(e01[u]), x1 = bf_hi(e01[u]), x8 = bf_lo(e89[u]), x9 = bf_hi(e89[u]);
-      float s2 = fmaf(x0, x0, fmaf(x1, x1, fmaf(x8, x8, x9 * x9)));
-      const float y0 = x0 * bf_lo(g01[u]), y1 = x1 * bf_hi(g01[u]);
-      const float y8 = x8 * bf_lo(g89[u]), y9 = x9 * bf_hi(g89[u]);
-      const uint16_t h0 = f2bf(y0), h1 = f2bf(y1), h8 = f2bf(y8), h9 = f2bf(y9);
-      uint4 o;
-      o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
-      o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
-      o.z = (uint32_t)f2bf(y0 - bf2f(h0)) | ((uint32_t)f2bf(y1 - bf2f(h1)) << 16);
-      o.w = (uint32_t)f2bf(y8 - bf2f(h8)) | ((uint32_t)f2bf(y9 - bf2f(h9)) << 16);
-      reinterpret_cast<uint4 *>(L0.xa)[un] = o;  // zeros for padded sequences
-      s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
-      if (t == 0 && b < p.B) L0.ssa[(size_t)b * p.n_parts + kb] = s2;
+      for (int t = 0; t < 4; ++t) {
+        const float a0 = x[2 * t], a1 = x[2 * t + 1], a8 = x[2 * t + 8], a9 = x[2 * t + 9];
+        st[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a8, a8, a9 * a9)));
+        const uint16_t h0 = f2bf(y[2 * t]), h1 = f2bf(y[2 * t + 1]);
+        const uint16_t h8 = f2bf(y[2 * t + 8]), h9 = f2bf(y[2 * t + 9]);
+        uint4 o;
+        o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
+        o.z = (uint32_t)f2bf(y[2 * t] - bf2f(h0)) | ((uint32_t)f2bf(y[2 * t + 1] - bf2f(h1)) << 16);
+        o.w = (uint32_t)f2bf(y[2 * t + 8] - bf2f(h8)) | ((uint32_t)f2bf(y[2 * t + 9] - bf2f(h9)) << 16);
+        xa[((size_t)kb * p.nn + (b >> 3)) * 32 + (b & 7) * 4 + t] = o;
+      }
+      if (b < p.B) {
+        // the sum in the order of a quad's two butterfly steps
+        L0.ssa[(size_t)b * p.n_parts + kb] = (st[0] + st[1]) + (st[2] + st[3]);
+        float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H + 16 * kb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+      }
     }
   }
 }
