@@ -1478,18 +1478,23 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
 }
 
 // One block of 8 positions [j0, j0 + 8) of a K/V tile (rows of D bf16) for
-// one warp, on tensor cores.  Query heads are the rows of the MMA (up to 8,
-// zero padded to 16), positions its columns:
-//   S  = Q K^T        m16n8k16, K fragments by ldmatrix from the row-major tile
+// one warp, on tensor cores.  Query heads are the rows of the MMA, positions
+// its columns:
+//   S  = Q K^T        m16n8k16; rows g < 8 hold q head g's hi bf16 term and
+//                     rows g + 8 its lo term, so lane (g, t) receives both
+//                     halves of head g's scores at positions 2t, 2t + 1 and
+//                     adds them (one MMA per k-step for both terms)
 //   P  = exp(S - m)   online softmax on the accumulator fragments: head g's 8
 //                     scores sit in the 4 lanes of quad g (2 each)
 //   O^T += V^T P^T    m16n8k8, V fragments by ldmatrix.trans; the B fragment
-//                     of P^T is the lane's own pair of probabilities
-// Q and P enter as hi/lo bf16 pairs (two MMAs each); K and V are exact bf16.
-// Positions >= n are masked; their rows are read from position n - 1 so
-// every value stays finite.  Lane (g, t) keeps head g's running max and sum
-// (m_run, l_run) and o[j] = O^T rows (16 j + g, 16 j + g + 8), heads
-// (2 t, 2 t + 1).
+//                     of P^T is the lane's own pair of probabilities.  pk (at
+//                     most 4 heads): P's hi term in columns h < 4 and its lo
+//                     term in columns h + 4 of the same MMA, added once at the
+//                     end of the task; else one MMA per term.
+// K and V are exact bf16.  Positions >= n are masked; their rows are read
+// from position n - 1 so every value stays finite.  Lane (g, t) keeps head
+// g's running max and sum (m_run, l_run) and o[j] = O^T rows (16 j + g,
+// 16 j + g + 8), columns (2 t, 2 t + 1).
 // Byte offset of (row r, 16-byte chunk c16 of the head dims) in a K or V
 // tile.  SWZ: D / 64 TMA boxes of 64 dims x `rows` rows with the 128-byte
 // swizzle (chunk c of row r stored at chunk c ^ (r mod 8) of its 128-byte
@@ -1502,29 +1507,29 @@ __device__ __forceinline__ uint32_t kv_off(int r, int c16, int rows) {
 
 template <int D, bool SWZ>
 __device__ __forceinline__ void attn_block_mma(uint32_t kbase, uint32_t vbase, int rows, int j0,
-                                               int n, const uint32_t (&qh)[D / 16][2],
+                                               int n, bool pk, const uint32_t (&qh)[D / 16][2],
                                                const uint32_t (&ql)[D / 16][2], float &m_run,
                                                float &l_run, float (&o)[D / 16][4]) {
   const int lane = threadIdx.x & 31, t = lane & 3;
   // ldmatrix rows: 8 consecutive positions (distinct r mod 8: no bank conflicts)
   const int pos = min(j0 + (lane & 7), n - 1);
   const int mat = lane >> 3;  // the 8 x 8 matrix this lane addresses
-  // four independent accumulation chains (hi/lo x even/odd k-step), summed
-  float sa[4][4];
+  // two independent accumulation chains (even / odd k-step), summed
+  float sa[2][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) sa[i][0] = sa[i][1] = sa[i][2] = sa[i][3] = 0.f;
+  for (int i = 0; i < 2; ++i) sa[i][0] = sa[i][1] = sa[i][2] = sa[i][3] = 0.f;
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {  // 32 dims (two k-steps) per ldmatrix.x4
     uint32_t b[4];
     ldmatrix_x4(b, kbase + kv_off<D, SWZ>(pos, 4 * c + mat, rows));
-    mma_bf16_top(sa[0], qh[2 * c][0], qh[2 * c][1], b[0], b[1]);
-    mma_bf16_top(sa[1], ql[2 * c][0], ql[2 * c][1], b[0], b[1]);
-    mma_bf16_top(sa[2], qh[2 * c + 1][0], qh[2 * c + 1][1], b[2], b[3]);
-    mma_bf16_top(sa[3], ql[2 * c + 1][0], ql[2 * c + 1][1], b[2], b[3]);
+    mma_bf16(sa[0], make_uint4(qh[2 * c][0], ql[2 * c][0], qh[2 * c][1], ql[2 * c][1]),
+             make_uint2(b[0], b[1]));
+    mma_bf16(sa[1], make_uint4(qh[2 * c + 1][0], ql[2 * c + 1][0], qh[2 * c + 1][1], ql[2 * c + 1][1]),
+             make_uint2(b[2], b[3]));
   }
   float s[2];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) s[i] = (sa[0][i] + sa[2][i]) + (sa[1][i] + sa[3][i]);
+  for (int i = 0; i < 2; ++i) s[i] = (sa[0][i] + sa[1][i]) + (sa[0][i + 2] + sa[1][i + 2]);
   const bool v0 = j0 + 2 * t < n, v1 = j0 + 2 * t + 1 < n;
   const float s0 = v0 ? s[0] : -INFINITY, s1 = v1 ? s[1] : -INFINITY;
   float mx = fmaxf(s0, s1);
@@ -1540,9 +1545,11 @@ __device__ __forceinline__ void attn_block_mma(uint32_t kbase, uint32_t vbase, i
   m_run = m_new;
   uint32_t ph, pl;
   split_pair(p0, p1, ph, pl);
-  // rescale factors of the heads 2t, 2t + 1 this lane accumulates
-  const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * t);
-  const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
+  // rescale factors of the heads of columns 2t, 2t + 1 (column c is head
+  // c & 3 when P is packed)
+  const int c0 = pk ? (2 * t) & 3 : 2 * t;
+  const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
+  const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) {
     o[j][0] *= a0;
@@ -1550,14 +1557,22 @@ __device__ __forceinline__ void attn_block_mma(uint32_t kbase, uint32_t vbase, i
     o[j][2] *= a0;
     o[j][3] *= a1;
   }
+  // packed: lanes of quads 4..7 supply the lo term of head g - 4
+  const uint32_t pl_up = __shfl_xor_sync(0xffffffffu, pl, 16);
+  const uint32_t pb = (lane >> 2) < 4 ? ph : pl_up;
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {  // two 16-dim m-tiles per ldmatrix.x4.trans
     uint32_t v[4];
     ldmatrix_x4_trans(v, vbase + kv_off<D, SWZ>(pos, 4 * c + mat, rows));
-    mma_bf16_k8(o[2 * c], v[0], v[1], ph);
-    mma_bf16_k8(o[2 * c], v[0], v[1], pl);
-    mma_bf16_k8(o[2 * c + 1], v[2], v[3], ph);
-    mma_bf16_k8(o[2 * c + 1], v[2], v[3], pl);
+    if (pk) {
+      mma_bf16_k8(o[2 * c], v[0], v[1], pb);
+      mma_bf16_k8(o[2 * c + 1], v[2], v[3], pb);
+    } else {
+      mma_bf16_k8(o[2 * c], v[0], v[1], ph);
+      mma_bf16_k8(o[2 * c], v[0], v[1], pl);
+      mma_bf16_k8(o[2 * c + 1], v[2], v[3], ph);
+      mma_bf16_k8(o[2 * c + 1], v[2], v[3], pl);
+    }
   }
 }
 
@@ -1656,6 +1671,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
+  const bool pk = rep <= 4;  // P's hi and lo terms share one MMA
   trace_mark(p, sm, 0);
 
   const int cached = a.cached_end - a.p0;
@@ -1674,15 +1690,22 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     const int base = st * (p.pps / NP);
     for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * NP; j0 < n;
          j0 += kComputeWarps * NP)
-      attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, qh, ql, m_run, l_run, o);
+      attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
     release_stage(sm, p, k);
     ++k;
   }
   // the new row: one more block, on the warp after the last cached block
   if (a.has_new && warp == ((cached + NP - 1) / NP) % kComputeWarps)
-    attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, qh, ql, m_run, l_run, o);
+    attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, pk, qh, ql, m_run, l_run,
+                             o);
 
   trace_mark(p, sm, 1);
+  if (pk) {  // add the lo-term columns h + 4 into the columns h of lanes tq < 2
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[j][i] += __shfl_down_sync(0xffffffffu, o[j][i], 2);
+  }
   // every warp's state to shared memory: o (heads 2 tq, 2 tq + 1), then the
   // running max and sum of head gq_row
   static_assert(kStateSlots == kComputeWarps, "one state slot per warp");
