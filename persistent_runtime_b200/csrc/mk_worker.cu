@@ -1576,6 +1576,102 @@ __device__ __forceinline__ void attn_block_mma(uint32_t kbase, uint32_t vbase, i
   }
 }
 
+// Two 8-position tiles [j0, j0 + 8) and [j0 + 8, j0 + 16) at once: the same
+// S and softmax steps on both (independent MMA chains), one rescale of o,
+// and O^T += V^T P^T as m16n8k16 over the 16 positions (the B fragment of
+// P^T is the lane's own probabilities of both tiles).
+template <int D, bool SWZ>
+__device__ __forceinline__ void attn_block16_mma(uint32_t kbase, uint32_t vbase, int rows, int j0,
+                                                 int n, bool pk, const uint32_t (&qh)[D / 16][2],
+                                                 const uint32_t (&ql)[D / 16][2], float &m_run,
+                                                 float &l_run, float (&o)[D / 16][4]) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  const int pa = min(j0 + (lane & 7), n - 1), pb = min(j0 + 8 + (lane & 7), n - 1);
+  const int mat = lane >> 3;
+  float sa[2][4], sb[2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) sa[i][r] = sb[i][r] = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t ka[4], kb[4];
+    ldmatrix_x4(ka, kbase + kv_off<D, SWZ>(pa, 4 * c + mat, rows));
+    ldmatrix_x4(kb, kbase + kv_off<D, SWZ>(pb, 4 * c + mat, rows));
+    const uint4 q0 = make_uint4(qh[2 * c][0], ql[2 * c][0], qh[2 * c][1], ql[2 * c][1]);
+    const uint4 q1 = make_uint4(qh[2 * c + 1][0], ql[2 * c + 1][0], qh[2 * c + 1][1], ql[2 * c + 1][1]);
+    mma_bf16(sa[0], q0, make_uint2(ka[0], ka[1]));
+    mma_bf16(sb[0], q0, make_uint2(kb[0], kb[1]));
+    mma_bf16(sa[1], q1, make_uint2(ka[2], ka[3]));
+    mma_bf16(sb[1], q1, make_uint2(kb[2], kb[3]));
+  }
+  float sv[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    sv[i] = (sa[0][i] + sa[1][i]) + (sa[0][i + 2] + sa[1][i + 2]);
+    sv[i + 2] = (sb[0][i] + sb[1][i]) + (sb[0][i + 2] + sb[1][i + 2]);
+  }
+  bool ok[4];
+  ok[0] = j0 + 2 * t < n;
+  ok[1] = j0 + 2 * t + 1 < n;
+  ok[2] = j0 + 8 + 2 * t < n;
+  ok[3] = j0 + 9 + 2 * t < n;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sv[i] = ok[i] ? sv[i] : -INFINITY;
+    mx = fmaxf(mx, sv[i]);
+  }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float m_new = fmaxf(m_run, mx);  // finite: position j0 < n is valid
+  const float alpha = m_run == -INFINITY ? 0.f : __expf(m_run - m_new);
+  float pr[4], sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pr[i] = ok[i] ? __expf(sv[i] - m_new) : 0.f;
+    sum += pr[i];
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  l_run = l_run * alpha + sum;
+  m_run = m_new;
+  uint32_t pha, pla, phb, plb;
+  split_pair(pr[0], pr[1], pha, pla);
+  split_pair(pr[2], pr[3], phb, plb);
+  const int c0 = pk ? (2 * t) & 3 : 2 * t;
+  const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
+  const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
+#pragma unroll
+  for (int j = 0; j < D / 16; ++j) {
+    o[j][0] *= a0;
+    o[j][1] *= a1;
+    o[j][2] *= a0;
+    o[j][3] *= a1;
+  }
+  const bool upper = (lane >> 2) < 4;
+  const uint32_t pla_up = __shfl_xor_sync(0xffffffffu, pla, 16);
+  const uint32_t plb_up = __shfl_xor_sync(0xffffffffu, plb, 16);
+  const uint2 bp = make_uint2(upper ? pha : pla_up, upper ? phb : plb_up);
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t va[4], vb[4];
+    ldmatrix_x4_trans(va, vbase + kv_off<D, SWZ>(pa, 4 * c + mat, rows));
+    ldmatrix_x4_trans(vb, vbase + kv_off<D, SWZ>(pb, 4 * c + mat, rows));
+    const uint4 v0 = make_uint4(va[0], va[1], vb[0], vb[1]);
+    const uint4 v1 = make_uint4(va[2], va[3], vb[2], vb[3]);
+    if (pk) {
+      mma_bf16(o[2 * c], v0, bp);
+      mma_bf16(o[2 * c + 1], v1, bp);
+    } else {
+      mma_bf16(o[2 * c], v0, make_uint2(pha, phb));
+      mma_bf16(o[2 * c], v0, make_uint2(pla, plb));
+      mma_bf16(o[2 * c + 1], v1, make_uint2(pha, phb));
+      mma_bf16(o[2 * c + 1], v1, make_uint2(pla, plb));
+    }
+  }
+}
+
 // Decode attention for one (sequence b, kv head g, split s): q/k RMSNorm and
 // RoPE prologue, K/V append, then every warp runs flash-decoding style over
 // its own 8-position blocks on tensor cores (no CTA barrier inside the loop)
@@ -1672,6 +1768,8 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
   const bool pk = rep <= 4;  // P's hi and lo terms share one MMA
+  // 16-position blocks when the stages hold whole ones (8-position otherwise)
+  const bool np16 = p.pps % (2 * NP) == 0;
   trace_mark(p, sm, 0);
 
   const int cached = a.cached_end - a.p0;
@@ -1687,15 +1785,23 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     // (warp w takes global blocks w, w + 8, ...), so a stage whose block
     // count is not a multiple of 8 does not leave the same warps idle every
     // time; warps drift apart by at most the ring depth
-    const int base = st * (p.pps / NP);
-    for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * NP; j0 < n;
-         j0 += kComputeWarps * NP)
-      attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
+    if (np16) {
+      const int base = st * (p.pps / (2 * NP));
+      for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * 2 * NP;
+           j0 < n; j0 += kComputeWarps * 2 * NP)
+        attn_block16_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
+    } else {
+      const int base = st * (p.pps / NP);
+      for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * NP; j0 < n;
+           j0 += kComputeWarps * NP)
+        attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
+    }
     release_stage(sm, p, k);
     ++k;
   }
   // the new row: one more block, on the warp after the last cached block
-  if (a.has_new && warp == ((cached + NP - 1) / NP) % kComputeWarps)
+  const int blk = np16 ? 2 * NP : NP;
+  if (a.has_new && warp == ((cached + blk - 1) / blk) % kComputeWarps)
     attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, pk, qh, ql, m_run, l_run,
                              o);
 
