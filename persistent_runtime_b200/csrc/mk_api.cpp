@@ -416,7 +416,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     // multiple of 8 (one share per warp), at most 8 per warp and stage
     const int units = t.ring_stage_bytes / 512;
     auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
-    auto kcb_of = [&](int mb) { return std::min(mk::kMmaMaxKCB, units / mb / 8 * 8); };
+    auto kcb_of = [&](int mb) { return std::min(8 * mk::mma_max_kpw(nn), units / mb / 8 * 8); };
     p.mma = 1;
     p.nn = nn;
     p.n_parts = n_parts;

@@ -1090,10 +1090,10 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 // activations are written earlier in this step by other SMs, so they are read
 // through L2 (never from a possibly stale L1 line).
 template <int NN>
-__device__ __forceinline__ void load_bfrag(uint4 (&bf)[kMmaMaxKPW][NN], const uint16_t *xb,
+__device__ __forceinline__ void load_bfrag(uint4 (&bf)[mma_max_kpw(NN)][NN], const uint16_t *xb,
                                            int kb0, int kpw, int warp, int lane) {
 #pragma unroll
-  for (int j = 0; j < kMmaMaxKPW; ++j) {
+  for (int j = 0; j < mma_max_kpw(NN); ++j) {
     if (j < kpw) {
 #pragma unroll
       for (int n = 0; n < NN; ++n)
@@ -1109,7 +1109,7 @@ __device__ __forceinline__ void load_bfrag(uint4 (&bf)[kMmaMaxKPW][NN], const ui
 // the next stage's first kpw_n k-blocks are refilled after their last use.
 template <int NN, int MBF, int KPWF, bool kGuard>
 __device__ __forceinline__ void mma_stage_fixed(float (&acc)[kMmaMaxMB][NN][4],
-                                                uint4 (&bc)[kMmaMaxKPW][NN], const uint8_t *slot,
+                                                uint4 (&bc)[mma_max_kpw(NN)][NN], const uint8_t *slot,
                                                 const uint16_t *xn, int kpw_n, int warp, int lane) {
   constexpr int NKB = 8 * KPWF;
 #pragma unroll
@@ -1133,7 +1133,7 @@ __device__ __forceinline__ void mma_stage_fixed(float (&acc)[kMmaMaxMB][NN][4],
   }
   // a next stage with more k-blocks (the first chunk after a short last one)
 #pragma unroll
-  for (int j = KPWF; j < (kGuard ? kMmaMaxKPW : 0); ++j) {
+  for (int j = KPWF; j < (kGuard ? mma_max_kpw(NN) : 0); ++j) {
     if (j < kpw_n) {
 #pragma unroll
       for (int n = 0; n < NN; ++n)
@@ -1188,7 +1188,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
   const int N = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
 
   if (!dep_wait()) return false;
-  uint4 bc[kMmaMaxKPW][NN];
+  uint4 bc[mma_max_kpw(NN)][NN];
   load_bfrag<NN>(bc, xb, 0, min(mt.kcb, mt.KB) >> 3, warp, lane);
   float inv = 1.f;
   if (ssp) {
@@ -1227,7 +1227,15 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
       trace_first_stage(p, sm, st);
       const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
       const bool same = kpw_n == kpw;  // the next stage refills every fragment
-      if (same && kpw == 3 && nm == 2) {
+      if (NN == 1 && same && kpw == 6 && nm == 2) {
+        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && same && kpw == 4 && nm == 3) {
+        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && kpw == 6 && nm == 2) {
+        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && kpw == 4 && nm == 3) {
+        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 3 && nm == 2) {
         mma_stage_fixed<NN, 2, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
       } else if (same && kpw == 3 && nm == 3) {
         mma_stage_fixed<NN, 3, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
@@ -1243,7 +1251,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
         mma_stage_fixed<NN, 3, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
       } else {
 #pragma unroll
-      for (int j = 0; j < kMmaMaxKPW; ++j) {
+      for (int j = 0; j < mma_max_kpw(NN); ++j) {
         if (j < kpw) {
           const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
 #pragma unroll
@@ -2290,9 +2298,10 @@ __device__ __noinline__ void argmax_task(const Params &p, int32_t *tok_out) {
 // The worker kernel
 // ---------------------------------------------------------------------------
 // kMma: projections on tensor cores (batch >= 2) instead of the CUDA-core
-// GEMV; the two modes are separate instantiations so that each gets its own
-// register allocation.
-template <bool kMma>
+// GEMV; kNN: the operand's 8-column tiles (1 or 2) of the tensor-core
+// projections (0 at batch 1).  The three modes are separate instantiations
+// so that each gets its own register allocation.
+template <bool kMma, int kNN>
 __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const Smem sm = carve(smem_raw, p);
@@ -2386,7 +2395,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           break;
         case 2: case 5: case 6: case 7: case 8: {
           if constexpr (kMma) {
-            ok = p.nn == 2 ? mma_task<2>(p, sm, t, k, id, dw) : mma_task<1>(p, sm, t, k, id, dw);
+            ok = mma_task<kNN == 2 ? 2 : 1>(p, sm, t, k, id, dw);
           } else {
             const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
             const int nch = K >> 3;
@@ -2501,38 +2510,46 @@ size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int
   return smem_offsets(stages, stage_bytes, pps, head_dim, rep_p).total;
 }
 
+// The instantiation for a parameter block's mode.
+static const void *worker_fn(const Params &p) {
+  if (!p.mma) return (const void *)mk_worker_kernel<false, 0>;
+  return p.nn == 2 ? (const void *)mk_worker_kernel<true, 2> : (const void *)mk_worker_kernel<true, 1>;
+}
+
 cudaError_t worker_configure(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(mk_worker_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(mk_worker_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem);
+  const void *fns[] = {(const void *)mk_worker_kernel<false, 0>, (const void *)mk_worker_kernel<true, 1>,
+                       (const void *)mk_worker_kernel<true, 2>};
+  for (const void *fn : fns) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t worker_max_blocks(int *blocks, size_t smem) {
-  int a = 0, b = 0;
-  cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, mk_worker_kernel<false>, kThreads, smem);
-  if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mk_worker_kernel<true>, kThreads, smem);
-  *blocks = a < b ? a : b;
-  return e;
+  const void *fns[] = {(const void *)mk_worker_kernel<false, 0>, (const void *)mk_worker_kernel<true, 1>,
+                       (const void *)mk_worker_kernel<true, 2>};
+  int lo = 1 << 30;
+  for (const void *fn : fns) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    lo = n < lo ? n : lo;
+  }
+  *blocks = lo;
+  return cudaSuccess;
 }
 
 // Persistent launch: one cooperative grid of `workers` CTAs.
 cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream) {
   void *args[] = {const_cast<Params *>(&p)};
-  const void *fn = p.mma ? (const void *)mk_worker_kernel<true> : (const void *)mk_worker_kernel<false>;
-  return cudaLaunchCooperativeKernel(fn, dim3(workers), dim3(kThreads), args, smem, stream);
+  return cudaLaunchCooperativeKernel(worker_fn(p), dim3(workers), dim3(kThreads), args, smem, stream);
 }
 
 // Per-operator launch: one CTA per task of the operator.
 cudaError_t launch_tasks(const Params &p, int n_ctas, size_t smem, cudaStream_t stream) {
-  if (p.mma)
-    mk_worker_kernel<true><<<n_ctas, kThreads, smem, stream>>>(p);
-  else
-    mk_worker_kernel<false><<<n_ctas, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  void *args[] = {const_cast<Params *>(&p)};
+  return cudaLaunchKernel(worker_fn(p), dim3(n_ctas), dim3(kThreads), args, smem, stream);
 }
 
 }  // namespace mk

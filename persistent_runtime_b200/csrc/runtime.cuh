@@ -22,8 +22,10 @@ constexpr int kMaxHeadDim = 128;
 constexpr int kMaxBatch = 16;
 // Tensor-core projections (batch >= 2): mma.sync m16n8k16, bf16 in, fp32 out.
 constexpr int kMmaMaxMB = 6;    // 16-row m-tiles per row block (accumulators per warp)
-constexpr int kMmaMaxKPW = 3;   // 16-column k-blocks per warp and ring stage
-constexpr int kMmaMaxKCB = 8 * kMmaMaxKPW;  // k-blocks per ring stage
+// 16-column k-blocks per warp and ring stage: a stage's B fragments take
+// kpw x nn x 4 registers per thread, so one column tile (batch <= 8) affords
+// twice as many as two
+__host__ __device__ constexpr int mma_max_kpw(int nn) { return nn == 1 ? 6 : 3; }
 constexpr int kMmaCredFloats = kComputeWarps * 4 * 16 * 9;  // cross-warp reduction buffer
 
 // Device status words: [0] status code, [1] task, [2] event, [3] block.

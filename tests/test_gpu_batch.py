@@ -114,3 +114,19 @@ def test_qwen3_8b_batched_full_size_sampled_sequences(w, seqs):
             g = synth.bf16_to_f32(dev[:, b, :, L].cpu().numpy().view(np.uint16)).astype(np.float64)
             r = synth.bf16_to_f32(host[:, b, :, L]).astype(np.float64)
             assert np.all(np.abs(g - r) <= 1e-2 * np.max(np.abs(r), axis=-1, keepdims=True))
+
+
+def test_tiny_batch_eight_position_attention_blocks():
+    # 10 KB ring stages: K/V stages of 40 positions (not a whole number of
+    # 16-position blocks), so the tensor-core attention takes its 8-position
+    # blocks; the projections run 1- and 2-m-tile stages of 8 and 16 k-blocks
+    w = tiny_batch(8, lo=0, hi=200)
+    c = Case(w, seed=34, extra_cap=2, ring_stage_bytes=10240, ring_stages=8)
+    chunk = c.mk.graph().tiling[6]
+    pps = min(256, chunk, 10240 // (4 * w.head_dim) // 8 * 8)
+    assert pps % 16 != 0
+    k, v, lens = c.k.copy(), c.v.copy(), c.lens.copy()
+    got = c.gpu_step()
+    ref = c.oracle_step(k=k, v=v, lens=lens)
+    compare_step(ref, got, w, "tiny-b8-np8")
+    kv_rows_close(c, k, v, c.lens, bf16_inputs=True)
