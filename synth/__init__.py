@@ -121,7 +121,10 @@ Q8B_4L = Q8B.with_(name="qwen3-8b-4layer", n_layers=4)
 # cached rows per sequence (about 4.5 GB on the device).
 Q8B_B16_4L = Q8B_B16.with_(name="qwen3-8b-b16-4layer", n_layers=4, kv_len=1024)
 
-WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16, Q8B_4L, Q8B_B16_4L)}
+# The same at batch 8 (the one-column-tile instantiation of the batched kernel).
+Q8B_B8_4L = Q8B_B8.with_(name="qwen3-8b-b8-4layer", n_layers=4, kv_len=1024)
+
+WORKLOADS = {w.name: w for w in (TINY, Q06B, Q8B, Q8B_B8, Q8B_B16, Q8B_4L, Q8B_B16_4L, Q8B_B8_4L)}
 
 # ----------------------------------------------------------------------------
 # Stream ids (one counter stream per tensor)
