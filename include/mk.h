@@ -95,7 +95,10 @@ typedef struct {
   int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
   int ring_stages;           /* shared-memory weight ring depth (4) */
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
-  int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring (0 = off) */
+  int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while a
+                                landed stage stays unreleased for over 1.5 us (the compute
+                                warps wait on an event or run attention); default 524288 at
+                                batch 1, off at batch >= 2; negative = off */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
   int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the
                                 paged pools (a multiple of 64), see mk_decode_steps_paged */

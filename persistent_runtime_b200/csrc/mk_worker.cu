@@ -240,15 +240,6 @@ __device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(b));
 }
 
-// m16n8k16 with the A rows g + 8 zero (a1 = a3 = 0).
-__device__ __forceinline__ void mma_bf16_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                             uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-}
-
 // Four 8 x 8 b16 matrices from shared memory; lanes 8i..8i+7 give the row
 // addresses of matrix i.  Plain: thread l receives row l / 4, columns
 // 2 (l % 4) and 2 (l % 4) + 1; .trans: rows 2 (l % 4), 2 (l % 4) + 1 of
@@ -653,6 +644,8 @@ __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
 // ---------------------------------------------------------------------------
 // Producer: one thread streams every stage of the worker's queue.
 // ---------------------------------------------------------------------------
+constexpr uint64_t kPrefetchHoldNs = 1500;  // see producer_loop
+
 struct Queue {
   int first, stride, count;  // tasks first, first + stride, ... (count of them)
 };
@@ -663,10 +656,10 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
   // L2 prefetch cursor (task pf_n, stage pf_st, global stage index pf_k) in
-  // the worker's stream of stages, across task boundaries.  While the ring is
-  // full of landed stages that the compute warps have not consumed yet (they
-  // wait on an event or run a compute-heavy body, so HBM has spare capacity)
-  // the producer prefetches the next stages into L2, up to
+  // the worker's stream of stages, across task boundaries.  While the ring's
+  // oldest stage has landed and stayed unconsumed for over kPrefetchHoldNs
+  // (the compute warps wait on an event or run attention, so HBM has spare
+  // capacity) the producer prefetches the next stages into L2, up to
   // l2_prefetch_bytes ahead of the ring.
   const long long dist = p.l2_prefetch_bytes;
   const uint64_t pol = stream_policy(p.evict_first != 0);
@@ -719,17 +712,24 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       const uint32_t use = k / NS;
       if (use > 0) {
         const uint32_t par = (use - 1) & 1u;
-        uint64_t t0 = 0;
+        uint64_t t0 = 0, t_held = 0;
         uint32_t spins = 0;
         while (!mbar_test(&sm.empty[slot], par)) {
           if (sm.ctl[kAbort]) goto out;
           ++spins;
           // prefetch only while the consumer, not HBM, holds the ring back:
           // the oldest stage in flight (this slot's previous use) has landed
-          // but is not released yet (the compute warps wait on an event or
-          // are busy with a compute-heavy body)
+          // and stayed unreleased for over kPrefetchHoldNs (the compute warps
+          // wait on an event or run attention; a stage of streaming work is
+          // released well within that time)
+          bool idle = false;
           if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count &&
               mbar_test(&sm.full[slot], par)) {
+            const uint64_t now = global_timer();
+            if (t_held == 0) t_held = now;
+            idle = now - t_held > kPrefetchHoldNs;
+          }
+          if (idle) {
             if (pfs.nst < 0) pfs = task_stream<kMma>(p, p.tasks[q.first + pf_n * q.stride]);
             if (pf_st >= pfs.nst) {
               ++pf_n;
