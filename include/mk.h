@@ -98,7 +98,9 @@ typedef struct {
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while a
                                 landed stage stays unreleased for over 1.5 us (the compute
                                 warps wait on an event or run attention); default 524288 at
-                                batch 1, off at batch >= 2; negative = off */
+                                batch 1 (single-step launches; mk_decode_steps* with more than
+                                one step run without it unless it is set), off at batch >= 2;
+                                negative = off */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
   int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the
                                 paged pools (a multiple of 64), see mk_decode_steps_paged */

@@ -118,6 +118,7 @@ mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int
   if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
   h->cfg = *cfg;
   h->tune = fill_defaults(tuning, cfg->batch);
+  h->prefetch_defaulted = !tuning || tuning->l2_prefetch_bytes == 0;
   h->tune.num_workers = num_workers;
   mk_status s = plan(cfg, h->tune, num_workers, h);
   if (s != MK_OK) {
@@ -170,6 +171,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   h->device = device;
   h->cfg = *cfg;
   h->tune = fill_defaults(tuning, cfg->batch);
+  h->prefetch_defaulted = !tuning || tuning->l2_prefetch_bytes == 0;
   mk_tuning &t = h->tune;
   const mk_model_config &c = *cfg;
   const int D = c.head_dim;
@@ -703,6 +705,15 @@ mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_to
   return MK_OK;
 }
 
+// Multi-step launches run without the default idle-window L2 prefetch: the
+// step boundary inside one launch is a long idle window, and prefetching
+// through it cost more than it gave (Qwen3-8B bs1, one box: 3154 us per step
+// with it, 3117 us without; single launches 3097 us with it, 3124 without).
+// An explicit l2_prefetch_bytes is kept.
+static void multi_step_prefetch(const mk_handle *h, int n_steps, Params *p) {
+  if (n_steps > 1 && h->prefetch_defaulted) p->l2_prefetch_bytes = 0;
+}
+
 mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
                           int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
                           void *d_v_cache, float *d_logits, void *stream) {
@@ -713,6 +724,7 @@ mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
   p.logits = d_logits;
   p.persistent = 1;
   p.n_steps = n_steps;
+  multi_step_prefetch(h, n_steps, &p);
   cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
@@ -732,6 +744,7 @@ mk_status mk_decode_steps_paged(mk_handle *h, int n_steps, const int32_t *d_toke
   p.logits = d_logits;
   p.persistent = 1;
   p.n_steps = n_steps;
+  multi_step_prefetch(h, n_steps, &p);
   cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");

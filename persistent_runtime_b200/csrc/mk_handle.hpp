@@ -32,6 +32,7 @@ std::string encode_kv_maps(const mk_handle *h, const void *k_cache, const void *
 struct mk_handle {
   mk_model_config cfg{};
   mk_tuning tune{};
+  bool prefetch_defaulted = false;  // l2_prefetch_bytes was left to its default
   mk::TaskGraph graph;
   bool host_only = true;
   int device = -1;
