@@ -139,6 +139,10 @@ typedef struct {
   const int32_t *edge_src, *edge_dst; /* raw data dependencies, final task ids */
   /* tiling chosen for the decode graph (0 for generic graphs) */
   int32_t qkv_rows, o_rows, gu_rows, down_rows, lm_rows, attn_splits, attn_chunk;
+  /* batch >= 2: tensor-core tiles of QKV, O, GATE_UP, DOWN, LM_HEAD (in that
+   * order): 16-row m-tiles per row block and 16-column k-blocks per ring
+   * stage for the handle's ring stage size (0 at batch 1) */
+  int32_t mma_mb[5], mma_kcb[5];
 } mk_graph_view;
 
 /* Sizes and roofline inputs of a built handle. */

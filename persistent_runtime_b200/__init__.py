@@ -73,7 +73,8 @@ class GraphView(ctypes.Structure):
                              "task_trig", "event_count", "event_first", "event_last",
                              "edge_src", "edge_dst")] + [
         (n, ctypes.c_int32) for n in ("qkv_rows", "o_rows", "gu_rows", "down_rows", "lm_rows",
-                                      "attn_splits", "attn_chunk")]
+                                      "attn_splits", "attn_chunk")] + [
+        ("mma_mb", ctypes.c_int32 * 5), ("mma_kcb", ctypes.c_int32 * 5)]
 
 
 class Info(ctypes.Structure):
@@ -162,6 +163,7 @@ class Graph:
     edge_dst: np.ndarray
     num_workers: int
     tiling: tuple
+    mma_tiling: tuple = ()  # ((mb, kcb) of QKV, O, GATE_UP, DOWN, LM_HEAD) at batch >= 2
 
     @property
     def n_tasks(self):
@@ -185,7 +187,8 @@ def _export(h) -> Graph:
                    ("event_count", "event_first", "event_last")),
                  arr(v.edge_src, v.n_edges), arr(v.edge_dst, v.n_edges), v.num_workers,
                  (v.qkv_rows, v.o_rows, v.gu_rows, v.down_rows, v.lm_rows, v.attn_splits,
-                  v.attn_chunk))
+                  v.attn_chunk),
+                 tuple((int(v.mma_mb[i]), int(v.mma_kcb[i])) for i in range(5)))
 
 
 def plan_graph(w, kv_capacity: int, num_workers: int, **tuning) -> Graph:

@@ -84,6 +84,27 @@ std::string check_gpu_shape(const mk_model_config &c) {
   return "";
 }
 
+// Tensor-core tiling of the batched projections (QKV, O, GATE_UP, DOWN,
+// LM_HEAD, in that order).  m-tiles per row block: the task's rows up to the
+// accumulator limit; k-blocks per ring stage: what a stage holds for that
+// many m-tiles, a multiple of 8 (one share per warp), at most
+// mma_max_kpw(nn) per warp (the B-fragment registers of one stage).
+struct MmaTiling {
+  int mb[5], kcb[5];
+};
+
+MmaTiling mma_tiling(const mk::Tiling &T, int ring_stage_bytes, int nn) {
+  const int units = ring_stage_bytes / 512;
+  auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
+  const int rows[5] = {T.qkv_rows, T.o_rows, 2 * T.gu_rows, T.down_rows, T.lm_rows};
+  MmaTiling m{};
+  for (int i = 0; i < 5; ++i) {
+    m.mb[i] = mb_of(rows[i]);
+    m.kcb[i] = std::min(8 * mk::mma_max_kpw(nn), units / m.mb[i] / 8 * 8);
+  }
+  return m;
+}
+
 mk::ModelShape shape_of(const mk_model_config &c) {
   return mk::ModelShape{c.n_layers, c.hidden, c.n_q_heads, c.n_kv_heads, c.head_dim,
                         c.ffn,      c.vocab,  c.batch,     c.kv_capacity};
@@ -418,25 +439,20 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     return fail(nullptr, MK_ERR_ARG, "ring stage smaller than 8 K/V rows");
   }
   if (mma) {
-    // m-tiles per row block: the task's rows up to the accumulator limit;
-    // k-blocks per stage: what the stage holds for that many m-tiles, a
-    // multiple of 8 (one share per warp), at most 8 per warp and stage
-    const int units = t.ring_stage_bytes / 512;
-    auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
-    auto kcb_of = [&](int mb) { return std::min(8 * mk::mma_max_kpw(nn), units / mb / 8 * 8); };
+    const MmaTiling mt = mma_tiling(T, t.ring_stage_bytes, nn);
     p.mma = 1;
     p.nn = nn;
     p.n_parts = n_parts;
-    p.mb_qkv = mb_of(T.qkv_rows);
-    p.mb_o = mb_of(T.o_rows);
-    p.mb_gu = mb_of(2 * T.gu_rows);
-    p.mb_down = mb_of(T.down_rows);
-    p.mb_lm = mb_of(T.lm_rows);
-    p.kcb_qkv = kcb_of(p.mb_qkv);
-    p.kcb_o = kcb_of(p.mb_o);
-    p.kcb_gu = kcb_of(p.mb_gu);
-    p.kcb_down = kcb_of(p.mb_down);
-    p.kcb_lm = kcb_of(p.mb_lm);
+    p.mb_qkv = mt.mb[0];
+    p.mb_o = mt.mb[1];
+    p.mb_gu = mt.mb[2];
+    p.mb_down = mt.mb[3];
+    p.mb_lm = mt.mb[4];
+    p.kcb_qkv = mt.kcb[0];
+    p.kcb_o = mt.kcb[1];
+    p.kcb_gu = mt.kcb[2];
+    p.kcb_down = mt.kcb[3];
+    p.kcb_lm = mt.kcb[4];
     p.xfb = reinterpret_cast<uint16_t *>(base + o_xa[Ly]);
     p.ssf = reinterpret_cast<float *>(base + o_ssa[Ly]);
     if (std::min({p.kcb_qkv, p.kcb_o, p.kcb_gu, p.kcb_down, p.kcb_lm}) < 8) {
@@ -833,6 +849,13 @@ mk_status mk_graph_export(const mk_handle *h, mk_graph_view *out) {
   out->lm_rows = T.lm_rows;
   out->attn_splits = T.attn_splits;
   out->attn_chunk = T.attn_chunk;
+  if (h->cfg.batch > 1 && T.qkv_rows > 0) {
+    const MmaTiling mt = mma_tiling(T, h->tune.ring_stage_bytes, (h->cfg.batch + 7) / 8);
+    for (int i = 0; i < 5; ++i) {
+      out->mma_mb[i] = mt.mb[i];
+      out->mma_kcb[i] = mt.kcb[i];
+    }
+  }
   return MK_OK;
 }
 
