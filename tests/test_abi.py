@@ -42,3 +42,33 @@ def test_bad_arguments_are_rejected_without_a_device():
     lib.mk_destroy(None)
     with pytest.raises(prb.MkError):
         prb.graph_from_edges([0, 1], [0, 0], [(1, 0)])
+
+
+STRUCTS = {"mk_model_config": prb.ModelConfig, "mk_tuning": prb.Tuning, "mk_weights": prb.Weights,
+           "mk_graph_view": prb.GraphView, "mk_info": prb.Info}
+
+
+def test_binding_structures_match_the_header_layouts(tmp_path):
+    # a C program compiled against include/mk.h prints every struct's size and
+    # the offset of each field the ctypes binding declares
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "mk.h"', "int main(void) {"]
+    for cname, py in STRUCTS.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)]).decode().split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l}
+    for cname, py in STRUCTS.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)
