@@ -393,3 +393,97 @@ def test_step_rejects_full_cache_and_bad_tokens():
     with pytest.raises(ValueError):
         m.step(np.array([w.vocab], dtype=np.int32), kl, k, v)
     assert kl[0] == 3
+
+
+# ------------------------------------------------------------ per-head q/k RMSNorm
+def _constant_heads(n_heads, D, H, consts):
+    """Projection rows of head h all equal to consts[h] / H: with x_hat constant
+    (= 1 / sqrt(1 + eps)), head h's output is the constant consts[h] * x_hat."""
+    w = np.zeros((n_heads * D, H), dtype=np.float64)
+    for h, c in enumerate(consts):
+        w[h * D:(h + 1) * D, :] = c / H
+    return bf16_exact(w)
+
+
+def _unit_input(w, weights, tok):
+    weights["embed"] = weights["embed"].copy()
+    weights["embed"][tok[0]] = bf16_exact(np.ones(w.hidden))
+    for lw in weights["layers"]:
+        lw["attn_norm"] = bf16_exact(np.ones(w.hidden))
+    return weights
+
+
+def test_step_k_norm_is_per_head_with_the_k_gain():
+    # Both kv heads project to constants of very different magnitude (0.5 and
+    # -3), the k gain is non-unit and differs from the q gain.  A per-head
+    # norm maps head g to g_k * sign(c_g) * |c_g| / sqrt(c_g^2 + eps); at
+    # kv_len 0 RoPE is the identity, so that is the appended key row (bf16).
+    # A norm over the concatenated heads, a dropped gain, or the q gain in
+    # its place gives other rows.
+    w = synth.TINY.with_(n_layers=1, kv_len=0)
+    D, H = w.head_dim, w.hidden
+    weights = _zero_mixing(synth.make_weights(w, 13))
+    tok = synth.make_tokens(w, 13)
+    weights = _unit_input(w, weights, tok)
+    xh = 1.0 / math.sqrt(1.0 + w.rms_eps)
+    consts = [0.5, -3.0]
+    lw = weights["layers"][0]
+    lw["wk"] = _constant_heads(w.n_kv_heads, D, H, consts)
+    lw["k_norm"] = bf16_exact(0.5 + np.arange(D) / D)
+    lw["q_norm"] = bf16_exact(2.0 - np.arange(D) / D)
+    k = np.zeros((1, 1, w.n_kv_heads, 1, D), dtype=np.uint16)
+    v = np.zeros_like(k)
+    kl = np.array([0], dtype=np.int32)
+    oracle.Model(w, weights, 1).step(tok, kl, k, v)
+    gk = synth.bf16_to_f32(lw["k_norm"]).astype(np.float64)
+    for g, c in enumerate(consts):
+        kc = np.float32(np.float32(c) * np.float32(xh))  # the constant head value
+        expect = gk * float(kc) / math.sqrt(float(kc) ** 2 + w.rms_eps)
+        got = synth.bf16_to_f32(k[0, 0, g, 0]).astype(np.float64)
+        np.testing.assert_allclose(got, synth.bf16_to_f32(bf16_exact(expect)), rtol=0, atol=0)
+        # the two heads differ only by the sign: per-head normalisation
+        assert np.allclose(np.abs(got), gk, rtol=8e-3)
+
+
+def test_step_q_norm_is_per_head_with_the_q_gain():
+    # q head h projects to the constant c_h (magnitudes 0.25 ... 3), the q
+    # gain g_q is non-unit; W_k = W_v = 0, so the new key and value are 0.
+    # With one cached row (K_0, V_0 = 1) the new token at position 1 attends
+    # with probability p_h = sigmoid(s_h) to row 0 and 1 - p_h to the new row,
+    # s_h = rope_1(g_q * sign(c_h) * |c_h| / sqrt(c_h^2 + eps)) . K_0 / sqrt(D).
+    # W_o = I then puts o_h = p_h * 1 into the hidden state: hidden = 1 + p_h.
+    w = synth.TINY.with_(n_layers=1, kv_len=1)
+    D, H, Hq = w.head_dim, w.hidden, w.n_q_heads
+    rep = Hq // w.n_kv_heads
+    weights = _zero_mixing(synth.make_weights(w, 17))
+    tok = synth.make_tokens(w, 17)
+    weights = _unit_input(w, weights, tok)
+    xh = 1.0 / math.sqrt(1.0 + w.rms_eps)
+    consts = [0.25, -3.0, 1.5, -0.5]
+    lw = weights["layers"][0]
+    lw["wq"] = _constant_heads(Hq, D, H, consts)
+    lw["q_norm"] = bf16_exact(0.5 + np.arange(D) / D)
+    lw["k_norm"] = bf16_exact(2.0 - np.arange(D) / D)
+    lw["wo"] = bf16_exact(np.eye(H, w.q_dim))
+    k0 = bf16_exact(np.random.default_rng(3).standard_normal((w.n_kv_heads, D)))
+    k = np.zeros((1, 1, w.n_kv_heads, 2, D), dtype=np.uint16)
+    v = np.zeros_like(k)
+    k[0, 0, :, 0, :] = k0
+    v[0, 0, :, 0, :] = bf16_exact(np.ones(D))
+    kl = np.array([1], dtype=np.int32)
+    out = oracle.Model(w, weights, 2).step(tok, kl, k, v)
+    gq = synth.bf16_to_f32(lw["q_norm"]).astype(np.float64)
+    half = D // 2
+    i = np.arange(half)
+    ang = 1.0 * w.rope_theta ** (-2.0 * i / D)
+    cs, sn = np.cos(ang), np.sin(ang)
+    expect = np.ones(H)
+    for h, c in enumerate(consts):
+        qc = float(np.float32(np.float32(c) * np.float32(xh)))
+        q = gq * qc / math.sqrt(qc * qc + w.rms_eps)
+        qr = np.concatenate([q[:half] * cs - q[half:] * sn, q[half:] * cs + q[:half] * sn])
+        s = qr @ synth.bf16_to_f32(k0[h // rep]).astype(np.float64) / math.sqrt(D)
+        expect[h * D:(h + 1) * D] += 1.0 / (1.0 + math.exp(-s))
+    np.testing.assert_allclose(out["hidden"][0], expect, rtol=2e-6, atol=2e-6)
+    # the appended row is zero (W_k = W_v = 0)
+    assert not synth.bf16_to_f32(k[0, 0, :, 1]).any() and not synth.bf16_to_f32(v[0, 0, :, 1]).any()
