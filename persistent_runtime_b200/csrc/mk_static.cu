@@ -11,13 +11,22 @@
 // a file-scope static array that every GPU loading the library holds until
 // the process exits.  The handle's graph tables, weights and status word are
 // used as they are; the handle's own working buffers are left untouched.
+// Each call issues, on the caller's stream: one memset of the counters, one
+// small kernel that writes the per-layer pointer table into the region (from
+// the handle's device table and the region's layout, passed by value), and
+// the worker launch.  No host buffer is read by a copy.
+//
+// Batched handles pad the tensor-core operands to 8 or 16 sequence columns.
+// The region is not cleared between calls, so the padding columns hold what
+// an earlier call left there; they cannot reach the outputs: a column of an
+// MMA's result depends only on the same column of its operand, and only the
+// batch's columns are ever stored.
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
-#include <vector>
 
 #include "mk_handle.hpp"
 
@@ -35,16 +44,19 @@ void *g_scratch_ptr[kMaxDevices] = {};
 
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
+// Offsets in the region.  Per-layer buffers sit in equal blocks, so layer l's
+// buffer is its layer-0 offset plus l times the block size.
 struct Layout {
   size_t counters, arrivals, epoch, status, layers, lm_val, lm_idx, x, total;
-  std::vector<size_t> qkv, part, att, xm, h;
-  // batch >= 2: operands and sums of squares (index n_layers of xa / ssa: the
-  // final hidden state)
-  std::vector<size_t> xa, ssa, attb, xmb, ssm, hb;
+  // per layer: offsets within layer 0's block, block size
+  size_t qkv, part, att, xm, h, lstride;
+  // batch >= 2: operand and sum-of-squares blocks; xa / ssa have n_layers + 1
+  // entries (the last: the final hidden state, input of the LM head)
+  size_t xa, ssa, xstride, attb, xmb, ssm, hb, bstride;
 };
 
 Layout layout_of(const mk_model_config &c, const mk::TaskGraph &g) {
-  Layout L;
+  Layout L{};
   const int B = c.batch, H = c.hidden, F = c.ffn, Ly = c.n_layers, D = c.head_dim;
   const int rep = c.n_q_heads / c.n_kv_heads;
   const size_t n_qkv = (size_t)c.n_kv_heads * (rep + 2) * D, qd = (size_t)c.n_q_heads * D;
@@ -64,28 +76,86 @@ Layout layout_of(const mk_model_config &c, const mk::TaskGraph &g) {
   L.lm_val = take(4 * (size_t)B * n_lm);
   L.lm_idx = take(4 * (size_t)B * n_lm);
   L.x = take(4 * (size_t)(Ly + 1) * B * H);
-  for (int l = 0; l < Ly; ++l) {
-    L.qkv.push_back(take(4 * (size_t)B * n_qkv));
-    L.part.push_back(S > 1 ? take(4 * (size_t)B * c.n_q_heads * S * (D + 2)) : 0);
-    L.att.push_back(take(4 * (size_t)B * qd));
-    L.xm.push_back(take(4 * (size_t)B * H));
-    L.h.push_back(take(4 * (size_t)B * F));
+  // one block per layer: qkv, split partials, att, x_mid, h
+  {
+    size_t o = 0;
+    auto sub = [&](size_t bytes) {
+      size_t r = o;
+      o = up256(o + bytes);
+      return r;
+    };
+    L.qkv = sub(4 * (size_t)B * n_qkv);
+    L.part = S > 1 ? sub(4 * (size_t)B * c.n_q_heads * S * (D + 2)) : 0;
+    L.att = sub(4 * (size_t)B * qd);
+    L.xm = sub(4 * (size_t)B * H);
+    L.h = sub(4 * (size_t)B * F);
+    L.lstride = o;
+    const size_t base = take(o * Ly);
+    L.qkv += base; L.att += base; L.xm += base; L.h += base;
+    if (S > 1) L.part += base;
   }
   if (B > 1) {
     const int Bp = B > 8 ? 16 : 8, n_parts = H / 16;
-    for (int l = 0; l <= Ly; ++l) {
-      L.xa.push_back(take(4 * (size_t)Bp * H));
-      L.ssa.push_back(take(4 * (size_t)B * n_parts));
-    }
-    for (int l = 0; l < Ly; ++l) {
-      L.attb.push_back(take(4 * (size_t)Bp * qd));
-      L.xmb.push_back(take(4 * (size_t)Bp * H));
-      L.ssm.push_back(take(4 * (size_t)B * n_parts));
-      L.hb.push_back(take(4 * (size_t)Bp * F));
-    }
+    size_t o = 0;
+    auto sub = [&](size_t bytes) {
+      size_t r = o;
+      o = up256(o + bytes);
+      return r;
+    };
+    L.xa = sub(4 * (size_t)Bp * H);
+    L.ssa = sub(4 * (size_t)B * n_parts);
+    L.xstride = o;
+    size_t base = take(o * (Ly + 1));
+    L.xa += base; L.ssa += base;
+    o = 0;
+    L.attb = sub(4 * (size_t)Bp * qd);
+    L.xmb = sub(4 * (size_t)Bp * H);
+    L.ssm = sub(4 * (size_t)B * n_parts);
+    L.hb = sub(4 * (size_t)Bp * F);
+    L.bstride = o;
+    base = take(o * Ly);
+    L.attb += base; L.xmb += base; L.ssm += base; L.hb += base;
   }
   L.total = off;
   return L;
+}
+
+// By-value description of the region for the pointer-table kernel.
+struct StaticLayers {
+  char *base;
+  Layout lay;
+  int B, H, Ly, has_part, batched;
+};
+
+// Layer l's entry of the region's pointer table: the handle's entry (weights
+// and gains) with every activation pointer moved into the region.
+__global__ void static_layers_kernel(const mk::DevLayer *src, mk::DevLayer *dst, StaticLayers s) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l >= s.Ly) return;
+  const Layout &y = s.lay;
+  char *b = s.base;
+  mk::DevLayer d = src[l];
+  const size_t lo = (size_t)l * y.lstride;
+  float *x = reinterpret_cast<float *>(b + y.x);
+  d.qkv = reinterpret_cast<float *>(b + y.qkv + lo);
+  d.part = s.has_part ? reinterpret_cast<float *>(b + y.part + lo) : nullptr;
+  d.att = reinterpret_cast<float *>(b + y.att + lo);
+  d.xm = reinterpret_cast<float *>(b + y.xm + lo);
+  d.h = reinterpret_cast<float *>(b + y.h + lo);
+  d.x_in = x + (size_t)l * s.B * s.H;
+  d.x_out = x + (size_t)(l + 1) * s.B * s.H;
+  if (s.batched) {
+    const size_t xo = (size_t)l * y.xstride, bo = (size_t)l * y.bstride;
+    d.xa = reinterpret_cast<uint16_t *>(b + y.xa + xo);
+    d.ssa = reinterpret_cast<float *>(b + y.ssa + xo);
+    d.xa_next = reinterpret_cast<uint16_t *>(b + y.xa + xo + y.xstride);
+    d.ssa_next = reinterpret_cast<float *>(b + y.ssa + xo + y.xstride);
+    d.attb = reinterpret_cast<uint16_t *>(b + y.attb + bo);
+    d.xmb = reinterpret_cast<uint16_t *>(b + y.xmb + bo);
+    d.ssm = reinterpret_cast<float *>(b + y.ssm + bo);
+    d.hb = reinterpret_cast<uint16_t *>(b + y.hb + bo);
+  }
+  dst[l] = d;
 }
 
 // Device address of g_step_scratch on `device`, looked up once per device
@@ -159,39 +229,7 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
   const mk_model_config &c = h->cfg;
   const int B = c.batch, H = c.hidden, Ly = c.n_layers;
 
-  // per-layer pointer table: the handle's weights, the static activations
-  std::vector<mk::DevLayer> layers(h->layers);
   float *x = reinterpret_cast<float *>(base + L.x);
-  for (int l = 0; l < Ly; ++l) {
-    mk::DevLayer &d = layers[l];
-    d.qkv = reinterpret_cast<float *>(base + L.qkv[l]);
-    d.part = L.part[l] ? reinterpret_cast<float *>(base + L.part[l]) : nullptr;
-    d.att = reinterpret_cast<float *>(base + L.att[l]);
-    d.xm = reinterpret_cast<float *>(base + L.xm[l]);
-    d.h = reinterpret_cast<float *>(base + L.h[l]);
-    d.x_in = x + (size_t)l * B * H;
-    d.x_out = x + (size_t)(l + 1) * B * H;
-    if (B > 1) {
-      d.xa = reinterpret_cast<uint16_t *>(base + L.xa[l]);
-      d.ssa = reinterpret_cast<float *>(base + L.ssa[l]);
-      d.attb = reinterpret_cast<uint16_t *>(base + L.attb[l]);
-      d.xmb = reinterpret_cast<uint16_t *>(base + L.xmb[l]);
-      d.ssm = reinterpret_cast<float *>(base + L.ssm[l]);
-      d.hb = reinterpret_cast<uint16_t *>(base + L.hb[l]);
-      d.xa_next = reinterpret_cast<uint16_t *>(base + L.xa[l + 1]);
-      d.ssa_next = reinterpret_cast<float *>(base + L.ssa[l + 1]);
-    }
-  }
-  // The region keeps the previous call's contents: counters, arrival counters
-  // and the epoch must start at zero (activations are fully rewritten).
-  e = cudaMemsetAsync(base + L.counters, 0, L.status - L.counters, st);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(base + L.layers, layers.data(), sizeof(mk::DevLayer) * Ly,
-                        cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) {
-    h->err = std::string("static region set-up: ") + cudaGetErrorString(e);
-    return MK_ERR_CUDA;
-  }
   mk::Params p = h->base;
   p.counters = reinterpret_cast<uint32_t *>(base + L.counters);
   p.arrivals = reinterpret_cast<uint32_t *>(base + L.arrivals);
@@ -204,8 +242,8 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
   p.lm_val = reinterpret_cast<float *>(base + L.lm_val);
   p.lm_idx = reinterpret_cast<int32_t *>(base + L.lm_idx);
   if (B > 1) {
-    p.xfb = reinterpret_cast<uint16_t *>(base + L.xa[Ly]);
-    p.ssf = reinterpret_cast<float *>(base + L.ssa[Ly]);
+    p.xfb = reinterpret_cast<uint16_t *>(base + L.xa + (size_t)Ly * L.xstride);
+    p.ssf = reinterpret_cast<float *>(base + L.ssa + (size_t)Ly * L.xstride);
   }
   p.trace = nullptr;
   p.tokens_in = d_tokens_in;
@@ -217,6 +255,19 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
   if (!me.empty()) {
     h->err = me;
     return MK_ERR_ARG;
+  }
+  // The region keeps the previous call's contents: counters, arrival counters
+  // and the epoch must start at zero (activations are fully rewritten).
+  e = cudaMemsetAsync(base + L.counters, 0, L.status - L.counters, st);
+  if (e == cudaSuccess) {
+    StaticLayers sl{base, L, B, H, Ly, h->graph.tiling.attn_splits > 1, B > 1};
+    static_layers_kernel<<<(Ly + 63) / 64, 64, 0, st>>>(
+        h->d_layers, reinterpret_cast<mk::DevLayer *>(base + L.layers), sl);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) {
+    h->err = std::string("static region set-up: ") + cudaGetErrorString(e);
+    return MK_ERR_CUDA;
   }
   p.logits = d_logits;
   p.persistent = 1;

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 import synth
-from gpu_helpers import Case, compare_step, torch
+from gpu_helpers import Case, lockstep_oracle, torch
 
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("built_libs")]
 
@@ -49,21 +49,19 @@ def test_multistep_equals_single_steps_bitwise(w):
     np.testing.assert_array_equal(a[2], c.lens + n)
 
 
-def test_multistep_matches_oracle_stepwise():
-    # the oracle advances with the tokens the GPU chose; after n steps the
-    # last logits and the caches agree within the step tolerances
-    w = synth.TINY.with_(kv_len=20, steps=4)
+@pytest.mark.parametrize("w,bf16_inputs", [
+    (synth.TINY.with_(kv_len=20, steps=4), False),
+    (synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None, kv_len_range=(0, 300), steps=4), True)],
+    ids=["tiny", "tiny-batch5-split"])
+def test_multistep_matches_oracle_stepwise(w, bf16_inputs):
+    # the oracle replays the launch's steps fed with the tokens the GPU chose:
+    # every step's token and appended K/V rows, and the last step's logits and
+    # hidden state, agree within the step tolerances
     n = w.steps
     c = Case(w, seed=42)
     toks, logits, lens, gk, gv = _run_steps(c, n)
-    k, v, kl = c.k.copy(), c.v.copy(), c.lens.copy()
-    tok = c.tokens.copy()
-    for s in range(n):
-        ref = c.oracle_step(tokens=tok, k=k, v=v, lens=kl)
-        if s < n - 1:
-            tok = toks[s].copy()
-    got = {"tokens": toks[-1], "logits": logits, "hidden": c.gpu_hidden(), "kv_len": lens}
-    compare_step(ref, got, w, "multistep-last")
+    last = {"tokens": toks[-1], "logits": logits, "hidden": c.gpu_hidden(), "kv_len": lens}
+    lockstep_oracle(c, toks, last, gk.view(np.uint16), gv.view(np.uint16), bf16_inputs, "multistep")
     np.testing.assert_array_equal(lens, c.lens + n)
 
 

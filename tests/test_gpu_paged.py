@@ -4,13 +4,15 @@ The same seeded inputs run through a handle built for contiguous caches and
 one built with kv_page_size = P.  The pools hold the cache rows in pages
 scattered by a random permutation (with spare pages); results must be
 bitwise those of the contiguous run (the stage partition is the same in
-these cases, so is the arithmetic), and the appended rows must land in the
-right pages."""
+these cases, so is the arithmetic), the appended rows must land in the right
+pages, and the oracle, replaying the steps with the GPU's tokens, must agree
+with every step's token, every appended row and the last step's logits and
+hidden state."""
 import numpy as np
 import pytest
 
 import synth
-from gpu_helpers import Case, dev_u16, torch
+from gpu_helpers import Case, dev_u16, lockstep_oracle, torch
 
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("built_libs")]
 
@@ -42,7 +44,7 @@ def from_pool(pool, table, cap):
     return out[:, :, :, :cap, :]
 
 
-def run_pair(w, seed, n_steps):
+def run_pair(w, seed, n_steps, against_oracle=False):
     t = torch()
     ref = Case(w, seed=seed)
     out_r = t.zeros((n_steps, w.batch), dtype=t.int32, device="cuda")
@@ -67,6 +69,10 @@ def run_pair(w, seed, n_steps):
     vv = from_pool(d_vp.cpu().numpy().view(np.uint16), table, cap)
     np.testing.assert_array_equal(kk, ref.d_k.cpu().numpy().view(np.uint16))
     np.testing.assert_array_equal(vv, ref.d_v.cpu().numpy().view(np.uint16))
+    if against_oracle:
+        last = {"tokens": out_p.cpu().numpy()[-1], "logits": pg.d_logits.cpu().numpy(),
+                "hidden": pg.gpu_hidden(), "kv_len": pg.d_len.cpu().numpy()}
+        lockstep_oracle(pg, out_p.cpu().numpy(), last, kk, vv, w.batch > 1, "paged")
     return pg, d_kp, d_vp, d_table, n_pages
 
 
@@ -75,8 +81,8 @@ def run_pair(w, seed, n_steps):
                                                    kv_len_range=(0, 300), steps=3), 3),
                                  (synth.Q06B.with_(steps=3), 3)],
                          ids=["tiny", "tiny-batch3-split", "qwen3-0.6b"])
-def test_paged_equals_contiguous_bitwise(w, n):
-    run_pair(w, 61, n)
+def test_paged_equals_contiguous_bitwise_and_matches_oracle(w, n):
+    run_pair(w, 61, n, against_oracle=True)
 
 
 def test_paged_rejects_bad_tables_and_wrong_entry_points():
