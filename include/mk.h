@@ -92,7 +92,6 @@ typedef struct {
                                 batch >= 2 needs a multiple of 16) */
   int attn_tasks_per_worker; /* at most this many attention tasks per worker (1) */
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
-  int use_mma;               /* ignored: batch >= 2 always runs on tensor cores */
   int ring_stages;           /* shared-memory weight ring depth (4) */
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while a
@@ -108,6 +107,19 @@ typedef struct {
                                 evict-first (default: they are read once per step and
                                 must not displace code, activations and counters),
                                 -1 = the normal policy */
+  int attn_jit;              /* attention tasks resolved at run time (MPK review, "Direction 4":
+                                data-dependent operators JIT, the rest ahead of time):
+                                attn_tasks_per_worker * W tasks per layer cut the live
+                                positions of all (sequence, kv head) pairs into equal
+                                chunks, which may cross pairs.  0 = default (on for batch
+                                >= 2), 1 = on (batch >= 2 only), -1 = off: splits fixed
+                                at build time from kv_capacity */
+  int dispatch;              /* 0 = static queues: worker w runs tasks w, w + W, ... and waits
+                                on their events itself (default); 1 = a scheduler CTA in the
+                                same launch hands ready tasks to the workers (the pages'
+                                dispatch design, kept as an ablation): W = SMs - 1 workers
+                                unless num_workers is set, one step per launch
+                                (mk_decode_step only) */
 } mk_tuning;
 
 /* Weights: device pointers, bf16, row-major [out][in].  Per-layer arrays are
@@ -140,8 +152,10 @@ typedef struct {
   /* tiling chosen for the decode graph (0 for generic graphs) */
   int32_t qkv_rows, o_rows, gu_rows, down_rows, lm_rows, attn_splits, attn_chunk;
   /* batch >= 2: tensor-core tiles of QKV, O, GATE_UP, DOWN, LM_HEAD (in that
-   * order): 16-row m-tiles per row block and 16-column k-blocks per ring
-   * stage for the handle's ring stage size (0 at batch 1) */
+   * order): 16-row m-tiles of a full pass (a task's rows run in passes of at
+   * most 256, one TMEM accumulator each) and 16-column k-blocks per ring stage
+   * of such a pass, for the handle's ring stage size (0 at batch 1, and a
+   * kcb of 0 when a stage cannot hold one k-block: mk_build_graph rejects it) */
   int32_t mma_mb[5], mma_kcb[5];
 } mk_graph_view;
 
@@ -179,9 +193,11 @@ mk_status mk_graph_from_edges(int n_tasks, const int32_t *task_op, const int32_t
  * tuning->num_workers is set), upload the task/event tables, and allocate the
  * event counters, the step epoch, the status word and the activation buffers
  * (all owned by the handle).  batch 1 runs the CUDA-core worker kernel;
- * batch 2..16 the tensor-core one (projections on mma.sync with the batch as
- * the N dimension, attention on mma.sync over TMA K/V tiles), which needs
- * col_align to be a multiple of 16.  Errors: MK_ERR_ARG, MK_ERR_CUDA,
+ * batch 2..16 the tensor-core one (projections on tcgen05.mma: the hi/lo
+ * activation operand as the 128-row A matrix, the task's weight rows as N,
+ * fp32 accumulators in tensor memory; attention on mma.sync over TMA K/V
+ * tiles), which needs col_align to be a multiple of 16.  Errors: MK_ERR_ARG
+ * (also for a ring stage too small for one tensor-core k-block), MK_ERR_CUDA,
  * MK_ERR_OOM.
  */
 mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, int device,
@@ -192,9 +208,10 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
  * out in task-stream order: QKV rows group-major (per kv head: its q heads,
  * then k, then v), gate and up rows interleaved, every task's weight tile one
  * contiguous range.  For batch >= 2 handles the projection matrices are then
- * permuted on the device into mma.sync A-fragment order (512-byte blocks per
- * 16-row x 16-column tile) and the LM head is padded to whole 16-row tiles
- * (a separate copy even when tied); this uses a temporary device staging
+ * permuted on the device into the tcgen05 operand order of their tasks (per
+ * pass of at most 256 task rows, per 16-column k-block, 8-row x 16-byte core
+ * matrices) and the LM head is padded to whole 16-row tiles (a separate copy
+ * even when tied); this uses a temporary device staging
  * buffer of the largest layer matrix and synchronises `stream`.  Copies are
  * ordered on `stream`; the caller may free its tensors once the stream has
  * passed this call.  May be called again to replace the weights.  Errors:
@@ -303,7 +320,9 @@ mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_tokens_in, int32
 
 /* mk_sync_status - synchronize `stream`, then return the device status word
  * (MK_OK, MK_ERR_TIMEOUT or MK_ERR_DEVICE).  detail (nullable, 4 ints):
- * {status, task id, event id, block}.  The word stays set until mk_reset. */
+ * {status, task id, event id, block}; an event id of -2 after a failure means
+ * that a worker exited with copies into its shared memory still outstanding
+ * after its bounded wait for them.  The word stays set until mk_reset. */
 mk_status mk_sync_status(mk_handle *h, void *stream, int32_t *detail);
 
 /* mk_reset - stream-ordered: zero the event counters, the step epoch and the

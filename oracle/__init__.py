@@ -84,7 +84,8 @@ def _load():
                                           ctypes.c_int]
     lib.oracle_decode_step_ex.restype = ctypes.c_int
     lib.oracle_tgraph_decode.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_int, ctypes.c_int, ctypes.POINTER(vp)]
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(vp)]
     lib.oracle_tgraph_decode.restype = ctypes.c_int
     lib.oracle_tgraph_from_edges.argtypes = [ctypes.c_int, vp, vp, ctypes.c_int, vp, vp,
                                              ctypes.POINTER(vp)]
@@ -250,11 +251,13 @@ class TGraph:
 
 
 def tgraph_decode(workload, kv_capacity: int, num_workers: int, col_align: int = 16,
-                  attn_tasks_per_worker: int = 4, attn_min_chunk: int = 64) -> TGraph:
+                  attn_tasks_per_worker: int = 4, attn_min_chunk: int = 64,
+                  attn_jit: int = 0) -> TGraph:
     cfg = make_cfg(workload, kv_capacity)
     h = ctypes.c_void_p()
     rc = _load().oracle_tgraph_decode(ctypes.byref(cfg), num_workers, col_align,
-                                      attn_tasks_per_worker, attn_min_chunk, ctypes.byref(h))
+                                      attn_tasks_per_worker, attn_min_chunk, int(attn_jit),
+                                      ctypes.byref(h))
     if rc != 0:
         raise ValueError(f"oracle_tgraph_decode failed ({rc})")
     return TGraph(h)

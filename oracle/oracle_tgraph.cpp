@@ -23,6 +23,11 @@
 //               S = ceil(Lcap / chunk).  Every split writes its partial
 //               and may write the merged head block: the split of (b, g) that
 //               finishes last merges the partials (no separate merge op).
+//               JIT attention (data-dependent ranges resolved at run time,
+//               MPK review "Direction 4"): apw * W tasks per layer, each
+//               reading all of the layer's q/k/v and the KV lengths and
+//               writing all partials and heads; partial slots per (b, g):
+//               S = ceil(apw * W / (B * Hkv)) + 2; chunk = 0.
 //   regions     each task reads and writes rectangles of named buffers;
 //               activations are single-assignment (one buffer per layer/op).
 //   raw events  task a -> task c when op(a) < op(c) and a region of a and a
@@ -395,7 +400,7 @@ struct Lowered {
   int qkv_rows, o_rows, gu_rows, down_rows, lm_rows, splits, chunk;
 };
 
-Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_chunk) {
+Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_chunk, int jit) {
   Lowered L;
   const int Ly = c.n_layers, H = c.hidden, Hq = c.n_q_heads, Hkv = c.n_kv_heads, D = c.head_dim;
   const int F = c.ffn, V = c.vocab, B = c.batch, Lcap = c.kv_capacity, rep = Hq / Hkv;
@@ -408,9 +413,16 @@ Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_
       break;
     }
   }
-  int sp = (int)std::max(1L, (long)apw * W / ((long)B * Hkv));
-  int chunk = std::max(min_chunk, align_up(ceil_div(Lcap, sp), 64));
-  int S = ceil_div(Lcap, chunk);
+  int S, chunk, n_jit = 0;
+  if (jit) {
+    n_jit = std::max(1, apw * W);
+    S = ceil_div(n_jit, (long)B * Hkv) + 2;
+    chunk = 0;
+  } else {
+    int sp = (int)std::max(1L, (long)apw * W / ((long)B * Hkv));
+    chunk = std::max(min_chunk, align_up(ceil_div(Lcap, sp), 64));
+    S = ceil_div(Lcap, chunk);
+  }
   L.qkv_rows = qkv_rows;
   L.o_rows = gemv_rows(H);
   L.gu_rows = gemv_rows(F);
@@ -450,7 +462,10 @@ Lowered lower_decode(const OracleCfg &c, int W, int col_align, int apw, int min_
       add(T_QKV, l, j, {R(B_X(l), 0, B, 0, H),
                         Wr(B_QKV(l), 0, B, j * qkv_rows, std::min(Nqkv, (j + 1) * qkv_rows))});
     ++op;
-    for (int b = 0; b < B; ++b)
+    for (int a = 0; a < n_jit; ++a)
+      add(T_ATTN, l, a, {R(B_QKV(l), 0, B, 0, Nqkv), R(B_KVLEN, 0, B, 0, 1),
+                         Wr(B_PART(l), 0, B, 0, Hkv * S), Wr(B_ATT(l), 0, B, 0, qd)});
+    for (int b = 0; b < (jit ? 0 : B); ++b)
       for (int g = 0; g < Hkv; ++g)
         for (int s = 0; s < S; ++s) {
           std::vector<Rect> regs = {R(B_QKV(l), b, b + 1, g * G, (g + 1) * G),
@@ -511,12 +526,13 @@ std::vector<std::set<int>> region_preds(const std::vector<Task> &tasks) {
 extern "C" {
 
 int oracle_tgraph_decode(const OracleCfg *cfg, int num_workers, int col_align,
-                         int attn_tasks_per_worker, int attn_min_chunk, void **out) {
+                         int attn_tasks_per_worker, int attn_min_chunk, int attn_jit, void **out) {
   if (!cfg || !out || num_workers < 1 || col_align < 1 || attn_tasks_per_worker < 1 ||
       attn_min_chunk < 1)
     return -1;
   if (cfg->n_kv_heads < 1 || cfg->n_q_heads % cfg->n_kv_heads) return -1;
-  Lowered L = lower_decode(*cfg, num_workers, col_align, attn_tasks_per_worker, attn_min_chunk);
+  Lowered L = lower_decode(*cfg, num_workers, col_align, attn_tasks_per_worker, attn_min_chunk,
+                           attn_jit);
   auto preds = region_preds(L.tasks);
   Graph *g = new Graph(run_pipeline(L.tasks, preds));
   if (g->t_type.empty()) {

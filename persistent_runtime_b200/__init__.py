@@ -47,10 +47,11 @@ class ModelConfig(ctypes.Structure):
 class Tuning(ctypes.Structure):
     _fields_ = [("num_workers", ctypes.c_int), ("col_align", ctypes.c_int),
                 ("attn_tasks_per_worker", ctypes.c_int), ("attn_min_chunk", ctypes.c_int),
-                ("use_mma", ctypes.c_int), ("ring_stages", ctypes.c_int),
+                ("ring_stages", ctypes.c_int),
                 ("ring_stage_bytes", ctypes.c_int), ("l2_prefetch_bytes", ctypes.c_int),
                 ("wait_timeout_us", ctypes.c_uint), ("kv_page_size", ctypes.c_int),
-                ("l2_stream_policy", ctypes.c_int)]
+                ("l2_stream_policy", ctypes.c_int), ("attn_jit", ctypes.c_int),
+                ("dispatch", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)

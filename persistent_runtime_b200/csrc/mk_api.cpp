@@ -85,22 +85,29 @@ std::string check_gpu_shape(const mk_model_config &c) {
 }
 
 // Tensor-core tiling of the batched projections (QKV, O, GATE_UP, DOWN,
-// LM_HEAD, in that order).  m-tiles per row block: the task's rows up to the
-// accumulator limit; k-blocks per ring stage: what a stage holds for that
-// many m-tiles, a multiple of 8 (one share per warp), at most
-// mma_max_kpw(nn) per warp (the B-fragment registers of one stage).
+// LM_HEAD, in that order), as the worker derives it: a task's rows run in
+// passes of up to kUmmaMaxN rows (mb = 16-row m-tiles of a full pass), and a
+// pass streams ring stages of kcb 16-column k-blocks, as many as the stage's
+// weights (N * 32 bytes per k-block), its operand chunk (512 nn bytes per
+// k-block) and kUmmaSlack fit in one ring stage (at most the K / 16 k-blocks
+// of the operator; 0 when not even one fits).
 struct MmaTiling {
   int mb[5], kcb[5];
 };
 
-MmaTiling mma_tiling(const mk::Tiling &T, int ring_stage_bytes, int nn) {
-  const int units = ring_stage_bytes / 512;
-  auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
+int umma_nkb(int ring_stage_bytes, int N, int nn, int KB) {
+  const int n = (ring_stage_bytes - mk::kUmmaSlack) / (N * 32 + 512 * nn);
+  return std::min(KB, std::max(n, 0));
+}
+
+MmaTiling mma_tiling(const mk::Tiling &T, const mk_model_config &c, int ring_stage_bytes, int nn) {
   const int rows[5] = {T.qkv_rows, T.o_rows, 2 * T.gu_rows, T.down_rows, T.lm_rows};
+  const int K[5] = {c.hidden, c.n_q_heads * c.head_dim, c.hidden, c.ffn, c.hidden};
   MmaTiling m{};
   for (int i = 0; i < 5; ++i) {
-    m.mb[i] = mb_of(rows[i]);
-    m.kcb[i] = std::min(8 * mk::mma_max_kpw(nn), units / m.mb[i] / 8 * 8);
+    const int N = std::min(mk::kUmmaMaxN, (rows[i] + 15) / 16 * 16);
+    m.mb[i] = N / 16;
+    m.kcb[i] = umma_nkb(ring_stage_bytes, N, nn, K[i] / 16);
   }
   return m;
 }
@@ -110,12 +117,19 @@ mk::ModelShape shape_of(const mk_model_config &c) {
                         c.ffn,      c.vocab,  c.batch,     c.kv_capacity};
 }
 
+// JIT attention: on by default from batch 2 (the batch-1 kernel's attention
+// keeps its splits fixed at build time, see mk_build_graph).
+bool jit_attention(const mk_model_config &c, const mk_tuning &t) {
+  return t.attn_jit == 0 ? c.batch > 1 : t.attn_jit > 0;
+}
+
 mk_status plan(const mk_model_config *cfg, const mk_tuning &t, int workers, mk_handle *h) {
   mk::GraphTuning gt;
   gt.num_workers = workers;
   gt.col_align = t.col_align;
   gt.attn_tasks_per_worker = t.attn_tasks_per_worker;
   gt.attn_min_chunk = t.attn_min_chunk;
+  gt.attn_jit = jit_attention(*cfg, t) ? 1 : 0;
   int st = 0;
   std::string e = mk::plan_decode_graph(shape_of(*cfg), gt, &h->graph, &st);
   if (!e.empty()) return fail(h, st == -4 ? MK_ERR_GRAPH : MK_ERR_ARG, e);
@@ -208,6 +222,10 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     delete h;
     return fail(nullptr, MK_ERR_ARG, "batch > 1 needs col_align to be a multiple of 16");
   }
+  if (c.batch == 1 && t.attn_jit > 0) {
+    delete h;
+    return fail(nullptr, MK_ERR_ARG, "JIT attention needs batch >= 2");
+  }
   if (t.kv_page_size < 0 || t.kv_page_size % 64) {
     delete h;
     return fail(nullptr, MK_ERR_ARG, "kv_page_size must be 0 or a multiple of 64");
@@ -241,8 +259,9 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     delete h;
     return fail(nullptr, MK_ERR_CUDA, "worker kernel cannot be resident");
   }
-  const int W = t.num_workers > 0 ? t.num_workers : sms;
-  if (W > sms * per_sm) {
+  // dispatch mode: one CTA of the launch is the scheduler
+  const int W = t.num_workers > 0 ? t.num_workers : (t.dispatch > 0 ? sms - 1 : sms);
+  if (W < 1 || W + (t.dispatch > 0 ? 1 : 0) > sms * per_sm) {
     delete h;
     return fail(nullptr, MK_ERR_ARG, "more workers than co-resident CTAs");
   }
@@ -274,6 +293,11 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   const size_t o_status = take(16);
   const size_t o_layers = take(sizeof(mk::DevLayer) * Ly);
   const size_t o_optasks = take(4 * G.type.size());
+  // dispatch mode: per-worker queues (round-robin dealing gives each worker
+  // at most ceil(n_tasks / W) tasks, plus the end mark)
+  const int q_cap = (int)((G.type.size() + W - 1) / W) + 2;
+  const size_t o_qlist = t.dispatch > 0 ? take(4 * (size_t)W * q_cap) : 0;
+  const size_t o_qtail = t.dispatch > 0 ? take(4 * (size_t)W) : 0;
   const size_t o_rope = take(4 * (size_t)c.kv_capacity * D);
   const size_t o_lmv = take(4 * (size_t)B * T.n_lm);
   const size_t o_lmi = take(4 * (size_t)B * T.n_lm);
@@ -393,6 +417,14 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.epoch = reinterpret_cast<uint32_t *>(base + o_epoch);
   p.status = reinterpret_cast<int32_t *>(base + o_status);
   p.n_tasks = (int)tasks.size();
+  p.n_events = (int)events.size();
+  if (t.dispatch > 0) {
+    p.dispatch = 1;
+    p.n_workers = W;
+    p.q_cap = q_cap;
+    p.q_list = reinterpret_cast<int32_t *>(base + o_qlist);
+    p.q_tail = reinterpret_cast<uint32_t *>(base + o_qtail);
+  }
   p.layers = h->d_layers;
   p.x0 = reinterpret_cast<float *>(base + o_x);
   p.x_final = reinterpret_cast<float *>(base + o_x) + (size_t)Ly * B * H;
@@ -421,13 +453,17 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   p.rps_down = rps(F);
   p.rps_lm = rps(H);
   // KV positions per stage: K and V of pps rows each, a multiple of 8 (whole
-  // 1024-byte swizzle atoms), at most 256 (the TMA box height limit) and at
-  // most one split (a multiple of 64), so a short split is one exact box
-  p.pps = std::min(std::min(256, T.attn_chunk), t.ring_stage_bytes / (4 * D) / 8 * 8);
+  // 1024-byte swizzle atoms), at most 256 (the TMA box height limit) and, with
+  // splits fixed at build time, at most one split (a multiple of 64), so a
+  // short split is one exact box
+  p.jit = jit_attention(c, t) ? 1 : 0;
+  p.n_attn = T.n_attn;
+  p.pps = std::min(p.jit ? 256 : std::min(256, T.attn_chunk), t.ring_stage_bytes / (4 * D) / 8 * 8);
   if (t.kv_page_size > 0) {
     // paged pools: a stage must stay inside one page; splits start at
-    // multiples of 64 and pages hold multiples of 64 rows, so a stage of a
-    // divisor of 64 rows never crosses a page
+    // multiples of 64 (JIT pieces: stages start at multiples of pps within a
+    // pair) and pages hold multiples of 64 rows, so a stage of a divisor of
+    // 64 rows never crosses a page
     int q = 64;
     while (q > p.pps) q >>= 1;
     p.pps = q;
@@ -439,23 +475,13 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     return fail(nullptr, MK_ERR_ARG, "ring stage smaller than 8 K/V rows");
   }
   if (mma) {
-    const MmaTiling mt = mma_tiling(T, t.ring_stage_bytes, nn);
+    const MmaTiling mt = mma_tiling(T, c, t.ring_stage_bytes, nn);
     p.mma = 1;
     p.nn = nn;
     p.n_parts = n_parts;
-    p.mb_qkv = mt.mb[0];
-    p.mb_o = mt.mb[1];
-    p.mb_gu = mt.mb[2];
-    p.mb_down = mt.mb[3];
-    p.mb_lm = mt.mb[4];
-    p.kcb_qkv = mt.kcb[0];
-    p.kcb_o = mt.kcb[1];
-    p.kcb_gu = mt.kcb[2];
-    p.kcb_down = mt.kcb[3];
-    p.kcb_lm = mt.kcb[4];
     p.xfb = reinterpret_cast<uint16_t *>(base + o_xa[Ly]);
     p.ssf = reinterpret_cast<float *>(base + o_ssa[Ly]);
-    if (std::min({p.kcb_qkv, p.kcb_o, p.kcb_gu, p.kcb_down, p.kcb_lm}) < 8) {
+    if (std::min({mt.kcb[0], mt.kcb[1], mt.kcb[2], mt.kcb[3], mt.kcb[4]}) < 1) {
       mk_destroy(h);
       return fail(nullptr, MK_ERR_ARG, "ring stage too small for the tensor-core tiles");
     }
@@ -501,9 +527,9 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     o_gu[l] = take((size_t)2 * F * H);
     o_dn[l] = take((size_t)H * F);
   }
-  // batch >= 2: projection matrices in mma.sync fragment order, the LM head
-  // padded to whole 16-row m-tiles and kept apart from the (row-major)
-  // embedding table even when the two are tied
+  // batch >= 2: projection matrices in the tensor-core order of their tasks,
+  // the LM head padded to whole 16-row m-tiles and kept apart from the
+  // (row-major) embedding table even when the two are tied
   const bool mma = h->base.mma != 0;
   const size_t Vp = mma ? ((size_t)V + 15) / 16 * 16 : (size_t)V;
   const bool lm_shares_embed = c.tied_embeddings && !mma;
@@ -561,32 +587,35 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     if (!c.tied_embeddings) cp(o_lm, w->lm_head, (size_t)V * H * 2);
   } else {
     // each matrix goes row-major into a staging buffer, then a kernel writes
-    // it to the arena in fragment order; the LM head goes in row slabs
+    // it to the arena in the tensor-core order of its tasks; the LM head goes
+    // in row slabs of whole tasks
+    const mk::Tiling &Tl = h->graph.tiling;
     const size_t tmp_bytes =
         2 * std::max({n_qkv * H, (size_t)H * qd, (size_t)2 * F * H, (size_t)H * F});
     void *tmp = nullptr;
     if (cudaMalloc(&tmp, tmp_bytes) != cudaSuccess)
       return fail(h, MK_ERR_OOM, "cudaMalloc of the weight staging buffer failed");
     char *T = static_cast<char *>(tmp);
-    auto frag = [&](size_t dst_off, int rows, int K) {
-      if (e == cudaSuccess) e = mk::permute_to_fragments(A + dst_off, T, rows, K, st);
+    auto perm = [&](size_t dst_off, int row_base, int n, int rows, int rows_p, int K, int task_rows) {
+      if (e == cudaSuccess)
+        e = mk::permute_to_umma(A + dst_off, T, row_base, n, rows, rows_p, K, task_rows, st);
     };
     for (int l = 0; l < Ly; ++l) {
       put_qkv(T, l);
-      frag(o_qkv[l], (int)n_qkv, H);
+      perm(o_qkv[l], 0, (int)n_qkv, (int)n_qkv, (int)n_qkv, H, Tl.qkv_rows);
       cpy(T, w->wo[l], (size_t)H * qd * 2);
-      frag(o_o[l], H, (int)qd);
+      perm(o_o[l], 0, H, H, H, (int)qd, Tl.o_rows);
       put_gu(T, l);
-      frag(o_gu[l], 2 * F, H);
+      perm(o_gu[l], 0, 2 * F, 2 * F, 2 * F, H, 2 * Tl.gu_rows);
       cpy(T, w->w_down[l], (size_t)H * F * 2);
-      frag(o_dn[l], H, F);
+      perm(o_dn[l], 0, H, H, H, F, Tl.down_rows);
     }
-    const int slab = (int)std::min<size_t>((size_t)V, tmp_bytes / row / 16 * 16);
+    const int slab =
+        std::max(1, (int)std::min<size_t>((size_t)V, tmp_bytes / row) / Tl.lm_rows) * Tl.lm_rows;
     for (int r0 = 0; r0 < V; r0 += slab) {
       const int n = std::min(slab, V - r0);
       cpy(T, static_cast<const char *>(lm_src) + (size_t)r0 * row, (size_t)n * row);
-      // m-tile r0 / 16 of the padded head: 512-byte blocks, H / 16 per m-tile
-      frag(o_lm + (size_t)(r0 / 16) * (H / 16) * 512, n, H);
+      perm(o_lm, r0, n, V, (int)Vp, H, Tl.lm_rows);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // the staging buffer is freed next
     cudaFree(tmp);
@@ -715,7 +744,12 @@ mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_to
   if (s != MK_OK) return s;
   p.logits = d_logits;
   p.persistent = 1;
-  cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
+  if (p.dispatch) {  // the scheduler publishes the queues from zero
+    cudaError_t e = cudaMemsetAsync(p.q_tail, 0, 4 * (size_t)p.n_workers,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(h, e, "queue reset");
+  }
+  cudaError_t e = mk::launch_persistent(p, h->tune.num_workers + p.dispatch, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
   return MK_OK;
@@ -734,6 +768,11 @@ mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
                           int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
                           void *d_v_cache, float *d_logits, void *stream) {
   if (n_steps < 1) return fail(h, MK_ERR_ARG, "n_steps must be >= 1");
+  if (h && h->base.dispatch) {
+    if (n_steps > 1) return fail(h, MK_ERR_ARG, "dispatch mode runs one step per launch");
+    return mk_decode_step(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache,
+                          d_logits, stream);
+  }
   Params p;
   mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_cache, d_v_cache, &p);
   if (s != MK_OK) return s;
@@ -753,6 +792,7 @@ mk_status mk_decode_steps_paged(mk_handle *h, int n_steps, const int32_t *d_toke
                                 float *d_logits, void *stream) {
   if (n_steps < 1) return fail(h, MK_ERR_ARG, "n_steps must be >= 1");
   if (!d_page_table) return fail(h, MK_ERR_ARG, "null page table");
+  if (h && h->base.dispatch) return fail(h, MK_ERR_ARG, "dispatch mode: use mk_decode_step");
   Params p;
   mk_status s = step_args(h, d_tokens_in, d_tokens_out, d_kv_len, d_k_pool, d_v_pool, &p,
                           n_pages, d_page_table);
@@ -775,6 +815,7 @@ mk_status mk_decode_step_perop(mk_handle *h, const int32_t *d_tokens_in, int32_t
   if (s != MK_OK) return s;
   p.logits = d_logits;
   p.persistent = 0;
+  p.dispatch = 0;
   for (int o = 0; o + 1 < (int)h->op_offset.size(); ++o) {
     const int n = h->op_offset[o + 1] - h->op_offset[o];
     if (n == 0) continue;
@@ -850,7 +891,7 @@ mk_status mk_graph_export(const mk_handle *h, mk_graph_view *out) {
   out->attn_splits = T.attn_splits;
   out->attn_chunk = T.attn_chunk;
   if (h->cfg.batch > 1 && T.qkv_rows > 0) {
-    const MmaTiling mt = mma_tiling(T, h->tune.ring_stage_bytes, (h->cfg.batch + 7) / 8);
+    const MmaTiling mt = mma_tiling(T, h->cfg, h->tune.ring_stage_bytes, (h->cfg.batch + 7) / 8);
     for (int i = 0; i < 5; ++i) {
       out->mma_mb[i] = mt.mb[i];
       out->mma_kcb[i] = mt.kcb[i];

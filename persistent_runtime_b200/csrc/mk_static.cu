@@ -194,6 +194,10 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle *h, const int32_t *d_token
     h->err = "the handle was built for paged K/V: use mk_decode_steps_paged";
     return MK_ERR_ARG;
   }
+  if (h->base.dispatch) {
+    h->err = "the handle was built for dispatch mode: use mk_decode_step";
+    return MK_ERR_ARG;
+  }
   const Layout L = layout_of(h->cfg, h->graph);
   if (L.total > kStaticScratchBytes) {
     h->err = "step working memory of " + std::to_string(L.total) +

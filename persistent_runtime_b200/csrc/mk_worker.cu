@@ -216,14 +216,12 @@ __device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// Tensor cores (batch >= 2): mma.sync.m16n8k16, A = weights (16 rows x 16 k,
-// row major), B = activations (16 k x 8 sequences), fp32 accumulators.
-// Fragment ownership (PTX ISA, "Matrix Fragments for mma.m16n8k16"), lane l,
-// g = l / 4, t = l % 4:  A regs {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..),
-// (g+8, 2t+8..)};  B regs {(2t..2t+1, g), (2t+8..2t+9, g)};  C {(g, 2t),
-// (g, 2t+1), (g+8, 2t), (g+8, 2t+1)}.  Weights and activations are stored in
-// exactly this order, so each lane fetches its fragment with one 16-byte
-// (A) or 8-byte (B) load.
+// Warp-level tensor cores (batched attention): mma.sync.m16n8k16, A 16 x 16
+// row major, B 16 x 8, fp32 accumulators.  Fragment ownership (PTX ISA,
+// "Matrix Fragments for mma.m16n8k16"), lane l, g = l / 4, t = l % 4:  A regs
+// {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..), (g+8, 2t+8..)};  B regs
+// {(2t..2t+1, g), (2t+8..2t+9, g)};  C {(g, 2t), (g, 2t+1), (g+8, 2t),
+// (g+8, 2t+1)}.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, const uint2 &b) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
@@ -256,27 +254,95 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
+// ---------------------------------------------------------------------------
+// 5th-generation tensor cores (batched projections): tcgen05.mma kind::f16,
+// one thread issues, fp32 accumulators live in tensor memory (TMEM).  Both
+// operands are K-major in shared memory without swizzle: core matrices of 8
+// rows x 8 bf16 (16 bytes per row, 128 bytes each); within one 16-column
+// k-block the two 8-column halves of a row group are 128 bytes apart and the
+// 8-row groups 256 bytes apart.  Element (row, k) of a k-block therefore sits
+// at (row / 8) * 256 + (k / 8) * 128 + (row % 8) * 16 + (k % 8) * 2.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;  // stride between the two k halves
+  d |= (uint64_t)(256u >> 4) << 32;  // stride between 8-row groups
+  d |= 1ull << 46;                   // descriptor version of sm_100
+  return d;                          // base offset 0, no swizzle
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N rows.
+__device__ __forceinline__ uint32_t umma_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The mbarrier receives one arrival once every earlier tcgen05 operation of
+// this thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+// Lanes 32 (warp % 4) .. + 31 of TMEM, 32 columns from taddr: thread t of the
+// warp receives lane base + t.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_n(uint64_t *bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n)
+               : "memory");
+}
+
 // Activation operands are two-term bf16 expansions x = hi + lo, hi = bf16(x),
-// lo = bf16(x - hi): about 16 significant bits, so W x = W hi + W lo (two MMAs
-// into one fp32 accumulator) keeps the projection inputs close to fp32 while
-// the weights stay exactly bf16.  A single bf16 rounding of every input would
-// cost ~0.4 % of the residual stream per layer.
+// lo = bf16(x - hi): about 16 significant bits, so W x = W hi + W lo (two
+// operand rows, summed in the epilogue) keeps the projection inputs close to
+// fp32 while the weights stay exactly bf16.  A single bf16 rounding of every
+// input would cost ~0.4 % of the residual stream per layer.
 //
-// Element (k, sequence b) of an operand with nn 8-column tiles, in bf16
-// units: 512-byte blocks per (16-row k-block, column tile), 16 bytes per lane
-// inside a block: {hi b0, hi b1, lo b0, lo b1} of the lane's B fragment.
-// Returns the position of hi; lo is 4 elements further.
+// The operand is the A matrix of the projections: row a = hi(b) for a = b and
+// lo(b) for a = 8 nn + b (nn 8-sequence tiles, padded sequences stay 0), K
+// major, one 512 nn-byte block per 16-column k-block in the core-matrix order
+// above.  Element (k, sequence b) of hi, in bf16 units; lo is 8 nn rows
+// (nn * 128 elements) further.
 __device__ __forceinline__ size_t opnd_off(int k, int b, int nn) {
   const int kk = k & 15;
-  return ((size_t)(k >> 4) * nn + (b >> 3)) * 256 + ((b & 7) * 4 + ((kk & 7) >> 1)) * 8 +
-         (kk >> 3) * 2 + (kk & 1);
+  return (size_t)(k >> 4) * (256 * nn) + (b >> 3) * 128 + (kk >> 3) * 64 + (b & 7) * 8 + (kk & 7);
 }
 
 __device__ __forceinline__ void put_opnd(uint16_t *buf, int k, int b, int nn, float x) {
   const size_t o = opnd_off(k, b, nn);
   const uint16_t hi = f2bf(x);
   buf[o] = hi;
-  buf[o + 4] = f2bf(x - bf2f(hi));
+  buf[o + (size_t)nn * 128] = f2bf(x - bf2f(hi));
 }
 
 // ---------------------------------------------------------------------------
@@ -287,6 +353,9 @@ enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kLogit
 struct Smem {
   uint8_t *ring;
   uint64_t *full, *empty;
+  uint64_t *abar;   // [stages] tensor-core projections: the stage's operand chunk landed
+  uint64_t *mdone;  // the MMAs of a pass completed
+  uint32_t *tmem;   // TMEM base address of the CTA's accumulators
   volatile int *ctl;
   unsigned long long *tmark;  // [8] trace marks: prologue done, streaming done, ready,
                               // L2 prefetch bytes, first ring stage available
@@ -302,7 +371,7 @@ struct Smem {
   float *mls;   // [3][kMaxRep]
   float *ored;  // per warp and head: [D] output, running max, running sum (merge: weights)
   // tensor-core projection scratch
-  float *cred;  // [warp][m-tile of the pass][16 rows][8 nn + 1] accumulator partials
+  float *cred;  // [32 columns][33]: one chunk of the accumulators read back from TMEM
   float *minv;  // [kMaxBatch] 1 / rms of each sequence's input
   float *mlv;   // [16] partial argmax values (LM head)
   int *mli;     // [16] partial argmax indices
@@ -311,7 +380,7 @@ struct Smem {
 __host__ __device__ inline size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct SmemOffsets {
-  size_t full, empty, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, cred, minv,
+  size_t full, empty, abar, mdone, tmem, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, cred, minv,
       mlv, mli, total;
 };
 
@@ -323,6 +392,12 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   p += 8 * (size_t)stages;
   o.empty = p;
   p += 8 * (size_t)stages;
+  o.abar = p;
+  p += 8 * (size_t)stages;
+  o.mdone = p;
+  p += 8;
+  o.tmem = p;
+  p += 8;
   o.ctl = p;
   p += 4 * kCtlWords;
   p = align_to(p, 16);
@@ -375,6 +450,9 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
   s.ring = base;
   s.full = reinterpret_cast<uint64_t *>(base + o.full);
   s.empty = reinterpret_cast<uint64_t *>(base + o.empty);
+  s.abar = reinterpret_cast<uint64_t *>(base + o.abar);
+  s.mdone = reinterpret_cast<uint64_t *>(base + o.mdone);
+  s.tmem = reinterpret_cast<uint32_t *>(base + o.tmem);
   s.ctl = reinterpret_cast<volatile int *>(base + o.ctl);
   s.tmark = reinterpret_cast<unsigned long long *>(base + o.tmark);
   s.red = reinterpret_cast<float *>(base + o.red);
@@ -446,35 +524,75 @@ __device__ __forceinline__ Gemv gemv_of(const Params &p, int type, int layer, in
   return g;
 }
 
-// A projection task on tensor cores: its m-tiles [mt0, mt1) of the
-// fragment-ordered matrix are streamed as row blocks of mb m-tiles, each row
-// block as nkc ring stages of (up to) kcb k-blocks.  Every (m-tile, k-block)
-// is one 512-byte fragment block; stage (rb, kc) packs the blocks of its
-// m-tiles as [m-tile][k-block].
-struct MmaTile {
-  const uint16_t *w;  // the operator's matrix, fragment order
-  int KB;             // k-blocks per row (K / 16)
-  int mt0, mt1;       // m-tiles of this task
-  int mb, kcb, nkc, nrb;
+// A projection task on tcgen05 tensor cores (batch >= 2).  The task's rows
+// (padded to a multiple of 16) run in passes of up to kUmmaMaxN rows (one
+// accumulator of 128 lanes x N columns in TMEM); a pass streams its weights in
+// ring stages of nkb 16-column k-blocks.  In the arena each task's rows are
+// contiguous, pass by pass, and a pass of N rows holds, per k-block, its N x 16
+// weights in the core-matrix order (N * 32 bytes: the B operand of one MMA),
+// so a stage is one contiguous copy.  A stage's slot holds those weights, then
+// the matching operand chunk (512 nn bytes per k-block: the A operand), then
+// kUmmaSlack bytes that the A descriptors of the chunk's last k-blocks read
+// past it (rows 16 nn .. 127 of A, which only reach accumulator lanes that
+// are never read).
+struct UTile {
+  const uint8_t *w;  // the task's first weight byte
+  int K, KB;         // columns, 16-column k-blocks
+  int row0, rows;    // first row of the task, rows (a multiple of 16)
+  int npass, nlast;  // passes, rows of the last pass
+  int nkb_full, nkc_full, nkb_last, nkc_last;  // k-blocks per stage, stages of a pass
+  int nst;           // stages of the task
 };
 
-__device__ __forceinline__ MmaTile mma_tile(const Params &p, int type, int layer, int idx) {
+// k-blocks per stage for a pass of N rows (weights, operand and slack fit the slot).
+__device__ __forceinline__ int umma_nkb(const Params &p, int N, int KB) {
+  const int n = (p.stage_bytes - kUmmaSlack) / (N * 32 + 512 * p.nn);
+  return min(KB, max(n, 1));
+}
+
+__device__ __forceinline__ UTile umma_tile(const Params &p, int type, int layer, int idx) {
   const Gemv g = gemv_of(p, type, layer, idx);
-  MmaTile m;
-  m.w = g.w;
-  m.KB = g.K >> 4;
-  m.mt0 = g.row0 >> 4;
-  m.mt1 = (g.row1 + 15) >> 4;  // the LM head's last m-tile may hold zero padding rows
-  switch (type) {
-    case 2: m.mb = p.mb_qkv; m.kcb = p.kcb_qkv; break;
-    case 5: m.mb = p.mb_o; m.kcb = p.kcb_o; break;
-    case 6: m.mb = p.mb_gu; m.kcb = p.kcb_gu; break;
-    case 7: m.mb = p.mb_down; m.kcb = p.kcb_down; break;
-    default: m.mb = p.mb_lm; m.kcb = p.kcb_lm; break;
+  UTile u;
+  u.K = g.K;
+  u.KB = g.K >> 4;
+  u.row0 = g.row0;
+  u.rows = (g.row1 - g.row0 + 15) & ~15;  // the LM head's last task: zero padding rows
+  u.w = reinterpret_cast<const uint8_t *>(g.w) + (size_t)g.row0 * g.K * 2;
+  u.npass = (u.rows + kUmmaMaxN - 1) / kUmmaMaxN;
+  u.nlast = u.rows - (u.npass - 1) * kUmmaMaxN;
+  u.nkb_full = umma_nkb(p, kUmmaMaxN, u.KB);
+  u.nkc_full = (u.KB + u.nkb_full - 1) / u.nkb_full;
+  u.nkb_last = umma_nkb(p, u.nlast, u.KB);
+  u.nkc_last = (u.KB + u.nkb_last - 1) / u.nkb_last;
+  u.nst = (u.npass - 1) * u.nkc_full + u.nkc_last;
+  return u;
+}
+
+// Stage st of a task: pass q, rows N, first k-block kb0, k-blocks nkb of a
+// full stage of the pass and nkb_here of this one, weight byte offset.
+struct UStage {
+  int q, c, N, nkb, kb0, nkb_here;
+  size_t woff;
+};
+
+__device__ __forceinline__ UStage umma_stage(const UTile &u, int st) {
+  UStage s;
+  const int full = (u.npass - 1) * u.nkc_full;
+  if (st < full) {
+    s.q = st / u.nkc_full;
+    s.c = st - s.q * u.nkc_full;
+    s.N = kUmmaMaxN;
+    s.nkb = u.nkb_full;
+  } else {
+    s.q = u.npass - 1;
+    s.c = st - full;
+    s.N = u.nlast;
+    s.nkb = u.nkb_last;
   }
-  m.nkc = (m.KB + m.kcb - 1) / m.kcb;
-  m.nrb = (m.mt1 - m.mt0 + m.mb - 1) / m.mb;
-  return m;
+  s.kb0 = s.c * s.nkb;
+  s.nkb_here = min(s.nkb, u.KB - s.kb0);
+  s.woff = (size_t)s.q * kUmmaMaxN * u.K * 2 + (size_t)s.kb0 * s.N * 32;
+  return s;
 }
 
 struct AttnSpan {
@@ -499,6 +617,98 @@ __device__ __forceinline__ AttnSpan attn_span(const Params &p, int idx) {
   return a;
 }
 
+// JIT attention (MPK review, "Direction 4": the data-dependent operator is
+// resolved at run time).  The pairs p = b * Hkv + g, each with n_b = L_b + 1
+// positions (its cached rows and the new one), lie end to end on one line of
+// T positions; task a takes positions [a C, (a + 1) C) of it, so the tasks of
+// a layer carry equal work whatever the KV lengths, and a task may cover the
+// end of one pair and the start of the next.  C = the larger of ceil(T / A)
+// and ceil(max n_b / (S - 1)), rounded up to 16: at most S tasks touch a pair
+// (S = the partial slots per pair).  Every task and its producer derive the
+// same pieces from kv_len, which no task of the step changes before ARGMAX.
+struct JitPart {
+  int C, T;
+};
+
+__device__ __forceinline__ JitPart jit_part(const Params &p) {
+  int T = 0, nmax = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int n = __ldcg(p.kv_len + b) + 1;
+    T += n * p.Hkv;
+    nmax = max(nmax, n);
+  }
+  int C = (T + p.n_attn - 1) / p.n_attn;
+  C = max(C, (nmax + p.S - 2) / (p.S - 1));
+  return JitPart{(C + 15) & ~15, T};
+}
+
+// One piece of an attention task: cached rows [c0, c1) of pair (b, g)
+// streamed in stages at origin o (stage st covers [o + st pps, o + (st + 1)
+// pps), clipped to [c0, c1)), the new row (position L) if has_new; the
+// piece's result is partial slot `slot` of the `expect` tasks that complete
+// the pair (expect == 1: written straight to att), and the last of them
+// merges `nmerge` partials.
+struct AttnSeg {
+  int b, g, L;
+  int c0, c1, o;
+  bool has_new;
+  int slot, expect, nmerge;
+};
+
+__device__ __forceinline__ int seg_stages(const Params &p, const AttnSeg &s) {
+  return s.c1 > s.c0 ? (s.c1 - 1 - s.o) / p.pps + 1 : 0;
+}
+
+// The pieces of JIT task a, in line order.
+struct JitCursor {
+  int a, C, x, x1, b, g, r, n;
+  __device__ __forceinline__ void start(const Params &p, int task, const JitPart &jp) {
+    a = task;
+    C = jp.C;
+    x = min(a * C, jp.T);
+    x1 = min(x + C, jp.T);
+    int rest = x;
+    b = 0;
+    g = 0;
+    r = 0;
+    n = 1;
+    for (; b < p.B; ++b) {
+      n = __ldcg(p.kv_len + b) + 1;
+      if (rest < n * p.Hkv) {
+        g = rest / n;
+        r = rest - g * n;
+        break;
+      }
+      rest -= n * p.Hkv;
+    }
+  }
+  __device__ __forceinline__ bool next(const Params &p, AttnSeg &s) {
+    if (x >= x1) return false;
+    const int len = min(n - r, x1 - x);
+    const int pp = x - r;  // line position of the pair's row 0
+    s.b = b;
+    s.g = g;
+    s.L = n - 1;
+    s.c0 = r;
+    s.c1 = min(r + len, s.L);
+    s.o = r / p.pps * p.pps;
+    s.has_new = r + len == n;
+    s.slot = a - pp / C;
+    s.expect = (pp + n - 1) / C - pp / C + 1;
+    s.nmerge = s.expect;
+    x += len;
+    r += len;
+    if (r == n) {
+      r = 0;
+      if (++g == p.Hkv) {
+        g = 0;
+        if (++b < p.B) n = __ldcg(p.kv_len + b) + 1;
+      }
+    }
+    return true;
+  }
+};
+
 // Element offset of cache row `row` of (layer, sequence b, kv head g): the
 // contiguous layout, or row % P of the sequence's page of the paged pools.
 __device__ __forceinline__ size_t kv_row(const Params &p, int layer, int b, int g, int row) {
@@ -516,19 +726,34 @@ struct Stream {
   uint32_t bytes = 0, last_bytes = 0;  // bytes of a full / of the last stage
   uint32_t stride = 0;            // bytes between consecutive stages
   int nst = 0;                    // stages
-  // tensor-core projections: stage st = (row block st / nkc, k chunk st % nkc)
-  int nkc = 0;                    // 0 for the other streams
-  int KB = 0, mt0 = 0, mt1 = 0, mb = 0, kcb = 0;
+  // tensor-core projections: stages as umma_stage(u, st)
+  int uk = 0;                     // 0 for the other streams
+  UTile u{};
   // attention: K/V rows y0 + st * pps .. of the 2-D cache tensor maps (paged
   // pools: stage st starts at position kv_p0 + st * pps of (layer, b, g);
   // a stage never crosses a page)
   int kv = 0;
   int y0 = 0;
   int kv_l = 0, kv_b = 0, kv_g = 0, kv_p0 = 0;
+  // JIT attention: the pieces of task ja (see JitCursor), stages in piece order
+  int jit = 0, ja = 0;
+  JitPart jp{};
 };
 
 // First cache row (in rows of D elements) of K/V stage st of stream s.
 __device__ __forceinline__ int kv_stage_row(const Params &p, const Stream &s, int st) {
+  if (s.jit) {  // the piece holding stage st; the stage starts at its first row
+    JitCursor cur;
+    cur.start(p, s.ja, s.jp);
+    AttnSeg sg;
+    while (cur.next(p, sg)) {
+      const int n = seg_stages(p, sg);
+      if (st < n)
+        return (int)(kv_row(p, s.kv_l, sg.b, sg.g, max(sg.c0, sg.o + st * p.pps)) / p.D);
+      st -= n;
+    }
+    return 0;  // not reached: st < the task's stage count
+  }
   if (p.page_size > 0) return (int)(kv_row(p, s.kv_l, s.kv_b, s.kv_g, s.kv_p0 + st * p.pps) / p.D);
   return s.y0 + st * p.pps;
 }
@@ -539,15 +764,23 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
   Stream s{};
   const int type = t.type;
   if (kMma && (type == 2 || (type >= 5 && type <= 8))) {
-    const MmaTile m = mma_tile(p, type, t.layer, (int)t.idx);
-    s.src0 = reinterpret_cast<const uint8_t *>(m.w);
-    s.nst = m.nrb * m.nkc;
-    s.nkc = m.nkc;
-    s.KB = m.KB;
-    s.mt0 = m.mt0;
-    s.mt1 = m.mt1;
-    s.mb = m.mb;
-    s.kcb = m.kcb;
+    s.u = umma_tile(p, type, t.layer, (int)t.idx);
+    s.uk = 1;
+    s.nst = s.u.nst;
+    return s;
+  }
+  if (kMma && type == 3 && p.jit) {
+    // whole boxes of pps rows from each stage's first row (masked past its end)
+    s.jp = jit_part(p);
+    s.ja = (int)t.idx;
+    s.jit = 1;
+    s.kv = 1;
+    s.kv_l = t.layer;
+    JitCursor cur;
+    cur.start(p, s.ja, s.jp);
+    AttnSeg sg;
+    while (cur.next(p, sg)) s.nst += seg_stages(p, sg);
+    s.bytes = s.last_bytes = (uint32_t)(p.pps * p.D * 2);
     return s;
   }
   if (type == 3) {
@@ -579,11 +812,9 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
 // Bytes that stage st of stream s lands in the ring.
 template <bool kMma>
 __device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
-  if (kMma && s.nkc > 0) {
-    const int rb = st / s.nkc, kc = st - rb * s.nkc;
-    const int nm = min(s.mb, s.mt1 - (s.mt0 + rb * s.mb));
-    const int nkb = min(s.kcb, s.KB - kc * s.kcb);
-    return (uint32_t)(nm * nkb * 512);
+  if (kMma && s.uk) {
+    const UStage u = umma_stage(s.u, st);
+    return (uint32_t)(u.nkb_here * u.N * 32);
   }
   if (s.kv) return 2 * (st == s.nst - 1 ? s.last_bytes : s.bytes);  // K and V
   return st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -610,14 +841,9 @@ __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, in
     }
     return;
   }
-  if (kMma && s.nkc > 0) {
-    const int rb = st / s.nkc, kc = st - rb * s.nkc;
-    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
-    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
-    const uint32_t cb = (uint32_t)nkb * 512u;
-    for (int i = 0; i < nm; ++i)
-      bulk_g2s(dst + (size_t)i * cb, s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb, bar,
-               pol);
+  if (kMma && s.uk) {  // the stage's weights: one contiguous copy
+    const UStage u = umma_stage(s.u, st);
+    bulk_g2s(dst, s.u.w + u.woff, (uint32_t)(u.nkb_here * u.N * 32), bar, pol);
     return;
   }
   const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -627,13 +853,11 @@ __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, in
 // Prefetch stage st of stream s into L2; returns the bytes requested.
 template <bool kMma>
 __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
-  if (kMma && s.nkc > 0) {
-    const int rb = st / s.nkc, kc = st - rb * s.nkc;
-    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
-    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
-    const uint32_t cb = (uint32_t)nkb * 512u;
-    for (int i = 0; i < nm; ++i) prefetch_l2(s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb);
-    return cb * (uint32_t)nm;
+  if (kMma && s.uk) {
+    const UStage u = umma_stage(s.u, st);
+    const uint32_t nb = (uint32_t)(u.nkb_here * u.N * 32);
+    prefetch_l2(s.u.w + u.woff, nb);
+    return nb;
   }
   if (s.kv) return 0u;  // K/V tiles are not prefetched
   const uint32_t pb = st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -648,7 +872,31 @@ constexpr uint64_t kPrefetchHoldNs = 1500;  // see producer_loop
 
 struct Queue {
   int first, stride, count;  // tasks first, first + stride, ... (count of them)
+  // dispatch mode: the entries the scheduler publishes for this worker
+  const int32_t *list = nullptr;
+  const uint32_t *tail = nullptr;
 };
+
+// Task id of entry n of the worker's queue, or -1 past its end (static
+// queues) / at the scheduler's end mark.  In dispatch mode the entry is
+// waited for (bounded); -1 also when the CTA aborts or the wait runs out.
+__device__ __forceinline__ int queue_task(const Params &p, const Smem &sm, const Queue &q, int n) {
+  if (!q.list) return n < q.count ? q.first + n * q.stride : -1;
+  if ((int32_t)(ld_acquire(q.tail) - (uint32_t)n) <= 0) {
+    const uint64_t t0 = global_timer();
+    uint32_t spins = 0;
+    while ((int32_t)(ld_acquire(q.tail) - (uint32_t)n) <= 0) {
+      if (sm.ctl[kAbort]) return -1;
+      if (++spins > 16) __nanosleep(64);
+      if ((spins & 63u) == 0 && global_timer() - t0 > 4ull * p.timeout_ns + 1000000000ull) {
+        record_error(p, kDevTimeout, -1, -3);
+        sm.ctl[kAbort] = 1;
+        return -1;
+      }
+    }
+  }
+  return __ldcg(q.list + n);
+}
 
 template <bool kMma>
 __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
@@ -660,8 +908,12 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // oldest stage has landed and stayed unconsumed for over kPrefetchHoldNs
   // (the compute warps wait on an event or run attention, so HBM has spare
   // capacity) the producer prefetches the next stages into L2, up to
-  // l2_prefetch_bytes ahead of the ring.
-  const long long dist = p.l2_prefetch_bytes;
+  // l2_prefetch_bytes ahead of the ring, one stage per few polls of the ring:
+  // a burst of prefetches from every SM at once slows the attention tasks,
+  // which sit on the critical path (Qwen3-8B at batch 1: 3141 us per step
+  // with back-to-back prefetches in the attention window against 3095 us).
+  // (dispatch mode: the queue holds only tasks that are ready, no lookahead)
+  const long long dist = q.list ? 0 : p.l2_prefetch_bytes;
   const uint64_t pol = stream_policy(p.evict_first != 0);
   int pf_n = 0, pf_st = 0;
   Stream pfs{};
@@ -676,14 +928,16 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // streams are never gated, so they run ahead across the step boundary.
   bool kv_open = s == 0;
   for (int n = 0; n < q.count; ++n) {
-    const DevTask tk = p.tasks[q.first + n * q.stride];
+    const int tid_n = queue_task(p, sm, q, n);
+    if (tid_n < 0) break;
+    const DevTask tk = p.tasks[tid_n];
     if (tk.type == 3 && !kv_open) {
       const uint64_t t0 = global_timer();
       uint32_t spins = 0;
       while ((int32_t)(ld_acquire(p.epoch) - (epoch0 + (uint32_t)s - 1u)) < 0) {
         if (sm.ctl[kAbort]) goto out;
         if ((++spins & 63u) == 0 && global_timer() - t0 > budget) {
-          record_error(p, kDevTimeout, q.first + n * q.stride, -1);
+          record_error(p, kDevTimeout, tid_n, -1);
           goto out;
         }
       }
@@ -712,8 +966,9 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       const uint32_t use = k / NS;
       if (use > 0) {
         const uint32_t par = (use - 1) & 1u;
-        uint64_t t0 = 0, t_held = 0;
+        uint64_t t0 = 0;
         uint32_t spins = 0;
+        uint64_t t_held = 0;
         while (!mbar_test(&sm.empty[slot], par)) {
           if (sm.ctl[kAbort]) goto out;
           ++spins;
@@ -747,7 +1002,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
             uint64_t now = global_timer();
             if (t0 == 0) t0 = now;
             else if (now - t0 > budget) {
-              record_error(p, kDevTimeout, q.first + n * q.stride, -1);
+              record_error(p, kDevTimeout, tid_n, -1);
               goto out;
             }
           }
@@ -841,7 +1096,8 @@ struct DepWait {
   uint32_t epoch;
   int task;
   __device__ __forceinline__ bool operator()() const {
-    if (p.persistent && dep >= 0 && threadIdx.x == 0) {
+    // (dispatch mode: the scheduler hands out a task once its event fired)
+    if (p.persistent && !p.dispatch && dep >= 0 && threadIdx.x == 0) {
       if (!wait_event(p, dep, epoch, task)) sm.ctl[kAbort] = 1;
     }
     compute_sync();
@@ -1084,64 +1340,8 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 }
 
 // ---------------------------------------------------------------------------
-// Projection task on tensor cores (batch >= 2).
+// Projection task on tcgen05 tensor cores (batch >= 2).
 // ---------------------------------------------------------------------------
-// B fragments of k-blocks kb0 + warp + 8 j (j < kpw) of the operand xb: the
-// activations are written earlier in this step by other SMs, so they are read
-// through L2 (never from a possibly stale L1 line).
-template <int NN>
-__device__ __forceinline__ void load_bfrag(uint4 (&bf)[mma_max_kpw(NN)][NN], const uint16_t *xb,
-                                           int kb0, int kpw, int warp, int lane) {
-#pragma unroll
-  for (int j = 0; j < mma_max_kpw(NN); ++j) {
-    if (j < kpw) {
-#pragma unroll
-      for (int n = 0; n < NN; ++n)
-        bf[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
-                              xb + ((size_t)(kb0 + warp + 8 * j) * NN + n) * 256) + lane);
-    }
-  }
-}
-
-// One ring stage of a projection with compile-time tile counts (MBF m-tiles,
-// KPWF k-blocks per warp): the common cases, with no per-tile guards, so the
-// A fragments of a k-block are loaded before its MMAs.  The B fragments of
-// the next stage's first kpw_n k-blocks are refilled after their last use.
-template <int NN, int MBF, int KPWF, bool kGuard>
-__device__ __forceinline__ void mma_stage_fixed(float (&acc)[kMmaMaxMB][NN][4],
-                                                uint4 (&bc)[mma_max_kpw(NN)][NN], const uint8_t *slot,
-                                                const uint16_t *xn, int kpw_n, int warp, int lane) {
-  constexpr int NKB = 8 * KPWF;
-#pragma unroll
-  for (int j = 0; j < KPWF; ++j) {
-    const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
-    uint4 a[MBF];
-#pragma unroll
-    for (int m = 0; m < MBF; ++m) a[m] = *reinterpret_cast<const uint4 *>(blk + m * NKB * 512);
-#pragma unroll
-    for (int m = 0; m < MBF; ++m)
-#pragma unroll
-      for (int n = 0; n < NN; ++n) {
-        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
-        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
-      }
-    if (!kGuard || j < kpw_n) {
-#pragma unroll
-      for (int n = 0; n < NN; ++n)
-        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
-    }
-  }
-  // a next stage with more k-blocks (the first chunk after a short last one)
-#pragma unroll
-  for (int j = KPWF; j < (kGuard ? mma_max_kpw(NN) : 0); ++j) {
-    if (j < kpw_n) {
-#pragma unroll
-      for (int n = 0; n < NN; ++n)
-        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
-    }
-  }
-}
-
 // Sum over the 16 lanes of a half warp (lanes that share a sequence column).
 __device__ __forceinline__ float half_warp_sum(float v) {
 #pragma unroll
@@ -1149,29 +1349,63 @@ __device__ __forceinline__ float half_warp_sum(float v) {
   return v;
 }
 
-// The batched projection y[b][r] = sum_k W[r][k] x̂[b][k] of one task on
-// mma.sync.  The input arrives as a hi/lo bf16 operand of x[b][k] * gain[k]
-// written by the producing task's epilogue, with per-16-row sums of squares;
-// the RMSNorm's per-sequence factor 1 / rms(x_b) is applied to the fp32
-// accumulators in the epilogue (it factors out of the sum over k).
+// Bounded wait for the completion of phase `par` of an mbarrier by thread 0;
+// false (with the error recorded) on timeout or abort.
+__device__ bool wait_bar(const Params &p, const Smem &sm, uint64_t *bar, uint32_t par, int task) {
+  if (mbar_test(bar, par)) return true;
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  while (!mbar_test(bar, par)) {
+    if (sm.ctl[kAbort]) return false;
+    if ((++spins & 255u) == 0) {
+      const uint64_t now = global_timer();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > 4ull * p.timeout_ns + 1000000000ull) {
+        record_error(p, kDevTimeout, task, -1);
+        sm.ctl[kAbort] = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+// Per-CTA state of the tensor-core path, kept by the compute threads across
+// tasks: the parity of the next MMA-completion phase (every compute thread)
+// and, in thread 0, the parity of each slot's next operand phase and the
+// slots whose operand copy is in flight.
+struct UmmaState {
+  uint32_t mph = 0;
+  uint32_t aph = 0, apend = 0;
+};
+
+// The batched projection y[b][r] = sum_k W[r][k] x̂[b][k] of one task.  The
+// input arrives as the hi/lo bf16 operand of x[b][k] * gain[k] written by the
+// producing task's epilogue, with per-16-row sums of squares; the RMSNorm's
+// per-sequence factor 1 / rms(x_b) is applied to the fp32 sums in the
+// epilogue (it factors out of the sum over k).
 //
-// Work split: for each ring stage (row block x k chunk) warp w takes the
-// k-blocks w, w + 8, ... of the chunk for every m-tile of the row block, so
-// every B fragment is loaded by one warp, once per row block.  The warps'
-// partial sums of a row block are added in shared memory in a fixed order
-// (deterministic), PM m-tiles per pass, and the fused epilogue of the
-// operator runs on the sums: thread (row = tid % 16, sequence = tid / 16 % 8nn).
+// Thread 0 issues everything asynchronous: after the dependency event it
+// copies each stage's operand chunk into the stage's slot (bulk copies, up to
+// ring_stages - 1 stages ahead), waits for the stage's weights (the producer
+// warp) and operand, issues the stage's MMAs (M = 128: operand rows, N = the
+// pass's weight rows, one per k-block) into the pass's TMEM accumulator, and
+// commits them to the slot's empty barrier, which frees the slot once they
+// completed (the other seven arrivals of that barrier are made at once).  At
+// the end of a pass warp 0 reads the accumulator lanes 0 .. 31 (the operand
+// rows hi(b), lo(b)) back in 32-column chunks and the compute threads run the
+// operator's fused epilogue on hi + lo, thread (row tid % 16 of an m-tile,
+// sequence tid / 16 % 8 nn).
 template <int NN>
-__device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const DevTask &t,
-                                         uint32_t &k, int task_id, const DepWait &dep_wait) {
-  constexpr int NC = 8 * NN;          // operand columns (sequences, zero padded)
-  constexpr int PM = NN == 2 ? 2 : 4; // m-tiles per reduction pass
-  constexpr int CS = NC + 1;          // row stride of the reduction buffer (floats)
-  static_assert(kComputeWarps * PM * 16 * CS <= kMmaCredFloats, "reduction buffer");
+__device__ __forceinline__ bool umma_task(const Params &p, const Smem &sm, const DevTask &t,
+                                          uint32_t &k, UmmaState &us, int task_id,
+                                          const DepWait &dep_wait) {
+  constexpr int NC = 8 * NN;         // operand sequence columns (zero padded)
+  constexpr uint32_t AB = 512u * NN; // operand bytes per k-block
   const int type = t.type;
   const int layer = t.layer;
   const DevLayer *L = layer < p.Ly ? p.layers + layer : nullptr;
-  const MmaTile mt = mma_tile(p, type, layer, (int)t.idx);
+  const UTile u = umma_tile(p, type, layer, (int)t.idx);
   const uint16_t *xb;
   const float *ssp = nullptr;
   switch (type) {
@@ -1181,15 +1415,35 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
     case 7: xb = L->hb; break;
     default: xb = p.xfb; ssp = p.ssf; break;
   }
+  const uint8_t *xa = reinterpret_cast<const uint8_t *>(xb);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = tid & 15;          // row of an m-tile this thread finishes
   const int col = (tid >> 4) % NC;   // sequence this thread finishes
   const bool col_ok = col < p.B;
-  const int N = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
+  const int N_op = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
+  const int NS = p.ring_stages;
+  const uint64_t pol = stream_policy(false);  // the operand is read by every task of the operator
+  const uint32_t tmem = *sm.tmem;
 
   if (!dep_wait()) return false;
-  uint4 bc[mma_max_kpw(NN)][NN];
-  load_bfrag<NN>(bc, xb, 0, min(mt.kcb, mt.KB) >> 3, warp, lane);
+  // operand chunk of stage i (global stage k + i) into its slot, after the weights
+  auto issue_a = [&](int i) {
+    const UStage st = umma_stage(u, i);
+    const int slot = (int)((k + (uint32_t)i) % (uint32_t)NS);
+    uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes + (size_t)st.nkb * st.N * 32;
+    const uint32_t nb = (uint32_t)st.nkb_here * AB;
+    mbar_arrive_expect_tx(&sm.abar[slot], nb);
+    bulk_g2s(dst, xa + (size_t)st.kb0 * AB, nb, &sm.abar[slot], pol);
+    us.apend |= 1u << slot;
+  };
+  if (tid == 0) {
+    // the operand was written by other SMs and acquired with the event: order
+    // that before the bulk copies (async proxy) read it
+    fence_proxy_async_global();
+    // the slots of the first stages were freed by earlier tasks, which waited
+    // for their MMAs
+    for (int i = 0; i < min(NS - 1, u.nst); ++i) issue_a(i);
+  }
   float inv = 1.f;
   if (ssp) {
     for (int b = warp; b < p.B; b += kComputeWarps) {
@@ -1201,166 +1455,127 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
     compute_sync();
     inv = col_ok ? sm.minv[col] : 0.f;
   }
-
-  float acc[kMmaMaxMB][NN][4];
-#pragma unroll
-  for (int m = 0; m < kMmaMaxMB; ++m)
-#pragma unroll
-    for (int n = 0; n < NN; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
   float best_v = -INFINITY;
   int best_i = 0x7fffffff;
   trace_mark(p, sm, 0);
-  const int nst = mt.nrb * mt.nkc;
-  for (int st = 0; st < nst; ++st) {
-    const int rb = st / mt.nkc, kc = st - rb * mt.nkc;
-    const int m0 = mt.mt0 + rb * mt.mb, nm = min(mt.mb, mt.mt1 - m0);
-    const int nkb = min(mt.kcb, mt.KB - kc * mt.kcb), kpw = nkb >> 3;
-    // the next stage's k chunk (the same chunks repeat for every row block):
-    // each B fragment register is refilled for it right after its last use
-    const int kn = kc + 1 == mt.nkc ? 0 : kc + 1;
-    const int kpw_n = st + 1 < nst ? min(mt.kcb, mt.KB - kn * mt.kcb) >> 3 : 0;
-    const uint16_t *xn = xb + ((size_t)(kn * mt.kcb + warp) * NN) * 256;
-    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
-    if (got) {
-      trace_first_stage(p, sm, st);
-      const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
-      const bool same = kpw_n == kpw;  // the next stage refills every fragment
-      if (NN == 1 && same && kpw == 6 && nm == 2) {
-        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (NN == 1 && same && kpw == 4 && nm == 3) {
-        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (NN == 1 && kpw == 6 && nm == 2) {
-        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (NN == 1 && kpw == 4 && nm == 3) {
-        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (same && kpw == 3 && nm == 2) {
-        mma_stage_fixed<NN, 2, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (same && kpw == 3 && nm == 3) {
-        mma_stage_fixed<NN, 3, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (same && kpw == 2 && nm == 6) {
-        mma_stage_fixed<NN, 6, 2, false>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (kpw == 3 && nm == 2) {
-        mma_stage_fixed<NN, 2, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (kpw == 3 && nm == 3) {
-        mma_stage_fixed<NN, 3, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (kpw == 2 && nm == 2) {
-        mma_stage_fixed<NN, 2, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else if (kpw == 2 && nm == 3) {
-        mma_stage_fixed<NN, 3, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
-      } else {
-#pragma unroll
-      for (int j = 0; j < mma_max_kpw(NN); ++j) {
-        if (j < kpw) {
-          const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
-#pragma unroll
-          for (int m = 0; m < kMmaMaxMB; ++m) {
-            if (m < nm) {
-              const uint4 a = *reinterpret_cast<const uint4 *>(blk + (size_t)m * nkb * 512);
-#pragma unroll
-              for (int n = 0; n < NN; ++n) {
-                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
-                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
-              }
-            }
+  int st = 0;
+  for (int q = 0; q < u.npass; ++q) {
+    const int N = q < u.npass - 1 ? kUmmaMaxN : u.nlast;
+    const int nst_q = q < u.npass - 1 ? u.nkc_full : u.nkc_last;
+    if (tid == 0) {
+      const uint32_t idesc = umma_idesc(N);
+      for (int c = 0; c < nst_q; ++c, ++st) {
+        if (sm.ctl[kAbort]) continue;
+        const UStage s = umma_stage(u, st);
+        const uint32_t kg = k + (uint32_t)st;
+        const int slot = (int)(kg % (uint32_t)NS);
+        if (!wait_full(p, sm, kg, task_id)) continue;
+        if (!wait_bar(p, sm, &sm.abar[slot], (us.aph >> slot) & 1u, task_id)) continue;
+        us.aph ^= 1u << slot;
+        us.apend &= ~(1u << slot);
+        trace_first_stage(p, sm, st);
+        tc_fence_after();
+        const uint32_t wb = smem_u32(sm.ring + (size_t)slot * p.stage_bytes);
+        const uint32_t abase = wb + (uint32_t)(s.nkb * s.N * 32);
+        for (int j = 0; j < s.nkb_here; ++j)
+          umma_bf16(tmem, umma_desc(abase + (uint32_t)j * AB), umma_desc(wb + (uint32_t)(j * N * 32)),
+                    idesc, (c > 0 || j > 0) ? 1u : 0u);
+        umma_commit(&sm.empty[slot]);               // frees the slot once the MMAs completed
+        mbar_arrive_n(&sm.empty[slot], kComputeWarps - 1);
+        // the operand of stage st + NS - 1 goes into the slot of stage st - 1
+        if (st + NS - 1 < u.nst) {
+          if (st >= 1) {
+            const uint32_t kp = kg - 1u;
+            if (!wait_bar(p, sm, &sm.empty[kp % (uint32_t)NS], (kp / (uint32_t)NS) & 1u, task_id))
+              continue;
           }
-        }
-        if (j < kpw_n) {
-#pragma unroll
-          for (int n = 0; n < NN; ++n)
-            bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
-                                  xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+          issue_a(st + NS - 1);
         }
       }
-      }
-      release_stage(sm, p, k);
-      ++k;
+      umma_commit(sm.mdone);  // arrives once every MMA issued so far completed
+    } else {
+      st += nst_q;
     }
-    if (kc + 1 < mt.nkc) continue;
-
-    // row block done: cross-warp sums and the fused epilogue, PM m-tiles per pass
-#pragma unroll
-    for (int q0 = 0; q0 < kMmaMaxMB; q0 += PM) {
-      if (q0 >= nm) break;  // uniform over the CTA
-      {
-        const int g = lane >> 2, tq = lane & 3;
-#pragma unroll
-        for (int ml = 0; ml < PM; ++ml) {
-          const int m = q0 + ml;
-          if (m < kMmaMaxMB && m < nm) {
-            float *cw = sm.cred + (size_t)(warp * PM + ml) * 16 * CS;
-#pragma unroll
-            for (int n = 0; n < NN; ++n) {
-              const int c = n * 8 + 2 * tq;
-              cw[g * CS + c] = acc[m][n][0];
-              cw[g * CS + c + 1] = acc[m][n][1];
-              cw[(g + 8) * CS + c] = acc[m][n][2];
-              cw[(g + 8) * CS + c + 1] = acc[m][n][3];
-            }
+    // every compute thread: the pass's accumulator is complete
+    {
+      uint64_t t0 = 0;
+      uint32_t spins = 0;
+      while (!mbar_test(sm.mdone, us.mph & 1u)) {
+        if ((++spins & 255u) == 0) {
+          const uint64_t now = global_timer();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > 4ull * p.timeout_ns + 1000000000ull) {
+            if (tid == 0) record_error(p, kDevTimeout, task_id, -1);
+            sm.ctl[kAbort] = 1;
+            break;
           }
         }
+      }
+      us.mph ^= 1u;
+    }
+    compute_sync();
+    if (sm.ctl[kAbort]) break;
+    tc_fence_after();
+    // epilogue, 32 accumulator columns (two 16-row m-tiles of the pass) at a time
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      if (warp == 0) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (uint32_t)c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sm.cred[j * 33 + lane] = __uint_as_float(v[j]);
       }
       compute_sync();
-      if (!sm.ctl[kAbort]) {
 #pragma unroll
-        for (int it = 0; it < PM * NC / 16; ++it) {
-          const int ml = (tid + kComputeThreads * it) / (16 * NC);  // uniform per warp
-          const bool m_ok = q0 + ml < nm;
-          float v = 0.f;
-          if (m_ok) {
-#pragma unroll
-            for (int w = 0; w < kComputeWarps; ++w)
-              v += sm.cred[((size_t)(w * PM + ml) * 16 + row) * CS + col];
+      for (int it = 0; it < 32 * NC / kComputeThreads; ++it) {
+        const int ml = (tid + kComputeThreads * it) / (16 * NC);  // m-tile of the chunk, uniform per warp
+        const int j = ml * 16 + row;
+        const bool m_ok = c0 + ml * 16 < N;
+        const float v = m_ok ? sm.cred[j * 33 + col] + sm.cred[j * 33 + NC + col] : 0.f;
+        const int r = u.row0 + q * kUmmaMaxN + c0 + j;  // row of the operator's output
+        const bool store = m_ok && col_ok && r < N_op;
+        const size_t bH = (size_t)col * p.H;
+        if (type == 2) {
+          if (store) L->qkv[(size_t)col * p.n_qkv + r] = v * inv;
+        } else if (type == 5 || type == 7) {
+          // residual add, next operand (gain of the following norm), 16-row ss
+          float x = 0.f;
+          if (store) {
+            x = __ldcg((type == 5 ? L->x_in : L->xm) + bH + r) + v;
+            (type == 5 ? L->xm : L->x_out)[bH + r] = x;
+            const uint16_t *gn = type == 5 ? L->mlp_norm : L->gain_next;
+            put_opnd(type == 5 ? L->xmb : L->xa_next, r, col, NN, x * bf2f(gn[r]));
           }
-          const int r = (m0 + q0 + ml) * 16 + row;  // row of the operator's output
-          const bool store = m_ok && col_ok && r < N;
-          const size_t bH = (size_t)col * p.H;
-          if (type == 2) {
-            if (store) L->qkv[(size_t)col * p.n_qkv + r] = v * inv;
-          } else if (type == 5 || type == 7) {
-            // residual add, next operand (gain of the following norm), 16-row ss
-            float x = 0.f;
-            if (store) {
-              x = __ldcg((type == 5 ? L->x_in : L->xm) + bH + r) + v;
-              (type == 5 ? L->xm : L->x_out)[bH + r] = x;
-              const uint16_t *gn = type == 5 ? L->mlp_norm : L->gain_next;
-              put_opnd(type == 5 ? L->xmb : L->xa_next, r, col, NN, x * bf2f(gn[r]));
-            }
-            const float s2 = half_warp_sum(x * x);
-            if (store && row == 0)
-              (type == 5 ? L->ssm : L->ssa_next)[(size_t)col * p.n_parts + (r >> 4)] = s2;
-          } else if (type == 6) {
-            // rows (2i, 2i + 1) = (gate_i, up_i) sit on neighbouring lanes
-            const float gv = v * inv;
-            const float uv = __shfl_xor_sync(0xffffffffu, gv, 1);
-            if (store && !(row & 1)) {
-              const int i = r >> 1;
-              const float hv = gv / (1.f + __expf(-gv)) * uv;
-              L->h[(size_t)col * p.F + i] = hv;
-              put_opnd(L->hb, i, col, NN, hv);
-            }
-          } else {
-            const float lv = v * inv;
-            if (store) {
-              if (p.logits && sm.ctl[kLogits]) p.logits[(size_t)col * p.V + r] = lv;
-              if (lv > best_v || (lv == best_v && r < best_i)) {
-                best_v = lv;
-                best_i = r;
-              }
+          const float s2 = half_warp_sum(x * x);
+          if (store && row == 0)
+            (type == 5 ? L->ssm : L->ssa_next)[(size_t)col * p.n_parts + (r >> 4)] = s2;
+        } else if (type == 6) {
+          // rows (2i, 2i + 1) = (gate_i, up_i) sit on neighbouring lanes
+          const float gv = v * inv;
+          const float uv = __shfl_xor_sync(0xffffffffu, gv, 1);
+          if (store && !(row & 1)) {
+            const int i = r >> 1;
+            const float hv = gv / (1.f + __expf(-gv)) * uv;
+            L->h[(size_t)col * p.F + i] = hv;
+            put_opnd(L->hb, i, col, NN, hv);
+          }
+        } else {
+          const float lv = v * inv;
+          if (store) {
+            if (p.logits && sm.ctl[kLogits]) p.logits[(size_t)col * p.V + r] = lv;
+            if (lv > best_v || (lv == best_v && r < best_i)) {
+              best_v = lv;
+              best_i = r;
             }
           }
         }
       }
       compute_sync();
     }
-#pragma unroll
-    for (int m = 0; m < kMmaMaxMB; ++m)
-#pragma unroll
-      for (int n = 0; n < NN; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+    // the accumulator's reads are complete before the next pass's MMAs
+    tc_fence_before();
+    compute_sync();
   }
+  k += (uint32_t)u.nst;
   trace_mark(p, sm, 1);
   if (sm.ctl[kAbort]) return false;
   if (type == 8) {
@@ -1393,7 +1608,7 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
           bi = oi;
         }
       }
-      if (bi == 0x7fffffff) bi = mt.mt0 * 16;  // all values NaN: keep a valid index
+      if (bi == 0x7fffffff) bi = u.row0;  // all values NaN: keep a valid index
       p.lm_val[(size_t)tid * p.n_lm + t.idx] = bv;
       p.lm_idx[(size_t)tid * p.n_lm + t.idx] = bi;
     }
@@ -1412,20 +1627,21 @@ __device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const 
 // acquire-release atomic orders every split's partial before the merge reads.
 // Each warp owns (head, 64 dims) slices and issues a pass of kPass splits'
 // loads at once; passes combine online.
+// expect: the arrivals that complete (b, g); ns: the partial slots 0 .. ns - 1
+// to merge.
 __device__ __forceinline__ bool attn_arrive_and_merge(const Params &p, const Smem &sm, int layer,
-                                                      int b, int g) {
+                                                      int b, int g, int expect, int ns) {
   constexpr int kPass = 24;  // splits merged per round trip
   compute_sync();  // every thread's partial stores precede the arrival
   uint32_t *ctr = p.arrivals + ((size_t)layer * p.B + b) * p.Hkv + g;
   if (threadIdx.x == 0) {
     const uint32_t old = atom_acq_rel_add(ctr, 1u);
-    sm.ctl[kLast] = old + 1u == (uint32_t)p.S;
+    sm.ctl[kLast] = old + 1u == (uint32_t)expect;
   }
   compute_sync();
   if (!sm.ctl[kLast]) return true;
   if (threadIdx.x == 0) *ctr = 0u;  // every split of this step has arrived
   const DevLayer &L = p.layers[layer];
-  const int ns = min(p.S, __ldcg(p.kv_len + b) / p.chunk + 1);  // splits that hold any position
   const int D = p.D, rep = p.rep;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per_head = D / 64;  // warps per head (64 dims each, 2 per lane)
@@ -1680,51 +1896,38 @@ __device__ __forceinline__ void attn_block16_mma(uint32_t kbase, uint32_t vbase,
   }
 }
 
-// Decode attention for one (sequence b, kv head g, split s): q/k RMSNorm and
-// RoPE prologue, K/V append, then every warp runs flash-decoding style over
-// its own 8-position blocks on tensor cores (no CTA barrier inside the loop)
-// and the warps' states are merged once at the end.  D: head dim (64, 128);
-// SWZ: the K/V tiles arrive as swizzled TMA boxes (else as plain rows).
+// Decode attention of one piece (see AttnSeg) on tensor cores: q/k RMSNorm
+// and RoPE prologue, K/V append when the piece holds the new row, then every
+// warp runs flash-decoding style over its own position blocks of the piece's
+// stages (no CTA barrier inside the loop), the warps' states are merged once,
+// and the piece's result goes to att (a piece that completes its pair alone)
+// or to its partial slot, the last arriving piece of the pair merging.
+// D: head dim (64, 128); SWZ: the K/V tiles arrive as swizzled TMA boxes
+// (else as plain rows).  gq, gk: this lane's q/k norm gains.
 template <int D, bool SWZ>
-__device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
-                                          uint32_t &k, int task_id, const DepWait &dep_wait) {
+__device__ __forceinline__ bool attn_piece(const Params &p, const Smem &sm, int layer,
+                                           const AttnSeg &sg, const float (&gq)[4],
+                                           const float (&gk)[4], uint32_t &k, int task_id) {
   constexpr int NP = 8;  // positions per warp block
-  // the span read before the wait is exact when the launch runs one step
-  // (kv_len is fixed during it); a multi-step launch re-reads it after the wait
-  const AttnSpan a0 = attn_span(p, (int)t.idx);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rep = p.rep;
   constexpr int dpl = D >> 5;
-  const DevLayer &L = p.layers[t.layer];
-  const float *qkv = L.qkv + (size_t)a0.b * p.n_qkv + (size_t)a0.g * p.grp;
-  // gains and RoPE factors of this lane's dims (the RoPE position is the
-  // speculative one above): loaded before the wait
-  float gq[4], gk[4], rc[2], rs[2];
-  for (int i = 0; i < dpl; ++i) {
-    gq[i] = bf2f(L.q_norm[lane + 32 * i]);
-    gk[i] = bf2f(L.k_norm[lane + 32 * i]);
-  }
-  auto load_rope = [&](int pos) {  // [D/2][2] cos, sin of position pos
-    const float *rope = p.rope + (size_t)pos * D;
+  const DevLayer &L = p.layers[layer];
+  const float *qkv = L.qkv + (size_t)sg.b * p.n_qkv + (size_t)sg.g * p.grp;
+  float rc[2], rs[2];
+  {
+    const float *rope = p.rope + (size_t)sg.L * D;  // [D/2][2] cos, sin of position L
     for (int i = 0; i < (dpl >> 1); ++i) {
       rc[i] = rope[2 * (lane + 32 * i)];
       rs[i] = rope[2 * (lane + 32 * i) + 1];
     }
-  };
-  load_rope(a0.L);
-  if (!dep_wait()) return false;
-  AttnSpan a = a0;
-  if (p.n_steps > 1) {  // kv_len advanced by the previous step of this launch
-    a = attn_span(p, (int)t.idx);
-    if (a.L != a0.L) load_rope(a.L);
   }
-  if (!a.active)  // the split starts past the new row: it only arrives
-    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
-
-  // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
+  // every warp's state slots of the previous piece have been read
+  compute_sync();
+  // prologue: per-head RMSNorm + RoPE of q (and of the new k when this piece
   // holds position L; v is only rounded)
   for (int row = warp; row < rep + 2; row += kComputeWarps) {
-    if (row >= rep && !a.has_new) continue;
+    if (row >= rep && !sg.has_new) continue;
     float v[4];
     for (int i = 0; i < dpl; ++i) v[i] = __ldcg(qkv + row * D + lane + 32 * i);
     if (row <= rep) {  // q heads and k
@@ -1746,7 +1949,7 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     } else {
       uint16_t *cache = row == rep ? p.k_cache : p.v_cache;
       uint16_t *dst = row == rep ? sm.knew : sm.vnew;
-      const size_t off = kv_row(p, t.layer, a.b, a.g, a.L);
+      const size_t off = kv_row(p, layer, sg.b, sg.g, sg.L);
       for (int i = 0; i < dpl; ++i) {
         const uint16_t hb = f2bf(v[i]);
         cache[off + lane + 32 * i] = hb;
@@ -1780,16 +1983,16 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
   const bool np16 = p.pps % (2 * NP) == 0;
   trace_mark(p, sm, 0);
 
-  const int cached = a.cached_end - a.p0;
-  const int nst = cached > 0 ? (cached + p.pps - 1) / p.pps : 0;
+  const int nst = seg_stages(p, sg);
   for (int st = 0; st < nst; ++st) {
-    const int n = min(p.pps, cached - st * p.pps);
+    const int r0 = max(sg.c0, sg.o + st * p.pps);
+    const int n = min(sg.c1, sg.o + (st + 1) * p.pps) - r0;  // rows of the box that count
     const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
     if (!got) continue;
     trace_first_stage(p, sm, st);
     const uint32_t kb = smem_u32(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
     const uint32_t vb = kb + (uint32_t)(p.pps * D * 2);  // V boxes follow the K boxes
-    // blocks are numbered across the split's stages and dealt round-robin
+    // blocks are numbered across the piece's stages and dealt round-robin
     // (warp w takes global blocks w, w + 8, ...), so a stage whose block
     // count is not a multiple of 8 does not leave the same warps idle every
     // time; warps drift apart by at most the ring depth
@@ -1808,8 +2011,9 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
     ++k;
   }
   // the new row: one more block, on the warp after the last cached block
+  const int cached = max(0, sg.c1 - sg.c0);
   const int blk = np16 ? 2 * NP : NP;
-  if (a.has_new && warp == ((cached + blk - 1) / blk) % kComputeWarps)
+  if (sg.has_new && warp == ((cached + blk - 1) / blk) % kComputeWarps)
     attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, pk, qh, ql, m_run, l_run,
                              o);
 
@@ -1859,12 +2063,12 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
       den = fmaf(e, sw[D + 1], den);
       num = fmaf(e, sw[d], num);
     }
-    const int head = a.g * rep + h;
-    if (p.S == 1) {
-      L.att[(size_t)a.b * p.qdim + head * D + d] = num / den;
-      if (p.mma) put_opnd(L.attb, head * D + d, a.b, p.nn, num / den);
+    const int head = sg.g * rep + h;
+    if (sg.expect == 1) {
+      L.att[(size_t)sg.b * p.qdim + head * D + d] = num / den;
+      put_opnd(L.attb, head * D + d, sg.b, p.nn, num / den);
     } else {
-      float *dst = L.part + (((size_t)a.b * p.Hq + head) * p.S + a.s) * (D + 2);
+      float *dst = L.part + (((size_t)sg.b * p.Hq + head) * p.S + sg.slot) * (D + 2);
       dst[d] = num;
       if (d == 0) {
         dst[D] = M;
@@ -1872,8 +2076,53 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
       }
     }
   }
-  if (p.S == 1) return true;
-  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+  if (sg.expect == 1) return true;
+  return attn_arrive_and_merge(p, sm, layer, sg.b, sg.g, sg.expect, sg.nmerge);
+}
+
+// Decode attention task of the batched kernel: one (sequence b, kv head g,
+// split s) piece when the splits are fixed at build time, else the pieces of
+// JIT task t.idx (see JitCursor).
+template <int D, bool SWZ>
+__device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
+                                          uint32_t &k, int task_id, const DepWait &dep_wait) {
+  const int lane = threadIdx.x & 31;
+  constexpr int dpl = D >> 5;
+  const DevLayer &L = p.layers[t.layer];
+  // the norm gains of this lane's dims: weights, loaded before the wait
+  float gq[4], gk[4];
+  for (int i = 0; i < dpl; ++i) {
+    gq[i] = bf2f(L.q_norm[lane + 32 * i]);
+    gk[i] = bf2f(L.k_norm[lane + 32 * i]);
+  }
+  if (!dep_wait()) return false;
+  if (p.jit) {
+    const JitPart jp = jit_part(p);
+    JitCursor cur;
+    cur.start(p, (int)t.idx, jp);
+    AttnSeg sg;
+    while (cur.next(p, sg))
+      if (!attn_piece<D, SWZ>(p, sm, t.layer, sg, gq, gk, k, task_id)) return false;
+    return true;
+  }
+  // splits fixed at build time; kv_len is read after the wait (a multi-step
+  // launch advances it between steps)
+  const AttnSpan a = attn_span(p, (int)t.idx);
+  const int nmerge = min(p.S, a.L / p.chunk + 1);  // splits that hold any position
+  if (!a.active)  // the split starts past the new row: it only arrives
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g, p.S, nmerge);
+  AttnSeg sg;
+  sg.b = a.b;
+  sg.g = a.g;
+  sg.L = a.L;
+  sg.c0 = a.p0;
+  sg.c1 = a.cached_end;
+  sg.o = a.p0;
+  sg.has_new = a.has_new;
+  sg.slot = a.s;
+  sg.expect = p.S;
+  sg.nmerge = nmerge;
+  return attn_piece<D, SWZ>(p, sm, t.layer, sg, gq, gk, k, task_id);
 }
 
 // One block of up to NP = 32 / RP positions for one warp: scores, online
@@ -2005,8 +2254,9 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
     a = attn_span(p, (int)t.idx);
     if (a.L != a0.L) load_rope(a.L);
   }
+  const int nmerge = min(p.S, a.L / p.chunk + 1);  // splits that hold any position
   if (!a.active)  // the split starts past the new row: it only arrives
-    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g, p.S, nmerge);
 
   // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
   // holds position L; v is only rounded)
@@ -2156,7 +2406,7 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
     }
   }
   if (p.S == 1) return true;
-  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g);
+  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g, p.S, nmerge);
 }
 
 // Batch >= 2 EMBED: kept out of line so its load batches do not raise the
@@ -2166,12 +2416,11 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
 __device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
   // One item per (k-block kb, sequence b < 8 nn): its 16 embedding elements
   // 16 kb .. 16 kb + 15 (two 16-byte loads) become the fp32 row slice, the
-  // sum of squares of the 16-row part, and the 4 lane units of layer 0's
-  // QKV operand: unit (kb, column tile b / 8, lane (b % 8, t)) holds
-  // elements 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} times the attention-norm
-  // gains as hi, then lo, bf16 pairs (zeros for padded sequences).  One CTA
-  // does it all, so each thread keeps kU items' loads in flight before it
-  // uses any.
+  // sum of squares of the 16-row part, and layer 0's QKV operand rows hi(b)
+  // and lo(b) of that k-block (two 16-byte units each, see opnd_off): the
+  // elements times the attention-norm gains, zeros for padded sequences.
+  // One CTA does it all, so each thread keeps kU items' loads in flight
+  // before it uses any.
   constexpr int kU = 4;
   const DevLayer &L0 = p.layers[0];
   const int nb8 = 8 * p.nn, items = (p.H >> 4) * nb8;
@@ -2201,30 +2450,28 @@ __device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
                               e[u][1].x, e[u][1].y, e[u][1].z, e[u][1].w};
       const uint32_t gv[8] = {gw[u][0].x, gw[u][0].y, gw[u][0].z, gw[u][0].w,
                               gw[u][1].x, gw[u][1].y, gw[u][1].z, gw[u][1].w};
-      float x[16], y[16];
+      float x[16];
+      uint32_t hi[8], lo[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         x[2 * i] = bf_lo(ew[i]);
         x[2 * i + 1] = bf_hi(ew[i]);
-        y[2 * i] = x[2 * i] * bf_lo(gv[i]);
-        y[2 * i + 1] = x[2 * i + 1] * bf_hi(gv[i]);
+        split_pair(x[2 * i] * bf_lo(gv[i]), x[2 * i + 1] * bf_hi(gv[i]), hi[i], lo[i]);
       }
-      float st[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float a0 = x[2 * t], a1 = x[2 * t + 1], a8 = x[2 * t + 8], a9 = x[2 * t + 9];
-        st[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a8, a8, a9 * a9)));
-        const uint16_t h0 = f2bf(y[2 * t]), h1 = f2bf(y[2 * t + 1]);
-        const uint16_t h8 = f2bf(y[2 * t + 8]), h9 = f2bf(y[2 * t + 9]);
-        uint4 o;
-        o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
-        o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
-        o.z = (uint32_t)f2bf(y[2 * t] - bf2f(h0)) | ((uint32_t)f2bf(y[2 * t + 1] - bf2f(h1)) << 16);
-        o.w = (uint32_t)f2bf(y[2 * t + 8] - bf2f(h8)) | ((uint32_t)f2bf(y[2 * t + 9] - bf2f(h9)) << 16);
-        xa[((size_t)kb * p.nn + (b >> 3)) * 32 + (b & 7) * 4 + t] = o;
-      }
+      // rows hi(b) and lo(b) of k-block kb: 16-byte units (k halves 64 bf16 apart)
+      const size_t o = ((size_t)kb * 256 * p.nn + (b >> 3) * 128 + (b & 7) * 8) >> 3;
+      const size_t lo_o = (size_t)p.nn * 16;  // 8 nn rows further, in 16-byte units
+      xa[o] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      xa[o + 8] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      xa[o + lo_o] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      xa[o + lo_o + 8] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
       if (b < p.B) {
-        // the sum in the order of a quad's two butterfly steps
+        float st[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float a0 = x[2 * t], a1 = x[2 * t + 1], a8 = x[2 * t + 8], a9 = x[2 * t + 9];
+          st[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a8, a8, a9 * a9)));
+        }
         L0.ssa[(size_t)b * p.n_parts + kb] = (st[0] + st[1]) + (st[2] + st[3]);
         float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H + 16 * kb);
 #pragma unroll
@@ -2295,6 +2542,91 @@ __device__ __noinline__ void argmax_task(const Params &p, int32_t *tok_out) {
 }
 
 // ---------------------------------------------------------------------------
+// Dispatch mode: a scheduler CTA beside the workers ("Mirage Persistent
+// Kernel (MPK)" page, section 5.1: scheduler CTAs hand tasks to the workers).
+// One warp polls the events in a window of 32 from the lowest one not yet
+// handled; when an event has collected its triggers for this step, its
+// dependents [first, last] (a contiguous range of the linearised graph) are
+// dealt round-robin to the workers' queues; the tasks without a dependency
+// (the linear order's prefix) go out first, and every queue ends with -1.
+// The workers run their queue in order without waiting on events.  Every
+// wait is bounded; on a timeout or an abort the queues are closed at once.
+// ---------------------------------------------------------------------------
+__device__ void scheduler_loop(const Params &p, const Smem &sm) {
+  const int lane = threadIdx.x & 31;
+  const int W = p.n_workers;
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(sm.ring);       // [W] entries per queue
+  uint32_t *done = cnt + ((W + 31) & ~31);                      // [n_events / 32] handled
+  const int nw32 = (p.n_events + 31) >> 5;
+  for (int i = lane; i < W; i += 32) cnt[i] = 0u;
+  for (int i = lane; i < nw32; i += 32) done[i] = 0u;
+  __syncwarp();
+  const uint32_t epoch = *(volatile uint32_t *)p.epoch + 1u;
+  int rr = 0;  // round-robin cursor over the workers
+  // deal tasks [t0, t1) to the queues: task t0 + i to worker (rr + i) % W
+  auto deal = [&](int t0, int t1) {
+    const int m = t1 - t0;
+    for (int i = lane; i < m; i += 32) {
+      const int g = rr + i, w = g % W;
+      const int g1 = rr + ((w - rr % W) % W + W) % W;  // first slot of this deal for worker w
+      const uint32_t pos = cnt[w] + (uint32_t)((g - g1) / W);
+      if (pos < (uint32_t)p.q_cap - 1u) p.q_list[(size_t)w * p.q_cap + pos] = t0 + i;
+    }
+    __threadfence();
+    __syncwarp();
+    for (int w = lane; w < W; w += 32) {
+      // entries of this deal for worker w
+      const int first = ((w - rr % W) % W + W) % W;
+      const int k = m > first ? (m - first + W - 1) / W : 0;
+      if (k > 0) {
+        cnt[w] += (uint32_t)k;
+        st_release(p.q_tail + w, cnt[w]);
+      }
+    }
+    __syncwarp();
+    rr = (rr + m) % W;
+  };
+  // the roots: the prefix of the linear order without a dependency event
+  int n_roots = 0;
+  while (n_roots < p.n_tasks && p.tasks[n_roots].dep < 0) ++n_roots;
+  deal(0, n_roots);
+  int head = 0;  // lowest event not yet handled
+  const uint64_t t0 = global_timer();
+  uint32_t spins = 0;
+  while (head < p.n_events) {
+    const int e = head + lane;
+    bool ready = false;
+    if (e < p.n_events && !((done[e >> 5] >> (e & 31)) & 1u)) {
+      const uint32_t target = p.events[e].count * epoch;
+      ready = (int32_t)(ld_acquire(p.counters + e) - target) >= 0;
+    }
+    uint32_t mask = __ballot_sync(0xffffffffu, ready);
+    while (mask) {  // in event order
+      const int b = __ffs(mask) - 1;
+      mask &= mask - 1u;
+      const int ev = head + b;
+      deal(p.events[ev].first, p.events[ev].last + 1);
+      if (lane == 0) done[ev >> 5] |= 1u << (ev & 31);
+      __syncwarp();
+    }
+    while (head < p.n_events && ((done[head >> 5] >> (head & 31)) & 1u)) ++head;
+    if (*(volatile int32_t *)p.status != 0) break;
+    if (++spins > 16) __nanosleep(64);
+    if ((spins & 63u) == 0 && global_timer() - t0 > 4ull * p.timeout_ns + 1000000000ull) {
+      if (lane == 0) record_error(p, kDevTimeout, -1, head);
+      break;
+    }
+  }
+  // close every queue (an abort closes them where they stand)
+  for (int w = lane; w < W; w += 32) {
+    const uint32_t pos = cnt[w] < (uint32_t)p.q_cap ? cnt[w] : (uint32_t)p.q_cap - 1u;
+    p.q_list[(size_t)w * p.q_cap + pos] = -1;
+    __threadfence();
+    st_release(p.q_tail + w, pos + 1u);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // The worker kernel
 // ---------------------------------------------------------------------------
 // kMma: projections on tensor cores (batch >= 2) instead of the CUDA-core
@@ -2309,7 +2641,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
   const int warp = tid >> 5;
 
   Queue q;
-  if (p.persistent) {
+  if (p.dispatch) {
+    if ((int)blockIdx.x == p.n_workers) {  // the scheduler CTA
+      if (tid < 32) scheduler_loop(p, sm);
+      return;
+    }
+    q.first = 0;
+    q.stride = 0;
+    q.count = p.q_cap;
+    q.list = p.q_list + (size_t)blockIdx.x * p.q_cap;
+    q.tail = p.q_tail + blockIdx.x;
+  } else if (p.persistent) {
     q.first = blockIdx.x;
     q.stride = gridDim.x;
     q.count = q.first < p.n_tasks ? (p.n_tasks - q.first + q.stride - 1) / q.stride : 0;
@@ -2324,7 +2666,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     for (int s = 0; s < p.ring_stages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kComputeWarps);
+      mbar_init(&sm.abar[s], 1);
     }
+    mbar_init(sm.mdone, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     int bad = 0;
     if (*(volatile int32_t *)p.status != 0) bad = 1;  // an earlier step failed: no-op
@@ -2359,6 +2703,20 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     }
   }
   if (sm.ctl[kAbort]) return;  // nothing issued yet
+  if (kMma) {
+    // the tensor-core projections' accumulators: one allocation per CTA (one
+    // CTA per SM), released on every path below
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(sm.tmem)),
+                   "n"(kUmmaTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
 
   if (warp == kComputeWarps) {
     if ((tid & 31) == 0) producer_loop<kMma>(p, sm, q);
@@ -2366,12 +2724,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
   } else {
     const uint32_t epoch0 = (uint32_t)sm.ctl[kEpoch];  // step 0's epoch
     uint32_t k = 0;
+    UmmaState us;
     bool run = true;
     for (int s = 0; s < p.n_steps && run; ++s) {
     const uint32_t epoch = epoch0 + (uint32_t)s;
     if (tid == 0) sm.ctl[kLogits] = s == p.n_steps - 1;  // seen after the next barrier
     for (int n = 0; n < q.count; ++n) {
-      const int id = q.first + n * q.stride;
+      const int id = queue_task(p, sm, q, n);
+      if (id < 0) break;
       const DevTask t = p.tasks[id];
       uint64_t t_wait = 0;
       if (p.trace && tid == 0) {
@@ -2395,7 +2755,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           break;
         case 2: case 5: case 6: case 7: case 8: {
           if constexpr (kMma) {
-            ok = mma_task<kNN == 2 ? 2 : 1>(p, sm, t, k, id, dw);
+            ok = umma_task<kNN == 2 ? 2 : 1>(p, sm, t, k, us, id, dw);
           } else {
             const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
             const int nch = K >> 3;
@@ -2452,57 +2812,97 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       }
     }
     }
-    if (tid == 0) sm.ctl[kConsumed] = (int)k;
-  }
-  __syncthreads();
-  if (sm.ctl[kAbort] && warp == kComputeWarps && (tid & 31) == 0) {
-    // wait for every copy issued but not consumed before the CTA exits
-    const uint32_t from = (uint32_t)sm.ctl[kConsumed], to = (uint32_t)sm.ctl[kIssued];
-    for (uint32_t kk = from; kk < to; ++kk) {
-      const int slot = (int)(kk % p.ring_stages);
-      const uint32_t par = (kk / p.ring_stages) & 1u;
-      const uint64_t t0 = global_timer();
-      while (!mbar_test(&sm.full[slot], par)) {
-        if (global_timer() - t0 > 1000000000ull) break;
+    if (tid == 0) {
+      sm.ctl[kConsumed] = (int)k;
+      // operand copies still in flight after an abort land before the CTA exits
+      for (int slot = 0; slot < p.ring_stages; ++slot) {
+        if (!((us.apend >> slot) & 1u)) continue;
+        const uint64_t t0 = global_timer();
+        while (!mbar_test(&sm.abar[slot], (us.aph >> slot) & 1u)) {
+          if (global_timer() - t0 > 4ull * p.timeout_ns + 1000000000ull) break;
+        }
       }
     }
   }
+  __syncthreads();
+  if (sm.ctl[kAbort] && warp == kComputeWarps && (tid & 31) == 0) {
+    // Copies into this CTA's shared memory must land before it exits.  Only
+    // the last ring_stages issued stages can still be in flight (each is the
+    // latest use of its slot, so its phase parity is unambiguous).  The wait
+    // has the kernel's timeout budget; if it runs out, the status words' event
+    // field is set to -2 to say that the CTA exited with copies outstanding.
+    const uint32_t to = (uint32_t)sm.ctl[kIssued];
+    const uint32_t from = to > (uint32_t)p.ring_stages ? to - (uint32_t)p.ring_stages : 0u;
+    const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
+    const uint64_t t0 = global_timer();
+    bool late = false;
+    for (uint32_t kk = from; kk < to && !late; ++kk) {
+      const int slot = (int)(kk % p.ring_stages);
+      const uint32_t par = (kk / p.ring_stages) & 1u;
+      while (!mbar_test(&sm.full[slot], par)) {
+        if (global_timer() - t0 > budget) {
+          late = true;
+          break;
+        }
+      }
+    }
+    if (late) {
+      p.status[2] = -2;
+      __threadfence();
+    }
+  }
+  if (kMma) {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*sm.tmem),
+                   "n"(kUmmaTmemCols)
+                   : "memory");
+  }
 }
 
-// Weight layout for the tensor-core path: a row-major [rows][K] bf16 matrix
-// to mma.sync A-fragment order.  Item (m-tile mt, k-block kb, lane) holds the
-// lane's 8 elements, so stage copies and fragment loads are 16 bytes per lane.
-// Rows >= rows (the last m-tile's padding) are zero.
-__global__ void frag_permute_kernel(uint4 *dst, const uint32_t *src, int rows, int K,
-                                    long long n_items) {
+// Weight layout for the tensor-core projections: rows [row_base, row_base +
+// n) of a row-major [rows][K] bf16 matrix (src holds those n rows) to the
+// order umma_tile streams.  Row r belongs to task t = r / task_rows and to
+// pass q = (r % task_rows) / kUmmaMaxN of it; a pass's N rows (the last task
+// is padded to rows_p, a multiple of 16) are contiguous from row
+// t * task_rows + q * kUmmaMaxN on, and per 16-column k-block hold their
+// N x 16 elements in core-matrix order (N * 32 bytes).  One item per 16 bytes
+// (8 elements of a row); padding rows (r >= rows) are zero.
+__global__ void umma_permute_kernel(uint4 *dst, const uint4 *src, int row_base, int rows,
+                                    int rows_p, int K, int task_rows, long long n_items) {
   const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (item >= n_items) return;
-  const int lane = (int)(item & 31);
-  const long long blk = item >> 5;
-  const int KB = K >> 4;
-  const int mt = (int)(blk / KB), kb = (int)(blk - (long long)mt * KB);
-  const int r0 = mt * 16 + (lane >> 2), r1 = r0 + 8;
-  const int c = kb * 16 + 2 * (lane & 3);  // even: one 32-bit word holds (c, c + 1)
-  const size_t w = (size_t)K / 2;
-  uint4 o;
-  o.x = r0 < rows ? src[(size_t)r0 * w + c / 2] : 0u;
-  o.y = r1 < rows ? src[(size_t)r1 * w + c / 2] : 0u;
-  o.z = r0 < rows ? src[(size_t)r0 * w + c / 2 + 4] : 0u;
-  o.w = r1 < rows ? src[(size_t)r1 * w + c / 2 + 4] : 0u;
-  dst[item] = o;
+  const int cpr = K >> 3;  // 16-byte units per row
+  const int rl = (int)(item / cpr), c = (int)(item - (long long)rl * cpr);
+  const int r = row_base + rl;
+  const int t = r / task_rows, rr = r - t * task_rows;
+  const int q = rr / kUmmaMaxN, i = rr - q * kUmmaMaxN;
+  const int trows = min(task_rows, rows_p - t * task_rows);
+  const int N = min(kUmmaMaxN, trows - q * kUmmaMaxN);
+  const int r0 = t * task_rows + q * kUmmaMaxN;  // first row of the pass
+  const int j = c >> 1, kh = c & 1;
+  const size_t o = (size_t)r0 * cpr + (size_t)j * N * 2 + (size_t)(i >> 3) * 16 + kh * 8 + (i & 7);
+  dst[o] = r < rows ? src[(size_t)rl * cpr + c] : make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace
 
-// dst receives ceil(rows / 16) m-tiles of K / 16 fragment blocks (512 bytes each).
-cudaError_t permute_to_fragments(void *dst, const void *src, int rows, int K,
-                                 cudaStream_t stream) {
-  const long long n_items = (long long)((rows + 15) / 16) * (K / 16) * 32;
-  if (n_items == 0) return cudaSuccess;
+// dst: the whole matrix in the tensor-core layout (rows_p rows); src: its rows
+// [row_base, row_base + n) row-major.  row_base must be a multiple of
+// task_rows; with row_base + n == rows the padding rows up to rows_p are
+// written too.
+cudaError_t permute_to_umma(void *dst, const void *src, int row_base, int n, int rows, int rows_p,
+                            int K, int task_rows, cudaStream_t stream) {
+  const int n_out = row_base + n >= rows ? rows_p - row_base : n;
+  const long long n_items = (long long)n_out * (K / 8);
+  if (n_items <= 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n_items + threads - 1) / threads;
-  frag_permute_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-      static_cast<uint4 *>(dst), static_cast<const uint32_t *>(src), rows, K, n_items);
+  umma_permute_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), row_base, rows, rows_p, K,
+      task_rows, n_items);
   return cudaGetLastError();
 }
 

@@ -94,12 +94,22 @@ std::string lower(const ModelShape &m, const GraphTuning &t, Lowering *L) {
   T.n_gu = (int)cdiv(m.ffn, T.gu_rows);
   T.n_down = (int)cdiv(m.hidden, T.down_rows);
   T.n_lm = (int)cdiv(m.vocab, T.lm_rows);
-  // splits per (sequence, kv head): at most attn_tasks_per_worker tasks per worker
-  long target = std::max(1L, (long)t.attn_tasks_per_worker * W / ((long)m.batch * m.n_kv_heads));
-  long chunk = cdiv(cdiv(m.kv_capacity, target), 64) * 64;
-  if (chunk < t.attn_min_chunk) chunk = t.attn_min_chunk;
-  T.attn_chunk = (int)chunk;
-  T.attn_splits = (int)cdiv(m.kv_capacity, chunk);
+  const long pairs = (long)m.batch * m.n_kv_heads;
+  if (t.attn_jit) {
+    // JIT: apw * W tasks; each (sequence, kv head) is cut by at most
+    // ceil(apw * W / pairs) + 2 of them (the run-time chunk is chosen so)
+    T.n_attn = std::max(1, t.attn_tasks_per_worker * W);
+    T.attn_splits = (int)(cdiv(T.n_attn, pairs) + 2);
+    T.attn_chunk = 0;
+  } else {
+    // splits per (sequence, kv head): at most attn_tasks_per_worker tasks per worker
+    long target = std::max(1L, (long)t.attn_tasks_per_worker * W / pairs);
+    long chunk = cdiv(cdiv(m.kv_capacity, target), 64) * 64;
+    if (chunk < t.attn_min_chunk) chunk = t.attn_min_chunk;
+    T.attn_chunk = (int)chunk;
+    T.attn_splits = (int)cdiv(m.kv_capacity, chunk);
+    T.n_attn = (int)(pairs * T.attn_splits);
+  }
   const int S = T.attn_splits;
 
   // Buffers: 0 tokens, 1 kv_len, 2 lm partials, then per layer boundary x_l
@@ -135,7 +145,18 @@ std::string lower(const ModelShape &m, const GraphTuning &t, Lowering *L) {
       acc(id, lbuf(l, 0), 0, B, j * T.qkv_rows, std::min(n_qkv, (j + 1) * T.qkv_rows), true);
     }
     new_op();
-    for (int b = 0; b < B; ++b)
+    if (t.attn_jit) {
+      // a JIT task may cover any (sequence, kv head): it reads every group's
+      // q, k, v and the KV lengths, and may write every partial and head
+      for (int a = 0; a < T.n_attn; ++a) {
+        int id = task(kAttn, l, a);
+        acc(id, lbuf(l, 0), 0, B, 0, n_qkv, false);
+        acc(id, kKvLen, 0, B, 0, 1, false);
+        acc(id, lbuf(l, 1), 0, B, 0, m.n_kv_heads * S, true);
+        acc(id, lbuf(l, 2), 0, B, 0, qdim, true);
+      }
+    }
+    for (int b = 0; b < B && !t.attn_jit; ++b)
       for (int g = 0; g < m.n_kv_heads; ++g)
         for (int s = 0; s < S; ++s) {
           int id = task(kAttn, l, (b * m.n_kv_heads + g) * S + s);

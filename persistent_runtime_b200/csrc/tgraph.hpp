@@ -29,13 +29,18 @@ struct GraphTuning {
   int col_align = 16;
   int attn_tasks_per_worker = 4;
   int attn_min_chunk = 64;
+  // 1: attention tasks are resolved at run time (JIT): apw * W tasks per
+  // layer, each reading every kv group and writing every head, whose position
+  // ranges come from the live KV lengths of the step
+  int attn_jit = 0;
 };
 
 // Rows per task chosen by the tiling rules.
 struct Tiling {
   int qkv_rows = 0, o_rows = 0, gu_rows = 0, down_rows = 0, lm_rows = 0;
-  int attn_splits = 0, attn_chunk = 0;
+  int attn_splits = 0, attn_chunk = 0;  // JIT: partial slots per (sequence, kv head), 0
   int n_qkv = 0, n_o = 0, n_gu = 0, n_down = 0, n_lm = 0;
+  int n_attn = 0;  // attention tasks per layer
 };
 
 // The finished graph: tasks in linear order, events by id.

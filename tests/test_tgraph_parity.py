@@ -22,16 +22,24 @@ def default_col_align(w):
     return 4 if w.batch == 1 else 16
 
 
+def default_jit(w):
+    # the library resolves attention at run time (JIT) from batch 2 on by default
+    return int(w.batch > 1)
+
+
 @pytest.mark.parametrize("w,W", CONFIGS, ids=[f"{w.name}-W{W}" for w, W in CONFIGS])
-@pytest.mark.parametrize("align", [16, None], ids=["align16", "default"])
+@pytest.mark.parametrize("align", [16, None, "aot"], ids=["align16", "default", "aot"])
 def test_decode_graph_bit_exact_with_oracle(w, W, align):
     cap = w.kv_capacity(0)
     if align is None:  # the library's defaults against the oracle with the same values
         mine = prb.plan_graph(w, cap, W)
-        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w), 1)
+        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w), 1, 64, default_jit(w))
+    elif align == "aot":  # attention splits fixed at build time at every batch size
+        mine = prb.plan_graph(w, cap, W, attn_jit=-1)
+        ref = oracle.tgraph_decode(w, cap, W, default_col_align(w), 1, 64, 0)
     else:
         mine = prb.plan_graph(w, cap, W, col_align=align, attn_tasks_per_worker=4)
-        ref = oracle.tgraph_decode(w, cap, W, align, 4)
+        ref = oracle.tgraph_decode(w, cap, W, align, 4, 64, default_jit(w))
     gc.assert_graphs_equal(mine, ref)
     np.testing.assert_array_equal(mine.edge_src, ref.edge_src)
     np.testing.assert_array_equal(mine.edge_dst, ref.edge_dst)
@@ -44,10 +52,11 @@ def test_decode_graph_bit_exact_with_oracle(w, W, align):
 def test_tuning_variants_bit_exact(col_align, apw, min_chunk):
     w = synth.Q8B_B8
     cap = w.kv_capacity(3)
-    mine = prb.plan_graph(w, cap, 148, col_align=col_align, attn_tasks_per_worker=apw,
-                          attn_min_chunk=min_chunk)
-    ref = oracle.tgraph_decode(w, cap, 148, col_align, apw, min_chunk)
-    gc.assert_graphs_equal(mine, ref)
+    for jit in (-1, 1):
+        mine = prb.plan_graph(w, cap, 148, col_align=col_align, attn_tasks_per_worker=apw,
+                              attn_min_chunk=min_chunk, attn_jit=jit)
+        ref = oracle.tgraph_decode(w, cap, 148, col_align, apw, min_chunk, int(jit > 0))
+        gc.assert_graphs_equal(mine, ref)
 
 
 @pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt"])
