@@ -94,12 +94,11 @@ typedef struct {
   int attn_min_chunk;        /* smallest KV positions per attention task (64) */
   int ring_stages;           /* shared-memory weight ring depth (4) */
   int ring_stage_bytes;      /* bytes per ring stage, multiple of 1024 (49152) */
-  int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while a
-                                landed stage stays unreleased for over 1.5 us (the compute
-                                warps wait on an event or run attention); default 524288 at
-                                batch 1 (single-step launches; mk_decode_steps* with more than
-                                one step run without it unless it is set), off at batch >= 2;
-                                negative = off */
+  int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while
+                                the compute warps wait for an O projection's event (the
+                                step's attention window, when HBM is otherwise idle);
+                                default 524288 at batch 1, off at batch >= 2 (attention
+                                streams the caches there); negative = off */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
   int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the
                                 paged pools (a multiple of 64), see mk_decode_steps_paged */
@@ -111,9 +110,9 @@ typedef struct {
                                 data-dependent operators JIT, the rest ahead of time):
                                 attn_tasks_per_worker * W tasks per layer cut the live
                                 positions of all (sequence, kv head) pairs into equal
-                                chunks, which may cross pairs.  0 = default (on for batch
-                                >= 2), 1 = on (batch >= 2 only), -1 = off: splits fixed
-                                at build time from kv_capacity */
+                                chunks, which may cross pairs.  0 = off (default): splits
+                                fixed at build time from kv_capacity; 1 = on (batch >= 2
+                                only; MK_ERR_ARG at batch 1) */
   int dispatch;              /* 0 = static queues: worker w runs tasks w, w + W, ... and waits
                                 on their events itself (default); 1 = a scheduler CTA in the
                                 same launch hands ready tasks to the workers (the pages'

@@ -51,10 +51,11 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   if (d.ring_stages <= 0) d.ring_stages = 4;
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
-  // batch 1: while the compute warps hold the ring (attention, event waits),
-  // the producer prefetches up to 512 KB of the following stages into L2
-  // (Qwen3-8B bs1: 3125 -> 3092 us per step); the batched kernel is not
-  // helped by it.  Negative: off.
+  // batch 1: while the compute warps wait for an O projection's event (the
+  // attention window), the producer prefetches up to 512 KB of its following
+  // stages into L2 (Qwen3-8B bs1, one box: 3079 us per step against 3095 us
+  // for 256 KB); at batch >= 2 attention streams the caches in that window.
+  // Negative: off.
   if (d.l2_prefetch_bytes == 0) d.l2_prefetch_bytes = batch > 1 ? 0 : 512 * 1024;
   if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
   return d;
@@ -85,29 +86,22 @@ std::string check_gpu_shape(const mk_model_config &c) {
 }
 
 // Tensor-core tiling of the batched projections (QKV, O, GATE_UP, DOWN,
-// LM_HEAD, in that order), as the worker derives it: a task's rows run in
-// passes of up to kUmmaMaxN rows (mb = 16-row m-tiles of a full pass), and a
-// pass streams ring stages of kcb 16-column k-blocks, as many as the stage's
-// weights (N * 32 bytes per k-block), its operand chunk (512 nn bytes per
-// k-block) and kUmmaSlack fit in one ring stage (at most the K / 16 k-blocks
-// of the operator; 0 when not even one fits).
+// LM_HEAD, in that order).  m-tiles per row block: the task's rows up to the
+// accumulator limit; k-blocks per ring stage: what a stage holds for that
+// many m-tiles, a multiple of 8 (one share per warp), at most
+// mma_max_kpw(nn) per warp (the B-fragment registers of one stage).
 struct MmaTiling {
   int mb[5], kcb[5];
 };
 
-int umma_nkb(int ring_stage_bytes, int N, int nn, int KB) {
-  const int n = (ring_stage_bytes - mk::kUmmaSlack) / (N * 32 + 512 * nn);
-  return std::min(KB, std::max(n, 0));
-}
-
-MmaTiling mma_tiling(const mk::Tiling &T, const mk_model_config &c, int ring_stage_bytes, int nn) {
+MmaTiling mma_tiling(const mk::Tiling &T, int ring_stage_bytes, int nn) {
+  const int units = ring_stage_bytes / 512;
+  auto mb_of = [&](int task_rows) { return std::max(1, std::min(mk::kMmaMaxMB, task_rows / 16)); };
   const int rows[5] = {T.qkv_rows, T.o_rows, 2 * T.gu_rows, T.down_rows, T.lm_rows};
-  const int K[5] = {c.hidden, c.n_q_heads * c.head_dim, c.hidden, c.ffn, c.hidden};
   MmaTiling m{};
   for (int i = 0; i < 5; ++i) {
-    const int N = std::min(mk::kUmmaMaxN, (rows[i] + 15) / 16 * 16);
-    m.mb[i] = N / 16;
-    m.kcb[i] = umma_nkb(ring_stage_bytes, N, nn, K[i] / 16);
+    m.mb[i] = mb_of(rows[i]);
+    m.kcb[i] = std::min(8 * mk::mma_max_kpw(nn), units / m.mb[i] / 8 * 8);
   }
   return m;
 }
@@ -117,10 +111,13 @@ mk::ModelShape shape_of(const mk_model_config &c) {
                         c.ffn,      c.vocab,  c.batch,     c.kv_capacity};
 }
 
-// JIT attention: on by default from batch 2 (the batch-1 kernel's attention
-// keeps its splits fixed at build time, see mk_build_graph).
+// JIT attention: opt-in from batch 2 (the batch-1 kernel's attention keeps
+// its splits fixed at build time, see mk_build_graph).  Measured on Qwen3-8B
+// (one box): bs8 4413 us per step with it, 4324 us without; bs16 10904 vs
+// 8549 us -- the cache stream is bound near 5.7 TB/s either way, so spreading
+// it over all SMs gains nothing, and every pair then needs a merge.
 bool jit_attention(const mk_model_config &c, const mk_tuning &t) {
-  return t.attn_jit == 0 ? c.batch > 1 : t.attn_jit > 0;
+  return c.batch > 1 && t.attn_jit > 0;
 }
 
 mk_status plan(const mk_model_config *cfg, const mk_tuning &t, int workers, mk_handle *h) {
@@ -153,7 +150,6 @@ mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int
   if (!h) return fail(nullptr, MK_ERR_OOM, "out of host memory");
   h->cfg = *cfg;
   h->tune = fill_defaults(tuning, cfg->batch);
-  h->prefetch_defaulted = !tuning || tuning->l2_prefetch_bytes == 0;
   h->tune.num_workers = num_workers;
   mk_status s = plan(cfg, h->tune, num_workers, h);
   if (s != MK_OK) {
@@ -206,7 +202,6 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
   h->device = device;
   h->cfg = *cfg;
   h->tune = fill_defaults(tuning, cfg->batch);
-  h->prefetch_defaulted = !tuning || tuning->l2_prefetch_bytes == 0;
   mk_tuning &t = h->tune;
   const mk_model_config &c = *cfg;
   const int D = c.head_dim;
@@ -475,13 +470,23 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     return fail(nullptr, MK_ERR_ARG, "ring stage smaller than 8 K/V rows");
   }
   if (mma) {
-    const MmaTiling mt = mma_tiling(T, c, t.ring_stage_bytes, nn);
+    const MmaTiling mt = mma_tiling(T, t.ring_stage_bytes, nn);
     p.mma = 1;
     p.nn = nn;
     p.n_parts = n_parts;
+    p.mb_qkv = mt.mb[0];
+    p.mb_o = mt.mb[1];
+    p.mb_gu = mt.mb[2];
+    p.mb_down = mt.mb[3];
+    p.mb_lm = mt.mb[4];
+    p.kcb_qkv = mt.kcb[0];
+    p.kcb_o = mt.kcb[1];
+    p.kcb_gu = mt.kcb[2];
+    p.kcb_down = mt.kcb[3];
+    p.kcb_lm = mt.kcb[4];
     p.xfb = reinterpret_cast<uint16_t *>(base + o_xa[Ly]);
     p.ssf = reinterpret_cast<float *>(base + o_ssa[Ly]);
-    if (std::min({mt.kcb[0], mt.kcb[1], mt.kcb[2], mt.kcb[3], mt.kcb[4]}) < 1) {
+    if (std::min({p.kcb_qkv, p.kcb_o, p.kcb_gu, p.kcb_down, p.kcb_lm}) < 8) {
       mk_destroy(h);
       return fail(nullptr, MK_ERR_ARG, "ring stage too small for the tensor-core tiles");
     }
@@ -527,9 +532,9 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     o_gu[l] = take((size_t)2 * F * H);
     o_dn[l] = take((size_t)H * F);
   }
-  // batch >= 2: projection matrices in the tensor-core order of their tasks,
-  // the LM head padded to whole 16-row m-tiles and kept apart from the
-  // (row-major) embedding table even when the two are tied
+  // batch >= 2: projection matrices in mma.sync fragment order, the LM head
+  // padded to whole 16-row m-tiles and kept apart from the (row-major)
+  // embedding table even when the two are tied
   const bool mma = h->base.mma != 0;
   const size_t Vp = mma ? ((size_t)V + 15) / 16 * 16 : (size_t)V;
   const bool lm_shares_embed = c.tied_embeddings && !mma;
@@ -587,35 +592,32 @@ mk_status mk_load_weights(mk_handle *h, const mk_weights *w, void *stream) {
     if (!c.tied_embeddings) cp(o_lm, w->lm_head, (size_t)V * H * 2);
   } else {
     // each matrix goes row-major into a staging buffer, then a kernel writes
-    // it to the arena in the tensor-core order of its tasks; the LM head goes
-    // in row slabs of whole tasks
-    const mk::Tiling &Tl = h->graph.tiling;
+    // it to the arena in fragment order; the LM head goes in row slabs
     const size_t tmp_bytes =
         2 * std::max({n_qkv * H, (size_t)H * qd, (size_t)2 * F * H, (size_t)H * F});
     void *tmp = nullptr;
     if (cudaMalloc(&tmp, tmp_bytes) != cudaSuccess)
       return fail(h, MK_ERR_OOM, "cudaMalloc of the weight staging buffer failed");
     char *T = static_cast<char *>(tmp);
-    auto perm = [&](size_t dst_off, int row_base, int n, int rows, int rows_p, int K, int task_rows) {
-      if (e == cudaSuccess)
-        e = mk::permute_to_umma(A + dst_off, T, row_base, n, rows, rows_p, K, task_rows, st);
+    auto frag = [&](size_t dst_off, int rows, int K) {
+      if (e == cudaSuccess) e = mk::permute_to_fragments(A + dst_off, T, rows, K, st);
     };
     for (int l = 0; l < Ly; ++l) {
       put_qkv(T, l);
-      perm(o_qkv[l], 0, (int)n_qkv, (int)n_qkv, (int)n_qkv, H, Tl.qkv_rows);
+      frag(o_qkv[l], (int)n_qkv, H);
       cpy(T, w->wo[l], (size_t)H * qd * 2);
-      perm(o_o[l], 0, H, H, H, (int)qd, Tl.o_rows);
+      frag(o_o[l], H, (int)qd);
       put_gu(T, l);
-      perm(o_gu[l], 0, 2 * F, 2 * F, 2 * F, H, 2 * Tl.gu_rows);
+      frag(o_gu[l], 2 * F, H);
       cpy(T, w->w_down[l], (size_t)H * F * 2);
-      perm(o_dn[l], 0, H, H, H, F, Tl.down_rows);
+      frag(o_dn[l], H, F);
     }
-    const int slab =
-        std::max(1, (int)std::min<size_t>((size_t)V, tmp_bytes / row) / Tl.lm_rows) * Tl.lm_rows;
+    const int slab = (int)std::min<size_t>((size_t)V, tmp_bytes / row / 16 * 16);
     for (int r0 = 0; r0 < V; r0 += slab) {
       const int n = std::min(slab, V - r0);
       cpy(T, static_cast<const char *>(lm_src) + (size_t)r0 * row, (size_t)n * row);
-      perm(o_lm, r0, n, V, (int)Vp, H, Tl.lm_rows);
+      // m-tile r0 / 16 of the padded head: 512-byte blocks, H / 16 per m-tile
+      frag(o_lm + (size_t)(r0 / 16) * (H / 16) * 512, n, H);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // the staging buffer is freed next
     cudaFree(tmp);
@@ -755,15 +757,6 @@ mk_status mk_decode_step(mk_handle *h, const int32_t *d_tokens_in, int32_t *d_to
   return MK_OK;
 }
 
-// Multi-step launches run without the default idle-window L2 prefetch: the
-// step boundary inside one launch is a long idle window, and prefetching
-// through it cost more than it gave (Qwen3-8B bs1, one box: 3154 us per step
-// with it, 3117 us without; single launches 3097 us with it, 3124 without).
-// An explicit l2_prefetch_bytes is kept.
-static void multi_step_prefetch(const mk_handle *h, int n_steps, Params *p) {
-  if (n_steps > 1 && h->prefetch_defaulted) p->l2_prefetch_bytes = 0;
-}
-
 mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
                           int32_t *d_tokens_out, int32_t *d_kv_len, void *d_k_cache,
                           void *d_v_cache, float *d_logits, void *stream) {
@@ -779,7 +772,6 @@ mk_status mk_decode_steps(mk_handle *h, int n_steps, const int32_t *d_tokens_in,
   p.logits = d_logits;
   p.persistent = 1;
   p.n_steps = n_steps;
-  multi_step_prefetch(h, n_steps, &p);
   cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
@@ -800,7 +792,6 @@ mk_status mk_decode_steps_paged(mk_handle *h, int n_steps, const int32_t *d_toke
   p.logits = d_logits;
   p.persistent = 1;
   p.n_steps = n_steps;
-  multi_step_prefetch(h, n_steps, &p);
   cudaError_t e = mk::launch_persistent(p, h->tune.num_workers, h->smem,
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "persistent launch");
@@ -891,7 +882,7 @@ mk_status mk_graph_export(const mk_handle *h, mk_graph_view *out) {
   out->attn_splits = T.attn_splits;
   out->attn_chunk = T.attn_chunk;
   if (h->cfg.batch > 1 && T.qkv_rows > 0) {
-    const MmaTiling mt = mma_tiling(T, h->cfg, h->tune.ring_stage_bytes, (h->cfg.batch + 7) / 8);
+    const MmaTiling mt = mma_tiling(T, h->tune.ring_stage_bytes, (h->cfg.batch + 7) / 8);
     for (int i = 0; i < 5; ++i) {
       out->mma_mb[i] = mt.mb[i];
       out->mma_kcb[i] = mt.kcb[i];

@@ -17,8 +17,8 @@ cudaError_t worker_configure(size_t smem);
 cudaError_t worker_max_blocks(int *blocks, size_t smem);
 cudaError_t launch_persistent(const Params &p, int workers, size_t smem, cudaStream_t stream);
 cudaError_t launch_tasks(const Params &p, int n_ctas, size_t smem, cudaStream_t stream);
-cudaError_t permute_to_umma(void *dst, const void *src, int row_base, int n, int rows, int rows_p,
-                            int K, int task_rows, cudaStream_t stream);
+cudaError_t permute_to_fragments(void *dst, const void *src, int rows, int K,
+                                 cudaStream_t stream);
 }  // namespace mk
 
 struct mk_handle;
@@ -32,7 +32,6 @@ std::string encode_kv_maps(const mk_handle *h, const void *k_cache, const void *
 struct mk_handle {
   mk_model_config cfg{};
   mk_tuning tune{};
-  bool prefetch_defaulted = false;  // l2_prefetch_bytes was left to its default
   mk::TaskGraph graph;
   bool host_only = true;
   int device = -1;

@@ -216,12 +216,14 @@ __device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp-level tensor cores (batched attention): mma.sync.m16n8k16, A 16 x 16
-// row major, B 16 x 8, fp32 accumulators.  Fragment ownership (PTX ISA,
-// "Matrix Fragments for mma.m16n8k16"), lane l, g = l / 4, t = l % 4:  A regs
-// {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..), (g+8, 2t+8..)};  B regs
-// {(2t..2t+1, g), (2t+8..2t+9, g)};  C {(g, 2t), (g, 2t+1), (g+8, 2t),
-// (g+8, 2t+1)}.
+// Tensor cores (batch >= 2): mma.sync.m16n8k16, A = weights (16 rows x 16 k,
+// row major), B = activations (16 k x 8 sequences), fp32 accumulators.
+// Fragment ownership (PTX ISA, "Matrix Fragments for mma.m16n8k16"), lane l,
+// g = l / 4, t = l % 4:  A regs {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..),
+// (g+8, 2t+8..)};  B regs {(2t..2t+1, g), (2t+8..2t+9, g)};  C {(g, 2t),
+// (g, 2t+1), (g+8, 2t), (g+8, 2t+1)}.  Weights and activations are stored in
+// exactly this order, so each lane fetches its fragment with one 16-byte
+// (A) or 8-byte (B) load.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4 &a, const uint2 &b) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
@@ -254,111 +256,151 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
-// ---------------------------------------------------------------------------
-// 5th-generation tensor cores (batched projections): tcgen05.mma kind::f16,
-// one thread issues, fp32 accumulators live in tensor memory (TMEM).  Both
-// operands are K-major in shared memory without swizzle: core matrices of 8
-// rows x 8 bf16 (16 bytes per row, 128 bytes each); within one 16-column
-// k-block the two 8-column halves of a row group are 128 bytes apart and the
-// 8-row groups 256 bytes apart.  Element (row, k) of a k-block therefore sits
-// at (row / 8) * 256 + (k / 8) * 128 + (row % 8) * 16 + (k % 8) * 2.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)(128u >> 4) << 16;  // stride between the two k halves
-  d |= (uint64_t)(256u >> 4) << 32;  // stride between 8-row groups
-  d |= 1ull << 46;                   // descriptor version of sm_100
-  return d;                          // base offset 0, no swizzle
-}
-
-// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N rows.
-__device__ __forceinline__ uint32_t umma_idesc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The mbarrier receives one arrival once every earlier tcgen05 operation of
-// this thread has completed.
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-
-// Lanes 32 (warp % 4) .. + 31 of TMEM, 32 columns from taddr: thread t of the
-// warp receives lane base + t.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_n(uint64_t *bar, uint32_t n) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n)
-               : "memory");
-}
-
 // Activation operands are two-term bf16 expansions x = hi + lo, hi = bf16(x),
-// lo = bf16(x - hi): about 16 significant bits, so W x = W hi + W lo (two
-// operand rows, summed in the epilogue) keeps the projection inputs close to
-// fp32 while the weights stay exactly bf16.  A single bf16 rounding of every
-// input would cost ~0.4 % of the residual stream per layer.
+// lo = bf16(x - hi): about 16 significant bits, so W x = W hi + W lo (two MMAs
+// into one fp32 accumulator) keeps the projection inputs close to fp32 while
+// the weights stay exactly bf16.  A single bf16 rounding of every input would
+// cost ~0.4 % of the residual stream per layer.
 //
-// The operand is the A matrix of the projections: row a = hi(b) for a = b and
-// lo(b) for a = 8 nn + b (nn 8-sequence tiles, padded sequences stay 0), K
-// major, one 512 nn-byte block per 16-column k-block in the core-matrix order
-// above.  Element (k, sequence b) of hi, in bf16 units; lo is 8 nn rows
-// (nn * 128 elements) further.
+// Element (k, sequence b) of an operand with nn 8-column tiles, in bf16
+// units: 512-byte blocks per (16-row k-block, column tile), 16 bytes per lane
+// inside a block: {hi b0, hi b1, lo b0, lo b1} of the lane's B fragment.
+// Returns the position of hi; lo is 4 elements further.
 __device__ __forceinline__ size_t opnd_off(int k, int b, int nn) {
   const int kk = k & 15;
-  return (size_t)(k >> 4) * (256 * nn) + (b >> 3) * 128 + (kk >> 3) * 64 + (b & 7) * 8 + (kk & 7);
+  return ((size_t)(k >> 4) * nn + (b >> 3)) * 256 + ((b & 7) * 4 + ((kk & 7) >> 1)) * 8 +
+         (kk >> 3) * 2 + (kk & 1);
 }
 
 __device__ __forceinline__ void put_opnd(uint16_t *buf, int k, int b, int nn, float x) {
   const size_t o = opnd_off(k, b, nn);
   const uint16_t hi = f2bf(x);
   buf[o] = hi;
-  buf[o + (size_t)nn * 128] = f2bf(x - bf2f(hi));
+  buf[o + 4] = f2bf(x - bf2f(hi));
 }
+
+// JIT attention (MPK review, "Direction 4": the data-dependent operator is
+// resolved at run time).  The pairs p = b * Hkv + g, each with n_b = L_b + 1
+// positions (its cached rows and the new one), lie end to end on one line of
+// T positions; task a takes positions [a C, (a + 1) C) of it, so the tasks of
+// a layer carry equal work whatever the KV lengths, and a task may cover the
+// end of one pair and the start of the next.  C = the larger of ceil(T / A)
+// and ceil(max n_b / (S - 1)), rounded up to 16: at most S tasks touch a pair
+// (S = the partial slots per pair).  Every task and its producer derive the
+// same pieces from kv_len, which no task of the step changes before ARGMAX.
+struct JitPart {
+  int C, T;
+  const int *n;  // positions of each sequence's pairs (kv_len + 1), in shared memory
+};
+
+// Reads kv_len once (independent loads) into `lens` (kMaxBatch ints of
+// shared memory owned by the calling thread) and derives C and T.
+__device__ __forceinline__ JitPart jit_part(const Params &p, int *lens) {
+  int T = 0, nmax = 0;
+  for (int b = 0; b < p.B; ++b) lens[b] = __ldcg(p.kv_len + b) + 1;
+  for (int b = 0; b < p.B; ++b) {
+    T += lens[b] * p.Hkv;
+    nmax = max(nmax, lens[b]);
+  }
+  int C = (T + p.n_attn - 1) / p.n_attn;
+  C = max(C, (nmax + p.S - 2) / (p.S - 1));
+  return JitPart{(C + 15) & ~15, T, lens};
+}
+
+// One piece of an attention task: cached rows [c0, c1) of pair (b, g)
+// streamed in stages at origin o (stage st covers [o + st pps, o + (st + 1)
+// pps), clipped to [c0, c1)), the new row (position L) if has_new; the
+// piece's result is partial slot `slot` of the `expect` tasks that complete
+// the pair (expect == 1: written straight to att), and the last of them
+// merges `nmerge` partials.
+struct AttnSeg {
+  int b, g, L;
+  int c0, c1, o;
+  bool has_new;
+  int slot, expect, nmerge;
+};
+
+__device__ __forceinline__ int seg_stages(const Params &p, const AttnSeg &s) {
+  return s.c1 > s.c0 ? (s.c1 - 1 - s.o) / p.pps + 1 : 0;
+}
+
+// The pieces of JIT task a, in line order (no memory reads: the lengths
+// come with the partition).
+struct JitCursor {
+  int a, C, x, x1, b, g, r, n;
+  const int *len;
+  __device__ __forceinline__ void start(const Params &p, int task, const JitPart &jp) {
+    len = jp.n;
+    a = task;
+    C = jp.C;
+    x = min(a * C, jp.T);
+    x1 = min(x + C, jp.T);
+    int rest = x;
+    b = 0;
+    g = 0;
+    r = 0;
+    n = 1;
+    for (; b < p.B; ++b) {
+      n = len[b];
+      if (rest < n * p.Hkv) {
+        g = rest / n;
+        r = rest - g * n;
+        break;
+      }
+      rest -= n * p.Hkv;
+    }
+  }
+  __device__ __forceinline__ bool next(const Params &p, AttnSeg &s) {
+    if (x >= x1) return false;
+    const int len_here = min(n - r, x1 - x);
+    const int pp = x - r;  // line position of the pair's row 0
+    s.b = b;
+    s.g = g;
+    s.L = n - 1;
+    s.c0 = r;
+    s.c1 = min(r + len_here, s.L);
+    s.o = r / p.pps * p.pps;
+    s.has_new = r + len_here == n;
+    s.slot = a - pp / C;
+    s.expect = (pp + n - 1) / C - pp / C + 1;
+    s.nmerge = s.expect;
+    x += len_here;
+    r += len_here;
+    if (r == n) {
+      r = 0;
+      if (++g == p.Hkv) {
+        g = 0;
+        if (++b < p.B) n = len[b];
+      }
+    }
+    return true;
+  }
+};
+
+// JIT attention state kept in shared memory rather than registers: the
+// producer's lengths, and the compute side's lengths, cursor and current
+// piece (thread 0 advances the cursor; every compute thread reads the piece).
+struct JitShared {
+  int lens_p[kMaxBatch];
+  int lens_c[kMaxBatch];
+  JitCursor cur;
+  AttnSeg seg;
+  int more;
+};
 
 // ---------------------------------------------------------------------------
 // Shared memory layout (identical computation on host: see smem_bytes()).
 // ---------------------------------------------------------------------------
-enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kLogits = 5, kCtlWords = 16 };
+enum Ctl { kAbort = 0, kEpoch = 1, kConsumed = 2, kIssued = 3, kLast = 4, kLogits = 5, kWindow = 6,
+           kCtlWords = 16 };
 
 struct Smem {
   uint8_t *ring;
   uint64_t *full, *empty;
-  uint64_t *abar;   // [stages] tensor-core projections: the stage's operand chunk landed
-  uint64_t *mdone;  // the MMAs of a pass completed
-  uint32_t *tmem;   // TMEM base address of the CTA's accumulators
   volatile int *ctl;
   unsigned long long *tmark;  // [8] trace marks: prologue done, streaming done, ready,
                               // L2 prefetch bytes, first ring stage available
+  JitShared *jit;             // JIT attention state
   // GEMV scratch
   float *red;   // [kRedRows][kComputeWarps] warp partial sums of tile rows
   float *ss;    // [kComputeWarps]
@@ -371,7 +413,7 @@ struct Smem {
   float *mls;   // [3][kMaxRep]
   float *ored;  // per warp and head: [D] output, running max, running sum (merge: weights)
   // tensor-core projection scratch
-  float *cred;  // [32 columns][33]: one chunk of the accumulators read back from TMEM
+  float *cred;  // [warp][m-tile of the pass][16 rows][8 nn + 1] accumulator partials
   float *minv;  // [kMaxBatch] 1 / rms of each sequence's input
   float *mlv;   // [16] partial argmax values (LM head)
   int *mli;     // [16] partial argmax indices
@@ -380,7 +422,7 @@ struct Smem {
 __host__ __device__ inline size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct SmemOffsets {
-  size_t full, empty, abar, mdone, tmem, ctl, tmark, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, cred, minv,
+  size_t full, empty, ctl, tmark, jit, red, ss, lmv, lmi, q, knew, vnew, sc, mls, ored, cred, minv,
       mlv, mli, total;
 };
 
@@ -392,17 +434,13 @@ __host__ __device__ inline SmemOffsets smem_offsets(int stages, int stage_bytes,
   p += 8 * (size_t)stages;
   o.empty = p;
   p += 8 * (size_t)stages;
-  o.abar = p;
-  p += 8 * (size_t)stages;
-  o.mdone = p;
-  p += 8;
-  o.tmem = p;
-  p += 8;
   o.ctl = p;
   p += 4 * kCtlWords;
   p = align_to(p, 16);
   o.tmark = p;
   p += 64;
+  o.jit = p;
+  p += align_to(sizeof(JitShared), 16);
   // GEMV scratch
   size_t g = p;
   o.red = g;
@@ -450,11 +488,9 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const Params &p) {
   s.ring = base;
   s.full = reinterpret_cast<uint64_t *>(base + o.full);
   s.empty = reinterpret_cast<uint64_t *>(base + o.empty);
-  s.abar = reinterpret_cast<uint64_t *>(base + o.abar);
-  s.mdone = reinterpret_cast<uint64_t *>(base + o.mdone);
-  s.tmem = reinterpret_cast<uint32_t *>(base + o.tmem);
   s.ctl = reinterpret_cast<volatile int *>(base + o.ctl);
   s.tmark = reinterpret_cast<unsigned long long *>(base + o.tmark);
+  s.jit = reinterpret_cast<JitShared *>(base + o.jit);
   s.red = reinterpret_cast<float *>(base + o.red);
   s.ss = reinterpret_cast<float *>(base + o.ss);
   s.lmv = reinterpret_cast<float *>(base + o.lmv);
@@ -524,75 +560,35 @@ __device__ __forceinline__ Gemv gemv_of(const Params &p, int type, int layer, in
   return g;
 }
 
-// A projection task on tcgen05 tensor cores (batch >= 2).  The task's rows
-// (padded to a multiple of 16) run in passes of up to kUmmaMaxN rows (one
-// accumulator of 128 lanes x N columns in TMEM); a pass streams its weights in
-// ring stages of nkb 16-column k-blocks.  In the arena each task's rows are
-// contiguous, pass by pass, and a pass of N rows holds, per k-block, its N x 16
-// weights in the core-matrix order (N * 32 bytes: the B operand of one MMA),
-// so a stage is one contiguous copy.  A stage's slot holds those weights, then
-// the matching operand chunk (512 nn bytes per k-block: the A operand), then
-// kUmmaSlack bytes that the A descriptors of the chunk's last k-blocks read
-// past it (rows 16 nn .. 127 of A, which only reach accumulator lanes that
-// are never read).
-struct UTile {
-  const uint8_t *w;  // the task's first weight byte
-  int K, KB;         // columns, 16-column k-blocks
-  int row0, rows;    // first row of the task, rows (a multiple of 16)
-  int npass, nlast;  // passes, rows of the last pass
-  int nkb_full, nkc_full, nkb_last, nkc_last;  // k-blocks per stage, stages of a pass
-  int nst;           // stages of the task
+// A projection task on tensor cores: its m-tiles [mt0, mt1) of the
+// fragment-ordered matrix are streamed as row blocks of mb m-tiles, each row
+// block as nkc ring stages of (up to) kcb k-blocks.  Every (m-tile, k-block)
+// is one 512-byte fragment block; stage (rb, kc) packs the blocks of its
+// m-tiles as [m-tile][k-block].
+struct MmaTile {
+  const uint16_t *w;  // the operator's matrix, fragment order
+  int KB;             // k-blocks per row (K / 16)
+  int mt0, mt1;       // m-tiles of this task
+  int mb, kcb, nkc, nrb;
 };
 
-// k-blocks per stage for a pass of N rows (weights, operand and slack fit the slot).
-__device__ __forceinline__ int umma_nkb(const Params &p, int N, int KB) {
-  const int n = (p.stage_bytes - kUmmaSlack) / (N * 32 + 512 * p.nn);
-  return min(KB, max(n, 1));
-}
-
-__device__ __forceinline__ UTile umma_tile(const Params &p, int type, int layer, int idx) {
+__device__ __forceinline__ MmaTile mma_tile(const Params &p, int type, int layer, int idx) {
   const Gemv g = gemv_of(p, type, layer, idx);
-  UTile u;
-  u.K = g.K;
-  u.KB = g.K >> 4;
-  u.row0 = g.row0;
-  u.rows = (g.row1 - g.row0 + 15) & ~15;  // the LM head's last task: zero padding rows
-  u.w = reinterpret_cast<const uint8_t *>(g.w) + (size_t)g.row0 * g.K * 2;
-  u.npass = (u.rows + kUmmaMaxN - 1) / kUmmaMaxN;
-  u.nlast = u.rows - (u.npass - 1) * kUmmaMaxN;
-  u.nkb_full = umma_nkb(p, kUmmaMaxN, u.KB);
-  u.nkc_full = (u.KB + u.nkb_full - 1) / u.nkb_full;
-  u.nkb_last = umma_nkb(p, u.nlast, u.KB);
-  u.nkc_last = (u.KB + u.nkb_last - 1) / u.nkb_last;
-  u.nst = (u.npass - 1) * u.nkc_full + u.nkc_last;
-  return u;
-}
-
-// Stage st of a task: pass q, rows N, first k-block kb0, k-blocks nkb of a
-// full stage of the pass and nkb_here of this one, weight byte offset.
-struct UStage {
-  int q, c, N, nkb, kb0, nkb_here;
-  size_t woff;
-};
-
-__device__ __forceinline__ UStage umma_stage(const UTile &u, int st) {
-  UStage s;
-  const int full = (u.npass - 1) * u.nkc_full;
-  if (st < full) {
-    s.q = st / u.nkc_full;
-    s.c = st - s.q * u.nkc_full;
-    s.N = kUmmaMaxN;
-    s.nkb = u.nkb_full;
-  } else {
-    s.q = u.npass - 1;
-    s.c = st - full;
-    s.N = u.nlast;
-    s.nkb = u.nkb_last;
+  MmaTile m;
+  m.w = g.w;
+  m.KB = g.K >> 4;
+  m.mt0 = g.row0 >> 4;
+  m.mt1 = (g.row1 + 15) >> 4;  // the LM head's last m-tile may hold zero padding rows
+  switch (type) {
+    case 2: m.mb = p.mb_qkv; m.kcb = p.kcb_qkv; break;
+    case 5: m.mb = p.mb_o; m.kcb = p.kcb_o; break;
+    case 6: m.mb = p.mb_gu; m.kcb = p.kcb_gu; break;
+    case 7: m.mb = p.mb_down; m.kcb = p.kcb_down; break;
+    default: m.mb = p.mb_lm; m.kcb = p.kcb_lm; break;
   }
-  s.kb0 = s.c * s.nkb;
-  s.nkb_here = min(s.nkb, u.KB - s.kb0);
-  s.woff = (size_t)s.q * kUmmaMaxN * u.K * 2 + (size_t)s.kb0 * s.N * 32;
-  return s;
+  m.nkc = (m.KB + m.kcb - 1) / m.kcb;
+  m.nrb = (m.mt1 - m.mt0 + m.mb - 1) / m.mb;
+  return m;
 }
 
 struct AttnSpan {
@@ -617,98 +613,6 @@ __device__ __forceinline__ AttnSpan attn_span(const Params &p, int idx) {
   return a;
 }
 
-// JIT attention (MPK review, "Direction 4": the data-dependent operator is
-// resolved at run time).  The pairs p = b * Hkv + g, each with n_b = L_b + 1
-// positions (its cached rows and the new one), lie end to end on one line of
-// T positions; task a takes positions [a C, (a + 1) C) of it, so the tasks of
-// a layer carry equal work whatever the KV lengths, and a task may cover the
-// end of one pair and the start of the next.  C = the larger of ceil(T / A)
-// and ceil(max n_b / (S - 1)), rounded up to 16: at most S tasks touch a pair
-// (S = the partial slots per pair).  Every task and its producer derive the
-// same pieces from kv_len, which no task of the step changes before ARGMAX.
-struct JitPart {
-  int C, T;
-};
-
-__device__ __forceinline__ JitPart jit_part(const Params &p) {
-  int T = 0, nmax = 0;
-  for (int b = 0; b < p.B; ++b) {
-    const int n = __ldcg(p.kv_len + b) + 1;
-    T += n * p.Hkv;
-    nmax = max(nmax, n);
-  }
-  int C = (T + p.n_attn - 1) / p.n_attn;
-  C = max(C, (nmax + p.S - 2) / (p.S - 1));
-  return JitPart{(C + 15) & ~15, T};
-}
-
-// One piece of an attention task: cached rows [c0, c1) of pair (b, g)
-// streamed in stages at origin o (stage st covers [o + st pps, o + (st + 1)
-// pps), clipped to [c0, c1)), the new row (position L) if has_new; the
-// piece's result is partial slot `slot` of the `expect` tasks that complete
-// the pair (expect == 1: written straight to att), and the last of them
-// merges `nmerge` partials.
-struct AttnSeg {
-  int b, g, L;
-  int c0, c1, o;
-  bool has_new;
-  int slot, expect, nmerge;
-};
-
-__device__ __forceinline__ int seg_stages(const Params &p, const AttnSeg &s) {
-  return s.c1 > s.c0 ? (s.c1 - 1 - s.o) / p.pps + 1 : 0;
-}
-
-// The pieces of JIT task a, in line order.
-struct JitCursor {
-  int a, C, x, x1, b, g, r, n;
-  __device__ __forceinline__ void start(const Params &p, int task, const JitPart &jp) {
-    a = task;
-    C = jp.C;
-    x = min(a * C, jp.T);
-    x1 = min(x + C, jp.T);
-    int rest = x;
-    b = 0;
-    g = 0;
-    r = 0;
-    n = 1;
-    for (; b < p.B; ++b) {
-      n = __ldcg(p.kv_len + b) + 1;
-      if (rest < n * p.Hkv) {
-        g = rest / n;
-        r = rest - g * n;
-        break;
-      }
-      rest -= n * p.Hkv;
-    }
-  }
-  __device__ __forceinline__ bool next(const Params &p, AttnSeg &s) {
-    if (x >= x1) return false;
-    const int len = min(n - r, x1 - x);
-    const int pp = x - r;  // line position of the pair's row 0
-    s.b = b;
-    s.g = g;
-    s.L = n - 1;
-    s.c0 = r;
-    s.c1 = min(r + len, s.L);
-    s.o = r / p.pps * p.pps;
-    s.has_new = r + len == n;
-    s.slot = a - pp / C;
-    s.expect = (pp + n - 1) / C - pp / C + 1;
-    s.nmerge = s.expect;
-    x += len;
-    r += len;
-    if (r == n) {
-      r = 0;
-      if (++g == p.Hkv) {
-        g = 0;
-        if (++b < p.B) n = __ldcg(p.kv_len + b) + 1;
-      }
-    }
-    return true;
-  }
-};
-
 // Element offset of cache row `row` of (layer, sequence b, kv head g): the
 // contiguous layout, or row % P of the sequence's page of the paged pools.
 __device__ __forceinline__ size_t kv_row(const Params &p, int layer, int b, int g, int row) {
@@ -726,9 +630,9 @@ struct Stream {
   uint32_t bytes = 0, last_bytes = 0;  // bytes of a full / of the last stage
   uint32_t stride = 0;            // bytes between consecutive stages
   int nst = 0;                    // stages
-  // tensor-core projections: stages as umma_stage(u, st)
-  int uk = 0;                     // 0 for the other streams
-  UTile u{};
+  // tensor-core projections: stage st = (row block st / nkc, k chunk st % nkc)
+  int nkc = 0;                    // 0 for the other streams
+  int KB = 0, mt0 = 0, mt1 = 0, mb = 0, kcb = 0;
   // attention: K/V rows y0 + st * pps .. of the 2-D cache tensor maps (paged
   // pools: stage st starts at position kv_p0 + st * pps of (layer, b, g);
   // a stage never crosses a page)
@@ -737,12 +641,13 @@ struct Stream {
   int kv_l = 0, kv_b = 0, kv_g = 0, kv_p0 = 0;
   // JIT attention: the pieces of task ja (see JitCursor), stages in piece order
   int jit = 0, ja = 0;
-  JitPart jp{};
+  JitPart jp{0, 0, nullptr};
 };
 
 // First cache row (in rows of D elements) of K/V stage st of stream s.
+template <bool kExt>
 __device__ __forceinline__ int kv_stage_row(const Params &p, const Stream &s, int st) {
-  if (s.jit) {  // the piece holding stage st; the stage starts at its first row
+  if (kExt && s.jit) {  // the piece holding stage st; the stage starts at its first row
     JitCursor cur;
     cur.start(p, s.ja, s.jp);
     AttnSeg sg;
@@ -758,20 +663,28 @@ __device__ __forceinline__ int kv_stage_row(const Params &p, const Stream &s, in
   return s.y0 + st * p.pps;
 }
 
-// kMma: the batched kernel (tensor-core tiles, swizzled TMA K/V boxes).
-template <bool kMma>
-__device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t) {
+// kMma: the batched kernel (tensor-core tiles, swizzled TMA K/V boxes);
+// kExt: the extended kernels (JIT attention, dispatch mode).
+template <bool kMma, bool kExt>
+__device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t, int *jit_lens) {
   Stream s{};
   const int type = t.type;
   if (kMma && (type == 2 || (type >= 5 && type <= 8))) {
-    s.u = umma_tile(p, type, t.layer, (int)t.idx);
-    s.uk = 1;
-    s.nst = s.u.nst;
+    const MmaTile m = mma_tile(p, type, t.layer, (int)t.idx);
+    s.src0 = reinterpret_cast<const uint8_t *>(m.w);
+    s.nst = m.nrb * m.nkc;
+    s.nkc = m.nkc;
+    s.KB = m.KB;
+    s.mt0 = m.mt0;
+    s.mt1 = m.mt1;
+    s.mb = m.mb;
+    s.kcb = m.kcb;
     return s;
   }
-  if (kMma && type == 3 && p.jit) {
+
+  if (kMma && kExt && type == 3 && p.jit) {
     // whole boxes of pps rows from each stage's first row (masked past its end)
-    s.jp = jit_part(p);
+    s.jp = jit_part(p, jit_lens);
     s.ja = (int)t.idx;
     s.jit = 1;
     s.kv = 1;
@@ -812,9 +725,11 @@ __device__ __forceinline__ Stream task_stream(const Params &p, const DevTask &t)
 // Bytes that stage st of stream s lands in the ring.
 template <bool kMma>
 __device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
-  if (kMma && s.uk) {
-    const UStage u = umma_stage(s.u, st);
-    return (uint32_t)(u.nkb_here * u.N * 32);
+  if (kMma && s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int nm = min(s.mb, s.mt1 - (s.mt0 + rb * s.mb));
+    const int nkb = min(s.kcb, s.KB - kc * s.kcb);
+    return (uint32_t)(nm * nkb * 512);
   }
   if (s.kv) return 2 * (st == s.nst - 1 ? s.last_bytes : s.bytes);  // K and V
   return st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -822,11 +737,11 @@ __device__ __forceinline__ uint32_t stage_bytes_of(const Stream &s, int st) {
 
 // Issue the copies of stage st of stream s into ring slot dst (the full
 // barrier already expects stage_bytes_of(s, st) bytes).
-template <bool kMma>
+template <bool kMma, bool kExt>
 __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, int st, uint8_t *dst,
                                             uint64_t *bar, uint64_t pol) {
   if (s.kv) {
-    const int y = kv_stage_row(p, s, st);
+    const int y = kv_stage_row<kExt>(p, s, st);
     if (!kMma) {  // plain rows: K at dst, V pps rows further
       const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
       bulk_g2s(dst, p.k_cache + (size_t)y * p.D, nb, bar, pol);
@@ -841,9 +756,14 @@ __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, in
     }
     return;
   }
-  if (kMma && s.uk) {  // the stage's weights: one contiguous copy
-    const UStage u = umma_stage(s.u, st);
-    bulk_g2s(dst, s.u.w + u.woff, (uint32_t)(u.nkb_here * u.N * 32), bar, pol);
+  if (kMma && s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
+    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
+    const uint32_t cb = (uint32_t)nkb * 512u;
+    for (int i = 0; i < nm; ++i)
+      bulk_g2s(dst + (size_t)i * cb, s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb, bar,
+               pol);
     return;
   }
   const uint32_t nb = st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -853,11 +773,13 @@ __device__ __forceinline__ void issue_stage(const Params &p, const Stream &s, in
 // Prefetch stage st of stream s into L2; returns the bytes requested.
 template <bool kMma>
 __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
-  if (kMma && s.uk) {
-    const UStage u = umma_stage(s.u, st);
-    const uint32_t nb = (uint32_t)(u.nkb_here * u.N * 32);
-    prefetch_l2(s.u.w + u.woff, nb);
-    return nb;
+  if (kMma && s.nkc > 0) {
+    const int rb = st / s.nkc, kc = st - rb * s.nkc;
+    const int m0 = s.mt0 + rb * s.mb, nm = min(s.mb, s.mt1 - m0);
+    const int kb0 = kc * s.kcb, nkb = min(s.kcb, s.KB - kb0);
+    const uint32_t cb = (uint32_t)nkb * 512u;
+    for (int i = 0; i < nm; ++i) prefetch_l2(s.src0 + ((size_t)(m0 + i) * s.KB + kb0) * 512, cb);
+    return cb * (uint32_t)nm;
   }
   if (s.kv) return 0u;  // K/V tiles are not prefetched
   const uint32_t pb = st == s.nst - 1 ? s.last_bytes : s.bytes;
@@ -868,8 +790,6 @@ __device__ __forceinline__ uint32_t prefetch_stage(const Stream &s, int st) {
 // ---------------------------------------------------------------------------
 // Producer: one thread streams every stage of the worker's queue.
 // ---------------------------------------------------------------------------
-constexpr uint64_t kPrefetchHoldNs = 1500;  // see producer_loop
-
 struct Queue {
   int first, stride, count;  // tasks first, first + stride, ... (count of them)
   // dispatch mode: the entries the scheduler publishes for this worker
@@ -880,8 +800,9 @@ struct Queue {
 // Task id of entry n of the worker's queue, or -1 past its end (static
 // queues) / at the scheduler's end mark.  In dispatch mode the entry is
 // waited for (bounded); -1 also when the CTA aborts or the wait runs out.
+template <bool kExt>
 __device__ __forceinline__ int queue_task(const Params &p, const Smem &sm, const Queue &q, int n) {
-  if (!q.list) return n < q.count ? q.first + n * q.stride : -1;
+  if (!kExt || !q.list) return n < q.count ? q.first + n * q.stride : -1;
   if ((int32_t)(ld_acquire(q.tail) - (uint32_t)n) <= 0) {
     const uint64_t t0 = global_timer();
     uint32_t spins = 0;
@@ -898,20 +819,23 @@ __device__ __forceinline__ int queue_task(const Params &p, const Smem &sm, const
   return __ldcg(q.list + n);
 }
 
-template <bool kMma>
+template <bool kMma, bool kExt>
 __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   const int NS = p.ring_stages;
   uint32_t k = 0;
   const uint64_t budget = 4ull * p.timeout_ns + 1000000000ull;
   // L2 prefetch cursor (task pf_n, stage pf_st, global stage index pf_k) in
-  // the worker's stream of stages, across task boundaries.  While the ring's
-  // oldest stage has landed and stayed unconsumed for over kPrefetchHoldNs
-  // (the compute warps wait on an event or run attention, so HBM has spare
-  // capacity) the producer prefetches the next stages into L2, up to
-  // l2_prefetch_bytes ahead of the ring, one stage per few polls of the ring:
-  // a burst of prefetches from every SM at once slows the attention tasks,
-  // which sit on the critical path (Qwen3-8B at batch 1: 3141 us per step
-  // with back-to-back prefetches in the attention window against 3095 us).
+  // the worker's stream of stages, across task boundaries.  While the ring is
+  // full and the compute warps wait for an O projection's event
+  // (sm.ctl[kWindow]), the step is in its attention window: attention moves
+  // little data and no operator streams weights, so every SM has spare HBM
+  // bandwidth.  The producer then prefetches its next stages into L2, one per
+  // poll of the ring, up to l2_prefetch_bytes ahead of it.  (Prefetching
+  // whenever the ring stalls takes bandwidth from SMs still streaming the
+  // current operator; a burst from every SM while attention runs slows the
+  // attention tasks on the critical path.  Qwen3-8B at batch 1, one box:
+  // 3079 us per step with this window, 3130 us with the stall-gated rule,
+  // 3141 us with back-to-back prefetches during attention.)
   // (dispatch mode: the queue holds only tasks that are ready, no lookahead)
   const long long dist = q.list ? 0 : p.l2_prefetch_bytes;
   const uint64_t pol = stream_policy(p.evict_first != 0);
@@ -921,6 +845,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   uint32_t pf_k = 0;
   long long ahead = 0;
   const uint32_t epoch0 = (uint32_t)sm.ctl[kEpoch];
+  int *jl = sm.jit->lens_p;
   for (int s = 0; s < p.n_steps; ++s) {
   // K/V rows of step s > 0 include the rows step s - 1 appended (possibly on
   // another SM), and the stream's extent depends on kv_len: the first K/V
@@ -928,7 +853,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // streams are never gated, so they run ahead across the step boundary.
   bool kv_open = s == 0;
   for (int n = 0; n < q.count; ++n) {
-    const int tid_n = queue_task(p, sm, q, n);
+    const int tid_n = queue_task<kExt>(p, sm, q, n);
     if (tid_n < 0) break;
     const DevTask tk = p.tasks[tid_n];
     if (tk.type == 3 && !kv_open) {
@@ -944,13 +869,13 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       fence_proxy_async_global();  // the appended rows are read by bulk / tensor copies
       kv_open = true;
     }
-    const Stream ts = task_stream<kMma>(p, tk);
+    const Stream ts = task_stream<kMma, kExt>(p, tk, jl);
     for (int st = 0; st < ts.nst; ++st) {
       const uint32_t nb = stage_bytes_of<kMma>(ts, st);
       if (dist > 0) {
         // stages before k were issued without a prefetch: move the cursor on
         while (pf_k < k && pf_n < q.count) {
-          if (pfs.nst < 0) pfs = task_stream<kMma>(p, p.tasks[q.first + pf_n * q.stride]);
+          if (pfs.nst < 0) pfs = task_stream<kMma, kExt>(p, p.tasks[q.first + pf_n * q.stride], jl);
           if (pf_st >= pfs.nst) {
             ++pf_n;
             pf_st = 0;
@@ -968,24 +893,11 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
         const uint32_t par = (use - 1) & 1u;
         uint64_t t0 = 0;
         uint32_t spins = 0;
-        uint64_t t_held = 0;
         while (!mbar_test(&sm.empty[slot], par)) {
           if (sm.ctl[kAbort]) goto out;
           ++spins;
-          // prefetch only while the consumer, not HBM, holds the ring back:
-          // the oldest stage in flight (this slot's previous use) has landed
-          // and stayed unreleased for over kPrefetchHoldNs (the compute warps
-          // wait on an event or run attention; a stage of streaming work is
-          // released well within that time)
-          bool idle = false;
-          if (dist > 0 && ahead < dist && (spins & 7u) == 0 && pf_n < q.count &&
-              mbar_test(&sm.full[slot], par)) {
-            const uint64_t now = global_timer();
-            if (t_held == 0) t_held = now;
-            idle = now - t_held > kPrefetchHoldNs;
-          }
-          if (idle) {
-            if (pfs.nst < 0) pfs = task_stream<kMma>(p, p.tasks[q.first + pf_n * q.stride]);
+          if (dist > 0 && ahead < dist && pf_n < q.count && sm.ctl[kWindow]) {
+            if (pfs.nst < 0) pfs = task_stream<kMma, kExt>(p, p.tasks[q.first + pf_n * q.stride], jl);
             if (pf_st >= pfs.nst) {
               ++pf_n;
               pf_st = 0;
@@ -1010,7 +922,7 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
       }
       uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes;
       mbar_arrive_expect_tx(&sm.full[slot], nb);
-      issue_stage<kMma>(p, ts, st, dst, &sm.full[slot], pol);
+      issue_stage<kMma, kExt>(p, ts, st, dst, &sm.full[slot], pol);
       if (dist > 0 && pf_k > k) ahead -= nb;  // stage k was prefetched
       ++k;
     }
@@ -1095,10 +1007,14 @@ struct DepWait {
   int dep;
   uint32_t epoch;
   int task;
+  int type;
   __device__ __forceinline__ bool operator()() const {
     // (dispatch mode: the scheduler hands out a task once its event fired)
     if (p.persistent && !p.dispatch && dep >= 0 && threadIdx.x == 0) {
+      // the wait of an O projection is the step's attention window (see producer_loop)
+      sm.ctl[kWindow] = type == 5;
       if (!wait_event(p, dep, epoch, task)) sm.ctl[kAbort] = 1;
+      sm.ctl[kWindow] = 0;
     }
     compute_sync();
     if (p.trace && threadIdx.x == 0) sm.tmark[2] = global_timer();
@@ -1340,8 +1256,64 @@ __device__ __forceinline__ bool gemv_task(const Params &p, const Smem &sm, const
 }
 
 // ---------------------------------------------------------------------------
-// Projection task on tcgen05 tensor cores (batch >= 2).
+// Projection task on tensor cores (batch >= 2).
 // ---------------------------------------------------------------------------
+// B fragments of k-blocks kb0 + warp + 8 j (j < kpw) of the operand xb: the
+// activations are written earlier in this step by other SMs, so they are read
+// through L2 (never from a possibly stale L1 line).
+template <int NN>
+__device__ __forceinline__ void load_bfrag(uint4 (&bf)[mma_max_kpw(NN)][NN], const uint16_t *xb,
+                                           int kb0, int kpw, int warp, int lane) {
+#pragma unroll
+  for (int j = 0; j < mma_max_kpw(NN); ++j) {
+    if (j < kpw) {
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+        bf[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
+                              xb + ((size_t)(kb0 + warp + 8 * j) * NN + n) * 256) + lane);
+    }
+  }
+}
+
+// One ring stage of a projection with compile-time tile counts (MBF m-tiles,
+// KPWF k-blocks per warp): the common cases, with no per-tile guards, so the
+// A fragments of a k-block are loaded before its MMAs.  The B fragments of
+// the next stage's first kpw_n k-blocks are refilled after their last use.
+template <int NN, int MBF, int KPWF, bool kGuard>
+__device__ __forceinline__ void mma_stage_fixed(float (&acc)[kMmaMaxMB][NN][4],
+                                                uint4 (&bc)[mma_max_kpw(NN)][NN], const uint8_t *slot,
+                                                const uint16_t *xn, int kpw_n, int warp, int lane) {
+  constexpr int NKB = 8 * KPWF;
+#pragma unroll
+  for (int j = 0; j < KPWF; ++j) {
+    const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
+    uint4 a[MBF];
+#pragma unroll
+    for (int m = 0; m < MBF; ++m) a[m] = *reinterpret_cast<const uint4 *>(blk + m * NKB * 512);
+#pragma unroll
+    for (int m = 0; m < MBF; ++m)
+#pragma unroll
+      for (int n = 0; n < NN; ++n) {
+        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
+        mma_bf16(acc[m][n], a[m], make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
+      }
+    if (!kGuard || j < kpw_n) {
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+    }
+  }
+  // a next stage with more k-blocks (the first chunk after a short last one)
+#pragma unroll
+  for (int j = KPWF; j < (kGuard ? mma_max_kpw(NN) : 0); ++j) {
+    if (j < kpw_n) {
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+        bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+    }
+  }
+}
+
 // Sum over the 16 lanes of a half warp (lanes that share a sequence column).
 __device__ __forceinline__ float half_warp_sum(float v) {
 #pragma unroll
@@ -1349,63 +1321,29 @@ __device__ __forceinline__ float half_warp_sum(float v) {
   return v;
 }
 
-// Bounded wait for the completion of phase `par` of an mbarrier by thread 0;
-// false (with the error recorded) on timeout or abort.
-__device__ bool wait_bar(const Params &p, const Smem &sm, uint64_t *bar, uint32_t par, int task) {
-  if (mbar_test(bar, par)) return true;
-  uint64_t t0 = 0;
-  uint32_t spins = 0;
-  while (!mbar_test(bar, par)) {
-    if (sm.ctl[kAbort]) return false;
-    if ((++spins & 255u) == 0) {
-      const uint64_t now = global_timer();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > 4ull * p.timeout_ns + 1000000000ull) {
-        record_error(p, kDevTimeout, task, -1);
-        sm.ctl[kAbort] = 1;
-        return false;
-      }
-    }
-  }
-  return true;
-}
-
-// Per-CTA state of the tensor-core path, kept by the compute threads across
-// tasks: the parity of the next MMA-completion phase (every compute thread)
-// and, in thread 0, the parity of each slot's next operand phase and the
-// slots whose operand copy is in flight.
-struct UmmaState {
-  uint32_t mph = 0;
-  uint32_t aph = 0, apend = 0;
-};
-
-// The batched projection y[b][r] = sum_k W[r][k] x̂[b][k] of one task.  The
-// input arrives as the hi/lo bf16 operand of x[b][k] * gain[k] written by the
-// producing task's epilogue, with per-16-row sums of squares; the RMSNorm's
-// per-sequence factor 1 / rms(x_b) is applied to the fp32 sums in the
-// epilogue (it factors out of the sum over k).
+// The batched projection y[b][r] = sum_k W[r][k] x̂[b][k] of one task on
+// mma.sync.  The input arrives as a hi/lo bf16 operand of x[b][k] * gain[k]
+// written by the producing task's epilogue, with per-16-row sums of squares;
+// the RMSNorm's per-sequence factor 1 / rms(x_b) is applied to the fp32
+// accumulators in the epilogue (it factors out of the sum over k).
 //
-// Thread 0 issues everything asynchronous: after the dependency event it
-// copies each stage's operand chunk into the stage's slot (bulk copies, up to
-// ring_stages - 1 stages ahead), waits for the stage's weights (the producer
-// warp) and operand, issues the stage's MMAs (M = 128: operand rows, N = the
-// pass's weight rows, one per k-block) into the pass's TMEM accumulator, and
-// commits them to the slot's empty barrier, which frees the slot once they
-// completed (the other seven arrivals of that barrier are made at once).  At
-// the end of a pass warp 0 reads the accumulator lanes 0 .. 31 (the operand
-// rows hi(b), lo(b)) back in 32-column chunks and the compute threads run the
-// operator's fused epilogue on hi + lo, thread (row tid % 16 of an m-tile,
-// sequence tid / 16 % 8 nn).
+// Work split: for each ring stage (row block x k chunk) warp w takes the
+// k-blocks w, w + 8, ... of the chunk for every m-tile of the row block, so
+// every B fragment is loaded by one warp, once per row block.  The warps'
+// partial sums of a row block are added in shared memory in a fixed order
+// (deterministic), PM m-tiles per pass, and the fused epilogue of the
+// operator runs on the sums: thread (row = tid % 16, sequence = tid / 16 % 8nn).
 template <int NN>
-__device__ __forceinline__ bool umma_task(const Params &p, const Smem &sm, const DevTask &t,
-                                          uint32_t &k, UmmaState &us, int task_id,
-                                          const DepWait &dep_wait) {
-  constexpr int NC = 8 * NN;         // operand sequence columns (zero padded)
-  constexpr uint32_t AB = 512u * NN; // operand bytes per k-block
+__device__ __forceinline__ bool mma_task(const Params &p, const Smem &sm, const DevTask &t,
+                                         uint32_t &k, int task_id, const DepWait &dep_wait) {
+  constexpr int NC = 8 * NN;          // operand columns (sequences, zero padded)
+  constexpr int PM = NN == 2 ? 2 : 4; // m-tiles per reduction pass
+  constexpr int CS = NC + 1;          // row stride of the reduction buffer (floats)
+  static_assert(kComputeWarps * PM * 16 * CS <= kMmaCredFloats, "reduction buffer");
   const int type = t.type;
   const int layer = t.layer;
   const DevLayer *L = layer < p.Ly ? p.layers + layer : nullptr;
-  const UTile u = umma_tile(p, type, layer, (int)t.idx);
+  const MmaTile mt = mma_tile(p, type, layer, (int)t.idx);
   const uint16_t *xb;
   const float *ssp = nullptr;
   switch (type) {
@@ -1415,35 +1353,15 @@ __device__ __forceinline__ bool umma_task(const Params &p, const Smem &sm, const
     case 7: xb = L->hb; break;
     default: xb = p.xfb; ssp = p.ssf; break;
   }
-  const uint8_t *xa = reinterpret_cast<const uint8_t *>(xb);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = tid & 15;          // row of an m-tile this thread finishes
   const int col = (tid >> 4) % NC;   // sequence this thread finishes
   const bool col_ok = col < p.B;
-  const int N_op = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
-  const int NS = p.ring_stages;
-  const uint64_t pol = stream_policy(false);  // the operand is read by every task of the operator
-  const uint32_t tmem = *sm.tmem;
+  const int N = type == 2 ? p.n_qkv : type == 6 ? 2 * p.F : type == 8 ? p.V : p.H;
 
   if (!dep_wait()) return false;
-  // operand chunk of stage i (global stage k + i) into its slot, after the weights
-  auto issue_a = [&](int i) {
-    const UStage st = umma_stage(u, i);
-    const int slot = (int)((k + (uint32_t)i) % (uint32_t)NS);
-    uint8_t *dst = sm.ring + (size_t)slot * p.stage_bytes + (size_t)st.nkb * st.N * 32;
-    const uint32_t nb = (uint32_t)st.nkb_here * AB;
-    mbar_arrive_expect_tx(&sm.abar[slot], nb);
-    bulk_g2s(dst, xa + (size_t)st.kb0 * AB, nb, &sm.abar[slot], pol);
-    us.apend |= 1u << slot;
-  };
-  if (tid == 0) {
-    // the operand was written by other SMs and acquired with the event: order
-    // that before the bulk copies (async proxy) read it
-    fence_proxy_async_global();
-    // the slots of the first stages were freed by earlier tasks, which waited
-    // for their MMAs
-    for (int i = 0; i < min(NS - 1, u.nst); ++i) issue_a(i);
-  }
+  uint4 bc[mma_max_kpw(NN)][NN];
+  load_bfrag<NN>(bc, xb, 0, min(mt.kcb, mt.KB) >> 3, warp, lane);
   float inv = 1.f;
   if (ssp) {
     for (int b = warp; b < p.B; b += kComputeWarps) {
@@ -1455,127 +1373,166 @@ __device__ __forceinline__ bool umma_task(const Params &p, const Smem &sm, const
     compute_sync();
     inv = col_ok ? sm.minv[col] : 0.f;
   }
+
+  float acc[kMmaMaxMB][NN][4];
+#pragma unroll
+  for (int m = 0; m < kMmaMaxMB; ++m)
+#pragma unroll
+    for (int n = 0; n < NN; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
   float best_v = -INFINITY;
   int best_i = 0x7fffffff;
   trace_mark(p, sm, 0);
-  int st = 0;
-  for (int q = 0; q < u.npass; ++q) {
-    const int N = q < u.npass - 1 ? kUmmaMaxN : u.nlast;
-    const int nst_q = q < u.npass - 1 ? u.nkc_full : u.nkc_last;
-    if (tid == 0) {
-      const uint32_t idesc = umma_idesc(N);
-      for (int c = 0; c < nst_q; ++c, ++st) {
-        if (sm.ctl[kAbort]) continue;
-        const UStage s = umma_stage(u, st);
-        const uint32_t kg = k + (uint32_t)st;
-        const int slot = (int)(kg % (uint32_t)NS);
-        if (!wait_full(p, sm, kg, task_id)) continue;
-        if (!wait_bar(p, sm, &sm.abar[slot], (us.aph >> slot) & 1u, task_id)) continue;
-        us.aph ^= 1u << slot;
-        us.apend &= ~(1u << slot);
-        trace_first_stage(p, sm, st);
-        tc_fence_after();
-        const uint32_t wb = smem_u32(sm.ring + (size_t)slot * p.stage_bytes);
-        const uint32_t abase = wb + (uint32_t)(s.nkb * s.N * 32);
-        for (int j = 0; j < s.nkb_here; ++j)
-          umma_bf16(tmem, umma_desc(abase + (uint32_t)j * AB), umma_desc(wb + (uint32_t)(j * N * 32)),
-                    idesc, (c > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&sm.empty[slot]);               // frees the slot once the MMAs completed
-        mbar_arrive_n(&sm.empty[slot], kComputeWarps - 1);
-        // the operand of stage st + NS - 1 goes into the slot of stage st - 1
-        if (st + NS - 1 < u.nst) {
-          if (st >= 1) {
-            const uint32_t kp = kg - 1u;
-            if (!wait_bar(p, sm, &sm.empty[kp % (uint32_t)NS], (kp / (uint32_t)NS) & 1u, task_id))
-              continue;
-          }
-          issue_a(st + NS - 1);
-        }
-      }
-      umma_commit(sm.mdone);  // arrives once every MMA issued so far completed
-    } else {
-      st += nst_q;
-    }
-    // every compute thread: the pass's accumulator is complete
-    {
-      uint64_t t0 = 0;
-      uint32_t spins = 0;
-      while (!mbar_test(sm.mdone, us.mph & 1u)) {
-        if ((++spins & 255u) == 0) {
-          const uint64_t now = global_timer();
-          if (t0 == 0) t0 = now;
-          else if (now - t0 > 4ull * p.timeout_ns + 1000000000ull) {
-            if (tid == 0) record_error(p, kDevTimeout, task_id, -1);
-            sm.ctl[kAbort] = 1;
-            break;
-          }
-        }
-      }
-      us.mph ^= 1u;
-    }
-    compute_sync();
-    if (sm.ctl[kAbort]) break;
-    tc_fence_after();
-    // epilogue, 32 accumulator columns (two 16-row m-tiles of the pass) at a time
-    for (int c0 = 0; c0 < N; c0 += 32) {
-      if (warp == 0) {
-        uint32_t v[32];
-        tmem_ld32(tmem + (uint32_t)c0, v);
+  const int nst = mt.nrb * mt.nkc;
+  for (int st = 0; st < nst; ++st) {
+    const int rb = st / mt.nkc, kc = st - rb * mt.nkc;
+    const int m0 = mt.mt0 + rb * mt.mb, nm = min(mt.mb, mt.mt1 - m0);
+    const int nkb = min(mt.kcb, mt.KB - kc * mt.kcb), kpw = nkb >> 3;
+    // the next stage's k chunk (the same chunks repeat for every row block):
+    // each B fragment register is refilled for it right after its last use
+    const int kn = kc + 1 == mt.nkc ? 0 : kc + 1;
+    const int kpw_n = st + 1 < nst ? min(mt.kcb, mt.KB - kn * mt.kcb) >> 3 : 0;
+    const uint16_t *xn = xb + ((size_t)(kn * mt.kcb + warp) * NN) * 256;
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (got) {
+      trace_first_stage(p, sm, st);
+      const uint8_t *slot = sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes;
+      const bool same = kpw_n == kpw;  // the next stage refills every fragment
+      if (NN == 1 && same && kpw == 6 && nm == 2) {
+        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && same && kpw == 4 && nm == 3) {
+        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && kpw == 6 && nm == 2) {
+        mma_stage_fixed<NN, 2, (NN == 1 ? 6 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (NN == 1 && kpw == 4 && nm == 3) {
+        mma_stage_fixed<NN, 3, (NN == 1 ? 4 : 3), true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 3 && nm == 2) {
+        mma_stage_fixed<NN, 2, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 3 && nm == 3) {
+        mma_stage_fixed<NN, 3, 3, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (same && kpw == 2 && nm == 6) {
+        mma_stage_fixed<NN, 6, 2, false>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 3 && nm == 2) {
+        mma_stage_fixed<NN, 2, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 3 && nm == 3) {
+        mma_stage_fixed<NN, 3, 3, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 2 && nm == 2) {
+        mma_stage_fixed<NN, 2, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else if (kpw == 2 && nm == 3) {
+        mma_stage_fixed<NN, 3, 2, true>(acc, bc, slot, xn, kpw_n, warp, lane);
+      } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sm.cred[j * 33 + lane] = __uint_as_float(v[j]);
+      for (int j = 0; j < mma_max_kpw(NN); ++j) {
+        if (j < kpw) {
+          const uint8_t *blk = slot + (size_t)(warp + 8 * j) * 512 + lane * 16;
+#pragma unroll
+          for (int m = 0; m < kMmaMaxMB; ++m) {
+            if (m < nm) {
+              const uint4 a = *reinterpret_cast<const uint4 *>(blk + (size_t)m * nkb * 512);
+#pragma unroll
+              for (int n = 0; n < NN; ++n) {
+                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].x, bc[j][n].y));  // W hi
+                mma_bf16(acc[m][n], a, make_uint2(bc[j][n].z, bc[j][n].w));  // W lo
+              }
+            }
+          }
+        }
+        if (j < kpw_n) {
+#pragma unroll
+          for (int n = 0; n < NN; ++n)
+            bc[j][n] = __ldcg(reinterpret_cast<const uint4 *>(
+                                  xn + ((size_t)(8 * j) * NN + n) * 256) + lane);
+        }
+      }
+      }
+      release_stage(sm, p, k);
+      ++k;
+    }
+    if (kc + 1 < mt.nkc) continue;
+
+    // row block done: cross-warp sums and the fused epilogue, PM m-tiles per pass
+#pragma unroll
+    for (int q0 = 0; q0 < kMmaMaxMB; q0 += PM) {
+      if (q0 >= nm) break;  // uniform over the CTA
+      {
+        const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+        for (int ml = 0; ml < PM; ++ml) {
+          const int m = q0 + ml;
+          if (m < kMmaMaxMB && m < nm) {
+            float *cw = sm.cred + (size_t)(warp * PM + ml) * 16 * CS;
+#pragma unroll
+            for (int n = 0; n < NN; ++n) {
+              const int c = n * 8 + 2 * tq;
+              cw[g * CS + c] = acc[m][n][0];
+              cw[g * CS + c + 1] = acc[m][n][1];
+              cw[(g + 8) * CS + c] = acc[m][n][2];
+              cw[(g + 8) * CS + c + 1] = acc[m][n][3];
+            }
+          }
+        }
       }
       compute_sync();
+      if (!sm.ctl[kAbort]) {
 #pragma unroll
-      for (int it = 0; it < 32 * NC / kComputeThreads; ++it) {
-        const int ml = (tid + kComputeThreads * it) / (16 * NC);  // m-tile of the chunk, uniform per warp
-        const int j = ml * 16 + row;
-        const bool m_ok = c0 + ml * 16 < N;
-        const float v = m_ok ? sm.cred[j * 33 + col] + sm.cred[j * 33 + NC + col] : 0.f;
-        const int r = u.row0 + q * kUmmaMaxN + c0 + j;  // row of the operator's output
-        const bool store = m_ok && col_ok && r < N_op;
-        const size_t bH = (size_t)col * p.H;
-        if (type == 2) {
-          if (store) L->qkv[(size_t)col * p.n_qkv + r] = v * inv;
-        } else if (type == 5 || type == 7) {
-          // residual add, next operand (gain of the following norm), 16-row ss
-          float x = 0.f;
-          if (store) {
-            x = __ldcg((type == 5 ? L->x_in : L->xm) + bH + r) + v;
-            (type == 5 ? L->xm : L->x_out)[bH + r] = x;
-            const uint16_t *gn = type == 5 ? L->mlp_norm : L->gain_next;
-            put_opnd(type == 5 ? L->xmb : L->xa_next, r, col, NN, x * bf2f(gn[r]));
+        for (int it = 0; it < PM * NC / 16; ++it) {
+          const int ml = (tid + kComputeThreads * it) / (16 * NC);  // uniform per warp
+          const bool m_ok = q0 + ml < nm;
+          float v = 0.f;
+          if (m_ok) {
+#pragma unroll
+            for (int w = 0; w < kComputeWarps; ++w)
+              v += sm.cred[((size_t)(w * PM + ml) * 16 + row) * CS + col];
           }
-          const float s2 = half_warp_sum(x * x);
-          if (store && row == 0)
-            (type == 5 ? L->ssm : L->ssa_next)[(size_t)col * p.n_parts + (r >> 4)] = s2;
-        } else if (type == 6) {
-          // rows (2i, 2i + 1) = (gate_i, up_i) sit on neighbouring lanes
-          const float gv = v * inv;
-          const float uv = __shfl_xor_sync(0xffffffffu, gv, 1);
-          if (store && !(row & 1)) {
-            const int i = r >> 1;
-            const float hv = gv / (1.f + __expf(-gv)) * uv;
-            L->h[(size_t)col * p.F + i] = hv;
-            put_opnd(L->hb, i, col, NN, hv);
-          }
-        } else {
-          const float lv = v * inv;
-          if (store) {
-            if (p.logits && sm.ctl[kLogits]) p.logits[(size_t)col * p.V + r] = lv;
-            if (lv > best_v || (lv == best_v && r < best_i)) {
-              best_v = lv;
-              best_i = r;
+          const int r = (m0 + q0 + ml) * 16 + row;  // row of the operator's output
+          const bool store = m_ok && col_ok && r < N;
+          const size_t bH = (size_t)col * p.H;
+          if (type == 2) {
+            if (store) L->qkv[(size_t)col * p.n_qkv + r] = v * inv;
+          } else if (type == 5 || type == 7) {
+            // residual add, next operand (gain of the following norm), 16-row ss
+            float x = 0.f;
+            if (store) {
+              x = __ldcg((type == 5 ? L->x_in : L->xm) + bH + r) + v;
+              (type == 5 ? L->xm : L->x_out)[bH + r] = x;
+              const uint16_t *gn = type == 5 ? L->mlp_norm : L->gain_next;
+              put_opnd(type == 5 ? L->xmb : L->xa_next, r, col, NN, x * bf2f(gn[r]));
+            }
+            const float s2 = half_warp_sum(x * x);
+            if (store && row == 0)
+              (type == 5 ? L->ssm : L->ssa_next)[(size_t)col * p.n_parts + (r >> 4)] = s2;
+          } else if (type == 6) {
+            // rows (2i, 2i + 1) = (gate_i, up_i) sit on neighbouring lanes
+            const float gv = v * inv;
+            const float uv = __shfl_xor_sync(0xffffffffu, gv, 1);
+            if (store && !(row & 1)) {
+              const int i = r >> 1;
+              const float hv = gv / (1.f + __expf(-gv)) * uv;
+              L->h[(size_t)col * p.F + i] = hv;
+              put_opnd(L->hb, i, col, NN, hv);
+            }
+          } else {
+            const float lv = v * inv;
+            if (store) {
+              if (p.logits && sm.ctl[kLogits]) p.logits[(size_t)col * p.V + r] = lv;
+              if (lv > best_v || (lv == best_v && r < best_i)) {
+                best_v = lv;
+                best_i = r;
+              }
             }
           }
         }
       }
       compute_sync();
     }
-    // the accumulator's reads are complete before the next pass's MMAs
-    tc_fence_before();
-    compute_sync();
+#pragma unroll
+    for (int m = 0; m < kMmaMaxMB; ++m)
+#pragma unroll
+      for (int n = 0; n < NN; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
   }
-  k += (uint32_t)u.nst;
   trace_mark(p, sm, 1);
   if (sm.ctl[kAbort]) return false;
   if (type == 8) {
@@ -1608,7 +1565,7 @@ __device__ __forceinline__ bool umma_task(const Params &p, const Smem &sm, const
           bi = oi;
         }
       }
-      if (bi == 0x7fffffff) bi = u.row0;  // all values NaN: keep a valid index
+      if (bi == 0x7fffffff) bi = mt.mt0 * 16;  // all values NaN: keep a valid index
       p.lm_val[(size_t)tid * p.n_lm + t.idx] = bv;
       p.lm_idx[(size_t)tid * p.n_lm + t.idx] = bi;
     }
@@ -1896,6 +1853,205 @@ __device__ __forceinline__ void attn_block16_mma(uint32_t kbase, uint32_t vbase,
   }
 }
 
+// Decode attention for one (sequence b, kv head g, split s), splits fixed at
+// build time (the default kernels): q/k RMSNorm and RoPE prologue, K/V
+// append, then every warp runs flash-decoding style over
+// its own 8-position blocks on tensor cores (no CTA barrier inside the loop)
+// and the warps' states are merged once at the end.  D: head dim (64, 128);
+// SWZ: the K/V tiles arrive as swizzled TMA boxes (else as plain rows).
+template <int D, bool SWZ>
+__device__ __forceinline__ bool attn_task_fixed(const Params &p, const Smem &sm, const DevTask &t,
+                                                uint32_t &k, int task_id,
+                                                const DepWait &dep_wait) {
+  constexpr int NP = 8;  // positions per warp block
+  // the span read before the wait is exact when the launch runs one step
+  // (kv_len is fixed during it); a multi-step launch re-reads it after the wait
+  const AttnSpan a0 = attn_span(p, (int)t.idx);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rep = p.rep;
+  constexpr int dpl = D >> 5;
+  const DevLayer &L = p.layers[t.layer];
+  const float *qkv = L.qkv + (size_t)a0.b * p.n_qkv + (size_t)a0.g * p.grp;
+  // gains and RoPE factors of this lane's dims (the RoPE position is the
+  // speculative one above): loaded before the wait
+  float gq[4], gk[4], rc[2], rs[2];
+  for (int i = 0; i < dpl; ++i) {
+    gq[i] = bf2f(L.q_norm[lane + 32 * i]);
+    gk[i] = bf2f(L.k_norm[lane + 32 * i]);
+  }
+  auto load_rope = [&](int pos) {  // [D/2][2] cos, sin of position pos
+    const float *rope = p.rope + (size_t)pos * D;
+    for (int i = 0; i < (dpl >> 1); ++i) {
+      rc[i] = rope[2 * (lane + 32 * i)];
+      rs[i] = rope[2 * (lane + 32 * i) + 1];
+    }
+  };
+  load_rope(a0.L);
+  if (!dep_wait()) return false;
+  AttnSpan a = a0;
+  if (p.n_steps > 1) {  // kv_len advanced by the previous step of this launch
+    a = attn_span(p, (int)t.idx);
+    if (a.L != a0.L) load_rope(a.L);
+  }
+  const int nmerge = min(p.S, a.L / p.chunk + 1);  // splits that hold any position
+  if (!a.active)  // the split starts past the new row: it only arrives
+    return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g, p.S, nmerge);
+
+  // prologue: per-head RMSNorm + RoPE of q (and of the new k when this split
+  // holds position L; v is only rounded)
+  for (int row = warp; row < rep + 2; row += kComputeWarps) {
+    if (row >= rep && !a.has_new) continue;
+    float v[4];
+    for (int i = 0; i < dpl; ++i) v[i] = __ldcg(qkv + row * D + lane + 32 * i);
+    if (row <= rep) {  // q heads and k
+      float ss = 0.f;
+      for (int i = 0; i < dpl; ++i) ss = fmaf(v[i], v[i], ss);
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss / (float)D + p.eps);
+      for (int i = 0; i < dpl; ++i) v[i] = v[i] * inv * (row < rep ? gq[i] : gk[i]);
+      const int hp = dpl >> 1;  // dims lane + 32 i pair with lane + 32 (i + hp)
+      for (int i = 0; i < hp; ++i) {
+        const float c = rc[i], s = rs[i];
+        const float x0 = v[i], x1 = v[i + hp];
+        v[i] = x0 * c - x1 * s;
+        v[i + hp] = x1 * c + x0 * s;
+      }
+    }
+    if (row < rep) {
+      for (int i = 0; i < dpl; ++i) sm.q[row * kMaxHeadDim + lane + 32 * i] = v[i] * p.attn_scale;
+    } else {
+      uint16_t *cache = row == rep ? p.k_cache : p.v_cache;
+      uint16_t *dst = row == rep ? sm.knew : sm.vnew;
+      const size_t off = kv_row(p, t.layer, a.b, a.g, a.L);
+      for (int i = 0; i < dpl; ++i) {
+        const uint16_t hb = f2bf(v[i]);
+        cache[off + lane + 32 * i] = hb;
+        dst[lane + 32 * i] = hb;
+      }
+    }
+  }
+  compute_sync();
+  // Q fragments (rows = heads, zero from rep on) as hi/lo bf16 pairs
+  const int gq_row = lane >> 2, tq = lane & 3;
+  uint32_t qh[D / 16][2], ql[D / 16][2];
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c = 16 * kk + 2 * tq + 8 * half;
+      const bool ok = gq_row < rep;
+      const float x0 = ok ? sm.q[gq_row * kMaxHeadDim + c] : 0.f;
+      const float x1 = ok ? sm.q[gq_row * kMaxHeadDim + c + 1] : 0.f;
+      split_pair(x0, x1, qh[kk][half], ql[kk][half]);
+    }
+  }
+  float o[D / 16][4];
+#pragma unroll
+  for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const bool pk = rep <= 4;  // P's hi and lo terms share one MMA
+  // 16-position blocks when the stages hold whole ones (8-position otherwise)
+  const bool np16 = p.pps % (2 * NP) == 0;
+  trace_mark(p, sm, 0);
+
+  const int cached = a.cached_end - a.p0;
+  const int nst = cached > 0 ? (cached + p.pps - 1) / p.pps : 0;
+  for (int st = 0; st < nst; ++st) {
+    const int n = min(p.pps, cached - st * p.pps);
+    const bool got = sm.ctl[kAbort] ? false : wait_full(p, sm, k, task_id);
+    if (!got) continue;
+    trace_first_stage(p, sm, st);
+    const uint32_t kb = smem_u32(sm.ring + (size_t)(k % p.ring_stages) * p.stage_bytes);
+    const uint32_t vb = kb + (uint32_t)(p.pps * D * 2);  // V boxes follow the K boxes
+    // blocks are numbered across the split's stages and dealt round-robin
+    // (warp w takes global blocks w, w + 8, ...), so a stage whose block
+    // count is not a multiple of 8 does not leave the same warps idle every
+    // time; warps drift apart by at most the ring depth
+    if (np16) {
+      const int base = st * (p.pps / (2 * NP));
+      for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * 2 * NP;
+           j0 < n; j0 += kComputeWarps * 2 * NP)
+        attn_block16_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
+    } else {
+      const int base = st * (p.pps / NP);
+      for (int j0 = ((warp - base) % kComputeWarps + kComputeWarps) % kComputeWarps * NP; j0 < n;
+           j0 += kComputeWarps * NP)
+        attn_block_mma<D, SWZ>(kb, vb, p.pps, j0, n, pk, qh, ql, m_run, l_run, o);
+    }
+    release_stage(sm, p, k);
+    ++k;
+  }
+  // the new row: one more block, on the warp after the last cached block
+  const int blk = np16 ? 2 * NP : NP;
+  if (a.has_new && warp == ((cached + blk - 1) / blk) % kComputeWarps)
+    attn_block_mma<D, false>(smem_u32(sm.knew), smem_u32(sm.vnew), 0, 0, 1, pk, qh, ql, m_run, l_run,
+                             o);
+
+  trace_mark(p, sm, 1);
+  if (pk) {  // add the lo-term columns h + 4 into the columns h of lanes tq < 2
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[j][i] += __shfl_down_sync(0xffffffffu, o[j][i], 2);
+  }
+  // every warp's state to shared memory: o (heads 2 tq, 2 tq + 1), then the
+  // running max and sum of head gq_row
+  static_assert(kStateSlots == kComputeWarps, "one state slot per warp");
+  const int stride = D + 2;
+  {
+    float *st_w = sm.ored + (size_t)warp * p.rep_p * stride;
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      const int d = 16 * j + gq_row;
+      if (h0 < rep) {
+        st_w[h0 * stride + d] = o[j][0];
+        st_w[h0 * stride + d + 8] = o[j][2];
+      }
+      if (h1 < rep) {
+        st_w[h1 * stride + d] = o[j][1];
+        st_w[h1 * stride + d + 8] = o[j][3];
+      }
+    }
+    if (tq == 0 && gq_row < rep) {
+      st_w[gq_row * stride + D] = m_run;
+      st_w[gq_row * stride + D + 1] = l_run;
+    }
+  }
+  compute_sync();
+  if (sm.ctl[kAbort]) return false;
+  for (int oi = tid; oi < rep * D; oi += kComputeThreads) {
+    const int h = oi / D, d = oi - h * D;
+    float M = -INFINITY;
+    for (int w = 0; w < kStateSlots; ++w)
+      M = fmaxf(M, sm.ored[((size_t)w * p.rep_p + h) * stride + D]);
+    float num = 0.f, den = 0.f;
+    for (int w = 0; w < kStateSlots; ++w) {
+      const float *sw = sm.ored + ((size_t)w * p.rep_p + h) * stride;
+      const float mw = sw[D];
+      const float e = mw == -INFINITY ? 0.f : __expf(mw - M);
+      den = fmaf(e, sw[D + 1], den);
+      num = fmaf(e, sw[d], num);
+    }
+    const int head = a.g * rep + h;
+    if (p.S == 1) {
+      L.att[(size_t)a.b * p.qdim + head * D + d] = num / den;
+      if (p.mma) put_opnd(L.attb, head * D + d, a.b, p.nn, num / den);
+    } else {
+      float *dst = L.part + (((size_t)a.b * p.Hq + head) * p.S + a.s) * (D + 2);
+      dst[d] = num;
+      if (d == 0) {
+        dst[D] = M;
+        dst[D + 1] = den;
+      }
+    }
+  }
+  if (p.S == 1) return true;
+  return attn_arrive_and_merge(p, sm, t.layer, a.b, a.g, p.S, nmerge);
+}
+
 // Decode attention of one piece (see AttnSeg) on tensor cores: q/k RMSNorm
 // and RoPE prologue, K/V append when the piece holds the new row, then every
 // warp runs flash-decoding style over its own position blocks of the piece's
@@ -2080,9 +2236,9 @@ __device__ __forceinline__ bool attn_piece(const Params &p, const Smem &sm, int 
   return attn_arrive_and_merge(p, sm, layer, sg.b, sg.g, sg.expect, sg.nmerge);
 }
 
-// Decode attention task of the batched kernel: one (sequence b, kv head g,
-// split s) piece when the splits are fixed at build time, else the pieces of
-// JIT task t.idx (see JitCursor).
+// Decode attention task of the extended batched kernels (JIT attention or
+// dispatch mode): one (sequence b, kv head g, split s) piece when the splits
+// are fixed at build time, else the pieces of JIT task t.idx (see JitCursor).
 template <int D, bool SWZ>
 __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const DevTask &t,
                                           uint32_t &k, int task_id, const DepWait &dep_wait) {
@@ -2097,13 +2253,15 @@ __device__ __forceinline__ bool attn_task(const Params &p, const Smem &sm, const
   }
   if (!dep_wait()) return false;
   if (p.jit) {
-    const JitPart jp = jit_part(p);
-    JitCursor cur;
-    cur.start(p, (int)t.idx, jp);
-    AttnSeg sg;
-    while (cur.next(p, sg))
+    JitShared &js = *sm.jit;
+    if (threadIdx.x == 0) js.cur.start(p, (int)t.idx, jit_part(p, js.lens_c));
+    for (;;) {
+      if (threadIdx.x == 0) js.more = js.cur.next(p, js.seg);
+      compute_sync();
+      if (!js.more) return true;
+      const AttnSeg sg = js.seg;
       if (!attn_piece<D, SWZ>(p, sm, t.layer, sg, gq, gk, k, task_id)) return false;
-    return true;
+    }
   }
   // splits fixed at build time; kv_len is read after the wait (a multi-step
   // launch advances it between steps)
@@ -2416,11 +2574,12 @@ __device__ __forceinline__ bool attn_task_cc(const Params &p, const Smem &sm, co
 __device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
   // One item per (k-block kb, sequence b < 8 nn): its 16 embedding elements
   // 16 kb .. 16 kb + 15 (two 16-byte loads) become the fp32 row slice, the
-  // sum of squares of the 16-row part, and layer 0's QKV operand rows hi(b)
-  // and lo(b) of that k-block (two 16-byte units each, see opnd_off): the
-  // elements times the attention-norm gains, zeros for padded sequences.
-  // One CTA does it all, so each thread keeps kU items' loads in flight
-  // before it uses any.
+  // sum of squares of the 16-row part, and the 4 lane units of layer 0's
+  // QKV operand: unit (kb, column tile b / 8, lane (b % 8, t)) holds
+  // elements 16 kb + {2t, 2t + 1, 2t + 8, 2t + 9} times the attention-norm
+  // gains as hi, then lo, bf16 pairs (zeros for padded sequences).  One CTA
+  // does it all, so each thread keeps kU items' loads in flight before it
+  // uses any.
   constexpr int kU = 4;
   const DevLayer &L0 = p.layers[0];
   const int nb8 = 8 * p.nn, items = (p.H >> 4) * nb8;
@@ -2450,28 +2609,30 @@ __device__ __noinline__ void embed_batch(const Params &p, const int32_t *tok) {
                               e[u][1].x, e[u][1].y, e[u][1].z, e[u][1].w};
       const uint32_t gv[8] = {gw[u][0].x, gw[u][0].y, gw[u][0].z, gw[u][0].w,
                               gw[u][1].x, gw[u][1].y, gw[u][1].z, gw[u][1].w};
-      float x[16];
-      uint32_t hi[8], lo[8];
+      float x[16], y[16];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         x[2 * i] = bf_lo(ew[i]);
         x[2 * i + 1] = bf_hi(ew[i]);
-        split_pair(x[2 * i] * bf_lo(gv[i]), x[2 * i + 1] * bf_hi(gv[i]), hi[i], lo[i]);
+        y[2 * i] = x[2 * i] * bf_lo(gv[i]);
+        y[2 * i + 1] = x[2 * i + 1] * bf_hi(gv[i]);
       }
-      // rows hi(b) and lo(b) of k-block kb: 16-byte units (k halves 64 bf16 apart)
-      const size_t o = ((size_t)kb * 256 * p.nn + (b >> 3) * 128 + (b & 7) * 8) >> 3;
-      const size_t lo_o = (size_t)p.nn * 16;  // 8 nn rows further, in 16-byte units
-      xa[o] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      xa[o + 8] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-      xa[o + lo_o] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      xa[o + lo_o + 8] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-      if (b < p.B) {
-        float st[4];
+      float st[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float a0 = x[2 * t], a1 = x[2 * t + 1], a8 = x[2 * t + 8], a9 = x[2 * t + 9];
-          st[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a8, a8, a9 * a9)));
-        }
+      for (int t = 0; t < 4; ++t) {
+        const float a0 = x[2 * t], a1 = x[2 * t + 1], a8 = x[2 * t + 8], a9 = x[2 * t + 9];
+        st[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a8, a8, a9 * a9)));
+        const uint16_t h0 = f2bf(y[2 * t]), h1 = f2bf(y[2 * t + 1]);
+        const uint16_t h8 = f2bf(y[2 * t + 8]), h9 = f2bf(y[2 * t + 9]);
+        uint4 o;
+        o.x = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        o.y = (uint32_t)h8 | ((uint32_t)h9 << 16);
+        o.z = (uint32_t)f2bf(y[2 * t] - bf2f(h0)) | ((uint32_t)f2bf(y[2 * t + 1] - bf2f(h1)) << 16);
+        o.w = (uint32_t)f2bf(y[2 * t + 8] - bf2f(h8)) | ((uint32_t)f2bf(y[2 * t + 9] - bf2f(h9)) << 16);
+        xa[((size_t)kb * p.nn + (b >> 3)) * 32 + (b & 7) * 4 + t] = o;
+      }
+      if (b < p.B) {
+        // the sum in the order of a quad's two butterfly steps
         L0.ssa[(size_t)b * p.n_parts + kb] = (st[0] + st[1]) + (st[2] + st[3]);
         float4 *dst = reinterpret_cast<float4 *>(p.x0 + (size_t)b * p.H + 16 * kb);
 #pragma unroll
@@ -2631,9 +2792,11 @@ __device__ void scheduler_loop(const Params &p, const Smem &sm) {
 // ---------------------------------------------------------------------------
 // kMma: projections on tensor cores (batch >= 2) instead of the CUDA-core
 // GEMV; kNN: the operand's 8-column tiles (1 or 2) of the tensor-core
-// projections (0 at batch 1).  The three modes are separate instantiations
-// so that each gets its own register allocation.
-template <bool kMma, int kNN>
+// projections (0 at batch 1); kExt: the extended kernels (JIT attention and
+// dispatch mode), kept apart so that their code does not raise the register
+// demand of the default kernels.  Each mode is its own instantiation so that
+// each gets its own register allocation.
+template <bool kMma, int kNN, bool kExt>
 __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const Smem sm = carve(smem_raw, p);
@@ -2641,7 +2804,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
   const int warp = tid >> 5;
 
   Queue q;
-  if (p.dispatch) {
+  if (kExt && p.dispatch) {
     if ((int)blockIdx.x == p.n_workers) {  // the scheduler CTA
       if (tid < 32) scheduler_loop(p, sm);
       return;
@@ -2666,9 +2829,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     for (int s = 0; s < p.ring_stages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kComputeWarps);
-      mbar_init(&sm.abar[s], 1);
     }
-    mbar_init(sm.mdone, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     int bad = 0;
     if (*(volatile int32_t *)p.status != 0) bad = 1;  // an earlier step failed: no-op
@@ -2683,6 +2844,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     sm.ctl[kEpoch] = p.persistent ? (int)(*(volatile uint32_t *)p.epoch + 1u) : 0;
     sm.ctl[kConsumed] = 0;
     sm.ctl[kIssued] = 0;
+    sm.ctl[kWindow] = 0;
     sm.tmark[3] = 0;
   }
   __syncthreads();
@@ -2703,34 +2865,18 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
     }
   }
   if (sm.ctl[kAbort]) return;  // nothing issued yet
-  if (kMma) {
-    // the tensor-core projections' accumulators: one allocation per CTA (one
-    // CTA per SM), released on every path below
-    if (warp == 0) {
-      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                       smem_u32(sm.tmem)),
-                   "n"(kUmmaTmemCols)
-                   : "memory");
-      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
-
   if (warp == kComputeWarps) {
-    if ((tid & 31) == 0) producer_loop<kMma>(p, sm, q);
+    if ((tid & 31) == 0) producer_loop<kMma, kExt>(p, sm, q);
     __syncwarp();
   } else {
     const uint32_t epoch0 = (uint32_t)sm.ctl[kEpoch];  // step 0's epoch
     uint32_t k = 0;
-    UmmaState us;
     bool run = true;
     for (int s = 0; s < p.n_steps && run; ++s) {
     const uint32_t epoch = epoch0 + (uint32_t)s;
     if (tid == 0) sm.ctl[kLogits] = s == p.n_steps - 1;  // seen after the next barrier
     for (int n = 0; n < q.count; ++n) {
-      const int id = queue_task(p, sm, q, n);
+      const int id = queue_task<kExt>(p, sm, q, n);
       if (id < 0) break;
       const DevTask t = p.tasks[id];
       uint64_t t_wait = 0;
@@ -2738,7 +2884,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
         t_wait = global_timer();
         sm.tmark[0] = sm.tmark[1] = sm.tmark[2] = sm.tmark[4] = 0;  // tmark[3] accumulates
       }
-      const DepWait dw{p, sm, t.dep, epoch, id};
+      const DepWait dw{p, sm, t.dep, epoch, id, (int)t.type};
       bool ok = true;
       switch (t.type) {
         case 1:
@@ -2755,7 +2901,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
           break;
         case 2: case 5: case 6: case 7: case 8: {
           if constexpr (kMma) {
-            ok = umma_task<kNN == 2 ? 2 : 1>(p, sm, t, k, us, id, dw);
+            ok = mma_task<kNN == 2 ? 2 : 1>(p, sm, t, k, id, dw);
           } else {
             const int K = t.type == 5 ? p.qdim : t.type == 7 ? p.F : p.H;
             const int nch = K >> 3;
@@ -2773,8 +2919,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
         }
         case 3:
           if constexpr (kMma) {
-            ok = p.D == 128 ? attn_task<128, true>(p, sm, t, k, id, dw)
-                            : attn_task<64, true>(p, sm, t, k, id, dw);
+            if constexpr (kExt)
+              ok = p.D == 128 ? attn_task<128, true>(p, sm, t, k, id, dw)
+                              : attn_task<64, true>(p, sm, t, k, id, dw);
+            else
+              ok = p.D == 128 ? attn_task_fixed<128, true>(p, sm, t, k, id, dw)
+                              : attn_task_fixed<64, true>(p, sm, t, k, id, dw);
           } else {
             const int rp = p.rep_p;
             ok = rp <= 2 ? attn_task_cc<2>(p, sm, t, k, id, dw)
@@ -2812,17 +2962,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       }
     }
     }
-    if (tid == 0) {
-      sm.ctl[kConsumed] = (int)k;
-      // operand copies still in flight after an abort land before the CTA exits
-      for (int slot = 0; slot < p.ring_stages; ++slot) {
-        if (!((us.apend >> slot) & 1u)) continue;
-        const uint64_t t0 = global_timer();
-        while (!mbar_test(&sm.abar[slot], (us.aph >> slot) & 1u)) {
-          if (global_timer() - t0 > 4ull * p.timeout_ns + 1000000000ull) break;
-        }
-      }
-    }
+    if (tid == 0) sm.ctl[kConsumed] = (int)k;
   }
   __syncthreads();
   if (sm.ctl[kAbort] && warp == kComputeWarps && (tid & 31) == 0) {
@@ -2851,58 +2991,42 @@ __global__ void __launch_bounds__(kThreads, 1) mk_worker_kernel(const __grid_con
       __threadfence();
     }
   }
-  if (kMma) {
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0)
-      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*sm.tmem),
-                   "n"(kUmmaTmemCols)
-                   : "memory");
-  }
 }
 
-// Weight layout for the tensor-core projections: rows [row_base, row_base +
-// n) of a row-major [rows][K] bf16 matrix (src holds those n rows) to the
-// order umma_tile streams.  Row r belongs to task t = r / task_rows and to
-// pass q = (r % task_rows) / kUmmaMaxN of it; a pass's N rows (the last task
-// is padded to rows_p, a multiple of 16) are contiguous from row
-// t * task_rows + q * kUmmaMaxN on, and per 16-column k-block hold their
-// N x 16 elements in core-matrix order (N * 32 bytes).  One item per 16 bytes
-// (8 elements of a row); padding rows (r >= rows) are zero.
-__global__ void umma_permute_kernel(uint4 *dst, const uint4 *src, int row_base, int rows,
-                                    int rows_p, int K, int task_rows, long long n_items) {
+// Weight layout for the tensor-core path: a row-major [rows][K] bf16 matrix
+// to mma.sync A-fragment order.  Item (m-tile mt, k-block kb, lane) holds the
+// lane's 8 elements, so stage copies and fragment loads are 16 bytes per lane.
+// Rows >= rows (the last m-tile's padding) are zero.
+__global__ void frag_permute_kernel(uint4 *dst, const uint32_t *src, int rows, int K,
+                                    long long n_items) {
   const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (item >= n_items) return;
-  const int cpr = K >> 3;  // 16-byte units per row
-  const int rl = (int)(item / cpr), c = (int)(item - (long long)rl * cpr);
-  const int r = row_base + rl;
-  const int t = r / task_rows, rr = r - t * task_rows;
-  const int q = rr / kUmmaMaxN, i = rr - q * kUmmaMaxN;
-  const int trows = min(task_rows, rows_p - t * task_rows);
-  const int N = min(kUmmaMaxN, trows - q * kUmmaMaxN);
-  const int r0 = t * task_rows + q * kUmmaMaxN;  // first row of the pass
-  const int j = c >> 1, kh = c & 1;
-  const size_t o = (size_t)r0 * cpr + (size_t)j * N * 2 + (size_t)(i >> 3) * 16 + kh * 8 + (i & 7);
-  dst[o] = r < rows ? src[(size_t)rl * cpr + c] : make_uint4(0u, 0u, 0u, 0u);
+  const int lane = (int)(item & 31);
+  const long long blk = item >> 5;
+  const int KB = K >> 4;
+  const int mt = (int)(blk / KB), kb = (int)(blk - (long long)mt * KB);
+  const int r0 = mt * 16 + (lane >> 2), r1 = r0 + 8;
+  const int c = kb * 16 + 2 * (lane & 3);  // even: one 32-bit word holds (c, c + 1)
+  const size_t w = (size_t)K / 2;
+  uint4 o;
+  o.x = r0 < rows ? src[(size_t)r0 * w + c / 2] : 0u;
+  o.y = r1 < rows ? src[(size_t)r1 * w + c / 2] : 0u;
+  o.z = r0 < rows ? src[(size_t)r0 * w + c / 2 + 4] : 0u;
+  o.w = r1 < rows ? src[(size_t)r1 * w + c / 2 + 4] : 0u;
+  dst[item] = o;
 }
 
 }  // namespace
 
-// dst: the whole matrix in the tensor-core layout (rows_p rows); src: its rows
-// [row_base, row_base + n) row-major.  row_base must be a multiple of
-// task_rows; with row_base + n == rows the padding rows up to rows_p are
-// written too.
-cudaError_t permute_to_umma(void *dst, const void *src, int row_base, int n, int rows, int rows_p,
-                            int K, int task_rows, cudaStream_t stream) {
-  const int n_out = row_base + n >= rows ? rows_p - row_base : n;
-  const long long n_items = (long long)n_out * (K / 8);
-  if (n_items <= 0) return cudaSuccess;
+// dst receives ceil(rows / 16) m-tiles of K / 16 fragment blocks (512 bytes each).
+cudaError_t permute_to_fragments(void *dst, const void *src, int rows, int K,
+                                 cudaStream_t stream) {
+  const long long n_items = (long long)((rows + 15) / 16) * (K / 16) * 32;
+  if (n_items == 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n_items + threads - 1) / threads;
-  umma_permute_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-      static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), row_base, rows, rows_p, K,
-      task_rows, n_items);
+  frag_permute_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<uint4 *>(dst), static_cast<const uint32_t *>(src), rows, K, n_items);
   return cudaGetLastError();
 }
 
@@ -2912,14 +3036,21 @@ size_t worker_smem_bytes(int stages, int stage_bytes, int pps, int head_dim, int
 
 // The instantiation for a parameter block's mode.
 static const void *worker_fn(const Params &p) {
-  if (!p.mma) return (const void *)mk_worker_kernel<false, 0>;
-  return p.nn == 2 ? (const void *)mk_worker_kernel<true, 2> : (const void *)mk_worker_kernel<true, 1>;
+  const bool ext = p.jit || p.dispatch;
+  if (!p.mma)
+    return ext ? (const void *)mk_worker_kernel<false, 0, true> : (const void *)mk_worker_kernel<false, 0, false>;
+  if (p.nn == 2)
+    return ext ? (const void *)mk_worker_kernel<true, 2, true> : (const void *)mk_worker_kernel<true, 2, false>;
+  return ext ? (const void *)mk_worker_kernel<true, 1, true> : (const void *)mk_worker_kernel<true, 1, false>;
 }
 
+static const void *const kWorkerFns[] = {
+    (const void *)mk_worker_kernel<false, 0, false>, (const void *)mk_worker_kernel<true, 1, false>,
+    (const void *)mk_worker_kernel<true, 2, false>,  (const void *)mk_worker_kernel<false, 0, true>,
+    (const void *)mk_worker_kernel<true, 1, true>,   (const void *)mk_worker_kernel<true, 2, true>};
+
 cudaError_t worker_configure(size_t smem) {
-  const void *fns[] = {(const void *)mk_worker_kernel<false, 0>, (const void *)mk_worker_kernel<true, 1>,
-                       (const void *)mk_worker_kernel<true, 2>};
-  for (const void *fn : fns) {
+  for (const void *fn : kWorkerFns) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
@@ -2927,10 +3058,8 @@ cudaError_t worker_configure(size_t smem) {
 }
 
 cudaError_t worker_max_blocks(int *blocks, size_t smem) {
-  const void *fns[] = {(const void *)mk_worker_kernel<false, 0>, (const void *)mk_worker_kernel<true, 1>,
-                       (const void *)mk_worker_kernel<true, 2>};
   int lo = 1 << 30;
-  for (const void *fn : fns) {
+  for (const void *fn : kWorkerFns) {
     int n = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, smem);
     if (e != cudaSuccess) return e;

@@ -20,14 +20,13 @@ constexpr int kRedRows = 256;          // GEMV rows whose warp partials shared m
 constexpr int kMaxRep = 8;             // q heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxBatch = 16;
-// Tensor-core projections (batch >= 2) on tcgen05.mma (kind::f16, bf16 in,
-// fp32 accumulators in tensor memory): A = the activation operand (M = 128
-// rows, of which the 16 * nn rows hi(b), lo(b) carry data), B = the task's
-// weight rows (N = up to kUmmaMaxN rows per pass), K = 16 per instruction.
-constexpr int kUmmaMaxN = 256;       // weight rows per pass (TMEM columns)
-constexpr int kUmmaTmemCols = 256;   // tensor-memory columns a CTA allocates
-constexpr int kUmmaSlack = 4096;     // bytes after a stage's operand chunk (see umma_task)
-constexpr int kMmaCredFloats = kComputeWarps * 4 * 16 * 9;  // epilogue scratch (floats)
+// Tensor-core projections (batch >= 2): mma.sync m16n8k16, bf16 in, fp32 out.
+constexpr int kMmaMaxMB = 6;    // 16-row m-tiles per row block (accumulators per warp)
+// 16-column k-blocks per warp and ring stage: a stage's B fragments take
+// kpw x nn x 4 registers per thread, so one column tile (batch <= 8) affords
+// twice as many as two
+__host__ __device__ constexpr int mma_max_kpw(int nn) { return nn == 1 ? 6 : 3; }
+constexpr int kMmaCredFloats = kComputeWarps * 4 * 16 * 9;  // cross-warp reduction buffer
 
 // Device status words: [0] status code, [1] task, [2] event, [3] block.
 enum DeviceStatus : int { kDevOk = 0, kDevTimeout = -6, kDevBadInput = -7 };
@@ -48,8 +47,8 @@ struct DevEvent {  // 16 bytes
 };
 
 // Per-layer device pointers: weight arena slices and activation buffers.
-// With batch >= 2 the four projection matrices are stored in the tensor-core
-// operand order (see umma_permute_kernel in the worker), not row-major.
+// With batch >= 2 the four projection matrices are stored in mma.sync
+// A-fragment order (see frag_permute_kernel in the worker), not row-major.
 struct DevLayer {
   const uint16_t *w_qkv;   // [n_kv_heads * (rep + 2) * D][H], group-major rows
   const uint16_t *w_o;     // [H][Hq * D]
@@ -64,9 +63,9 @@ struct DevLayer {
   float *x_in;  // [B][H]  residual stream entering the layer
   float *x_out; // [B][H]  residual stream leaving the layer
   // Batch >= 2 only: the projection inputs as two-term bf16 expansions
-  // (x = hi + lo) in the tensor-core A-operand order (see opnd_off in the
-  // worker), with the following RMSNorm's gain folded in, and per-16-row sums
-  // of squares [B][H / 16] of the streams that feed an RMSNorm.
+  // (x = hi + lo) in mma.sync B-fragment order (see opnd_off in the worker),
+  // with the following RMSNorm's gain folded in, and per-16-row sums of
+  // squares [B][H / 16] of the streams that feed an RMSNorm.
   uint16_t *xa;    // x_in * attn_norm   (QKV input)
   float *ssa;      // sums of squares of x_in
   uint16_t *attb;  // att                (O input)
@@ -135,9 +134,11 @@ struct Params {
   int rps_qkv, rps_o, rps_gu, rps_down, rps_lm;  // GEMV rows per ring stage
   int pps;  // KV positions per ring stage (multiple of 8): K then V, D / 64 swizzled boxes each
   // tensor-core projections (batch >= 2)
-  int mma;      // 1: projections run on tcgen05.mma with operand-ordered weights
-  int nn;       // 8-sequence column tiles (1 or 2): the operand has 16 * nn rows
+  int mma;      // 1: projections run on mma.sync with fragment-ordered weights
+  int nn;       // 8-sequence column tiles (1 or 2)
   int n_parts;  // H / 16: sum-of-squares partials per sequence
+  int mb_qkv, mb_o, mb_gu, mb_down, mb_lm;        // m-tiles per row block
+  int kcb_qkv, kcb_o, kcb_gu, kcb_down, kcb_lm;   // k-blocks per ring stage
   uint16_t *xfb;  // operand of the LM head: x_final * final_norm
   float *ssf;     // sums of squares of x_final
   // ring

@@ -1,11 +1,10 @@
 """Batched decode steps (2..16 sequences; projections on tensor cores) against
 the CPU oracle, through the C ABI (libmk.so).
 
-With batch >= 2 every projection runs on tcgen05 tensor cores (the hi/lo
-bf16 activation operand against operand-ordered weights, fp32 accumulators in
-tensor memory) and attention on mma.sync over TMA K/V tiles, by default with
-its work cut from the live KV lengths at run time (JIT).  The tolerances are
-those of the batch-1 tests.
+With batch >= 2 every projection runs as mma.sync on fragment-ordered weights
+with hi/lo bf16 activations, and attention on mma.sync over TMA K/V tiles,
+its splits fixed at build time or (attn_jit) cut from the live KV lengths at
+run time.  The tolerances are those of the batch-1 tests.
 """
 import numpy as np
 import pytest
@@ -124,8 +123,8 @@ def test_tiny_batch_eight_position_attention_blocks():
     # blocks; the projections run 1- and 2-m-tile stages of 8 and 16 k-blocks
     w = tiny_batch(8, lo=0, hi=200)
     c = Case(w, seed=34, extra_cap=2, ring_stage_bytes=10240, ring_stages=8)
-    assert c.mk.graph().tiling[6] == 0  # JIT attention: stages of pps rows
-    pps = min(256, 10240 // (4 * w.head_dim) // 8 * 8)
+    chunk = c.mk.graph().tiling[6]
+    pps = min(256, chunk, 10240 // (4 * w.head_dim) // 8 * 8)
     assert pps % 16 != 0
     k, v, lens = c.k.copy(), c.v.copy(), c.lens.copy()
     got = c.gpu_step()
@@ -142,7 +141,7 @@ def _with_lengths(c, lens):
     return c
 
 
-@pytest.mark.parametrize("jit", [1, -1], ids=["jit", "fixed-splits"])
+@pytest.mark.parametrize("jit", [1, 0], ids=["jit", "fixed-splits"])
 def test_tiny_batch_attention_jit_and_fixed_splits_match_oracle(jit):
     # mixed lengths from 0 (only the new row) to 700: JIT pieces that cover
     # the end of one (sequence, kv head) and the start of the next, pairs
@@ -161,7 +160,7 @@ def test_tiny_batch_jit_pieces_over_many_short_pairs():
     # 15 empty caches and one of 900 rows on 148 workers: the short pairs
     # (one position each) share tasks, the long one is cut across many
     w = tiny_batch(16, lo=0, hi=0)
-    c = Case(w, seed=36, extra_cap=904)
+    c = Case(w, seed=36, extra_cap=904, attn_jit=1)
     lens = np.zeros(16, dtype=np.int32)
     lens[11] = 900
     _with_lengths(c, lens)

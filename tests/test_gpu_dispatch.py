@@ -39,7 +39,7 @@ def test_dispatch_mode_runs_one_step_per_launch():
     import persistent_runtime_b200 as prb
     t = torch()
     w = synth.TINY.with_(kv_len=40, steps=2)
-    c = Case(w, seed=52, dispatch=1)
+    c = Case(w, seed=52, extra_cap=4, dispatch=1)
     out = t.zeros((2, w.batch), dtype=t.int32, device="cuda")
     with pytest.raises(prb.MkError):
         c.mk.decode_steps(2, c.d_tok, out, c.d_len, c.d_k, c.d_v, c.d_logits)

@@ -49,16 +49,19 @@ def test_multistep_equals_single_steps_bitwise(w):
     np.testing.assert_array_equal(a[2], c.lens + n)
 
 
-@pytest.mark.parametrize("w,bf16_inputs", [
-    (synth.TINY.with_(kv_len=20, steps=4), False),
-    (synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None, kv_len_range=(0, 300), steps=4), True)],
-    ids=["tiny", "tiny-batch5-split"])
-def test_multistep_matches_oracle_stepwise(w, bf16_inputs):
+@pytest.mark.parametrize("w,bf16_inputs,tuning", [
+    (synth.TINY.with_(kv_len=20, steps=4), False, {}),
+    (synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None, kv_len_range=(0, 300), steps=4), True, {}),
+    (synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None, kv_len_range=(0, 300), steps=4), True,
+     {"attn_jit": 1})],
+    ids=["tiny", "tiny-batch5-split", "tiny-batch5-jit"])
+def test_multistep_matches_oracle_stepwise(w, bf16_inputs, tuning):
     # the oracle replays the launch's steps fed with the tokens the GPU chose:
     # every step's token and appended K/V rows, and the last step's logits and
-    # hidden state, agree within the step tolerances
+    # hidden state, agree within the step tolerances (with JIT attention the
+    # pieces are recut from the lengths every step)
     n = w.steps
-    c = Case(w, seed=42)
+    c = Case(w, seed=42, **tuning)
     toks, logits, lens, gk, gv = _run_steps(c, n)
     last = {"tokens": toks[-1], "logits": logits, "hidden": c.gpu_hidden(), "kv_len": lens}
     lockstep_oracle(c, toks, last, gk.view(np.uint16), gv.view(np.uint16), bf16_inputs, "multistep")

@@ -3,10 +3,8 @@
 The same seeded inputs run through a handle built for contiguous caches and
 one built with kv_page_size = P.  The pools hold the cache rows in pages
 scattered by a random permutation (with spare pages); results must be
-bitwise those of the contiguous run when both stream K/V in stages of the
-same rows (paged handles use 64-row stages; batched handles, whose attention
-cuts its work at run time, get 16 KB ring stages in both runs, i.e. 64-row
-K/V stages, so the arithmetic is the same), the appended rows must land in the right
+bitwise those of the contiguous run (the stage partition is the same in
+these cases, so is the arithmetic), the appended rows must land in the right
 pages, and the oracle, replaying the steps with the GPU's tokens, must agree
 with every step's token, every appended row and the last step's logits and
 hidden state."""
@@ -48,12 +46,11 @@ def from_pool(pool, table, cap):
 
 def run_pair(w, seed, n_steps, against_oracle=False):
     t = torch()
-    tun = {"ring_stage_bytes": 16384} if w.batch > 1 else {}
-    ref = Case(w, seed=seed, **tun)
+    ref = Case(w, seed=seed)
     out_r = t.zeros((n_steps, w.batch), dtype=t.int32, device="cuda")
     ref.mk.decode_steps(n_steps, ref.d_tok, out_r, ref.d_len, ref.d_k, ref.d_v, ref.d_logits)
     assert ref.mk.sync_status()[0] == 0
-    pg = Case(w, seed=seed, kv_page_size=P, **tun)
+    pg = Case(w, seed=seed, kv_page_size=P)
     kp, table, n_pages = to_pool(pg.k, P, seed)
     vp, _, _ = to_pool(pg.v, P, seed)
     d_kp, d_vp = dev_u16(kp), dev_u16(vp)

@@ -92,12 +92,11 @@ def test_jit_spreads_equal_long_pairs_over_all_workers():
 
 
 def test_library_exports_the_jit_tiling():
-    # batch >= 2 handles default to JIT attention: apw * W tasks per layer,
+    # JIT attention (opt-in, batch >= 2): apw * W tasks per layer,
     # S = ceil(apw W / (B Hkv)) + 2 partial slots, chunk 0
     w = synth.Q8B_B16
-    g = prb.plan_graph(w, 8224, 148)
+    g = prb.plan_graph(w, 8224, 148, attn_jit=1)
     assert g.tiling[5] == math.ceil(148 / 128) + 2 and g.tiling[6] == 0
     types, layers = np.asarray(g.task_type), np.asarray(g.task_layer)
     assert int(np.sum((types == 3) & (layers == 0))) == 148
-    g1 = prb.plan_graph(w, 8224, 148, attn_jit=-1)
-    assert g1.tiling[6] > 0
+    assert prb.plan_graph(w, 8224, 148).tiling[6] > 0  # default: splits fixed at build time
