@@ -223,8 +223,8 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1000,
            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic", "config": workload_config(w, lens, args.gpus),
-           "cpu_baseline": {"value": us, "unit": UNIT, "cores": 1, "kind": "oracle",
-                            "sample": sample},
+           "cpu_baseline": dict({"value": us, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": sample}, **host_cpu()),
            "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
     return 0
@@ -254,70 +254,91 @@ def workload_config(w, lens, n):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
-    ap.add_argument("--warmup", type=int, default=8)
-    ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
-    ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-baselines", action="store_true", help="skip the per-operator arms")
-    ap.add_argument("--tuning", default="", help="k=v,... passed to mk_tuning")
-    ap.add_argument("--kv-page-size", type=int, default=0,
-                    help="run on paged K/V pools with this many positions per page")
-    ap.add_argument("--trace", default="", help="write a Chrome trace of one step to this path")
-    args = ap.parse_args()
-    args.warmup = max(3, args.warmup)
-    if args.impl == "reference":
-        return run_reference(args)
+# The other configurations of the same model family, measured by default after
+# the headline workload: (workload, timed steps).  Steps follow the workload's
+# own decode length (64 steps at 0.6B and 8B batch 8, 32 at 8B batch 16).
+OTHER_WORKLOADS = (("qwen3-0.6b", 64), ("qwen3-8b-b8", 64), ("qwen3-8b-b16", 32))
 
-    import torch
-    import torch.distributed as dist
 
-    import persistent_runtime_b200 as prb
+def host_cpu():
+    """Cores and model name of the host (for the CPU baseline's context)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.cuda.current_device()
 
-    w = synth.WORKLOADS[args.workload]
-    cap = int(w.kv_lens(args.seed).max()) + max(args.steps, args.warmup)
-    tuning = {}
-    for kv in filter(None, args.tuning.split(",")):
-        key, val = kv.split("=")
-        tuning[key] = int(val)
+class Gpu:
+    """Process-wide GPU context: torch, the process group, the library."""
 
-    lens = w.kv_lens(args.seed)
-    tokens = synth.make_tokens(w, args.seed)
-    keep_host = rank == 0 and world == 1 and not args.no_cpu_baseline
-    weights = synth.make_weights(w, args.seed)
-    if args.kv_page_size:
-        tuning["kv_page_size"] = args.kv_page_size
-    mk = prb.Megakernel(w, cap, dev, **tuning)
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+
+        import persistent_runtime_b200 as prb
+
+        self.torch, self.dist, self.prb = torch, dist, prb
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            from datetime import timedelta
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                    device_id=torch.device("cuda", local))
+        else:
+            torch.cuda.set_device(0)
+        self.dev = torch.cuda.current_device()
+
+    def barrier(self):
+        self.torch.cuda.synchronize()
+        if self.world > 1:
+            self.dist.barrier()
+        self.torch.cuda.synchronize()
+
+    def max_over_ranks(self, x: float) -> float:
+        return reduce_max(x, self.world, self.dist, "cuda")
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def device_weights(g, w, seed):
+    """Seeded weights of workload w uploaded once (host copy returned too)."""
+    weights = synth.make_weights(w, seed)
+    torch = g.torch
     dw = {"embed": upload(torch, weights["embed"]), "final_norm": upload(torch, weights["final_norm"]),
           "lm_head": None if weights["lm_head"] is None else upload(torch, weights["lm_head"]),
           "layers": [{n: upload(torch, a) for n, a in lw.items()} for lw in weights["layers"]]}
+    return weights, dw
+
+
+def measure(g, w, args, steps, warmup, dw, tuning, *, baselines=True, trace_path="",
+            event_trace=False, keep_host=False):
+    """One workload: µs per step of K single-step launches (the value), the
+    end-to-end loop with host buffers, the per-operator arms, one multi-step
+    launch and, optionally, a traced step (outside every timed region).
+    Returns (result dict, host inputs for the CPU baseline or None)."""
+    torch, prb = g.torch, g.prb
+    lens = w.kv_lens(args.seed)
+    cap = int(lens.max()) + max(steps, warmup)
+    tokens = synth.make_tokens(w, args.seed)
+    mk = prb.Megakernel(w, cap, g.dev, **tuning)
     mk.load_weights(dw)
     torch.cuda.synchronize()
-    del dw
-    if not keep_host:
-        weights = None
-    torch.cuda.empty_cache()
     k_host, v_host = synth.make_kv(w, lens, cap, args.seed)
-    if args.kv_page_size:
+    paged = tuning.get("kv_page_size", 0)
+    if paged:
         # the same rows in pages scattered over the pools by a seeded permutation
-        kp, table, n_pages = paged_pools(k_host, args.kv_page_size, args.seed)
-        vp, _, _ = paged_pools(v_host, args.kv_page_size, args.seed)
+        kp, table, n_pages = paged_pools(k_host, paged, args.seed)
+        vp, _, _ = paged_pools(v_host, paged, args.seed)
         d_k, d_v = upload(torch, kp), upload(torch, vp)
         d_table = torch.from_numpy(table).cuda()
         del kp, vp
@@ -339,29 +360,20 @@ def main():
         if rc != 0:
             raise RuntimeError(f"device status {rc} {detail}")
 
-    def barrier():
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x: float) -> float:
-        return reduce_max(x, world, dist, "cuda")
-
     def timed(fn, k):
         reset()
-        barrier()
+        g.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(k):
             fn()
         e1.record(stream)
-        barrier()
+        g.barrier()
         check()
-        return max_over_ranks(e0.elapsed_time(e1))
+        return g.max_over_ranks(e0.elapsed_time(e1))
 
     def run_steps(n, out):
-        if args.kv_page_size:
+        if paged:
             mk.decode_steps_paged(n, d_tok, out, d_len, d_k, d_v, n_pages, d_table, d_logits)
         else:
             mk.decode_steps(n, d_tok, out, d_len, d_k, d_v, d_logits)
@@ -370,17 +382,17 @@ def main():
 
     # warm-up
     reset()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     check()
 
-    # timed region: persistent megakernel
-    with ClockSampler(dev) as clocks:
-        ms = timed(step, args.steps)
-    us_step = 1000.0 * ms / args.steps
-    bytes_k = steps_bytes(w, lens, args.steps)
+    # timed region: persistent megakernel, one launch per step
+    with ClockSampler(g.dev) as clocks:
+        ms = timed(step, steps)
+    us_step = 1000.0 * ms / steps
+    bytes_k = steps_bytes(w, lens, steps)
     gbs = bytes_k / (ms * 1e-3) / 1e9
-    tok_s = world * w.batch * args.steps / (ms * 1e-3)
+    tok_s = g.world * w.batch * steps / (ms * 1e-3)
 
     # end to end through the public API with host buffers
     h_tok = torch.from_numpy(tokens.copy()).pin_memory()
@@ -394,20 +406,18 @@ def main():
         h_tok.copy_(h_out)
 
     h_tok.copy_(torch.from_numpy(tokens))
-    e2e_ms = timed(e2e_step, args.steps)
-    e2e_us = 1000.0 * e2e_ms / args.steps
+    e2e_us = 1000.0 * timed(e2e_step, steps) / steps
 
-    baselines = {}
-    n_ops = mk.info().n_ops
-    if not args.no_baselines and not args.kv_page_size:  # the per-operator arms take no page table
+    base = {}
+    if baselines and not paged:  # the per-operator arms take no page table
         perop = lambda: mk.decode_step_perop(d_tok, d_tok, d_len, d_k, d_v, d_logits)  # noqa
         reset()
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             perop()
         check()
-        baselines["perop_eager_us"] = 1000.0 * timed(perop, args.steps) / args.steps
+        base["perop_eager_us"] = 1000.0 * timed(perop, steps) / steps
         try:
-            g = torch.cuda.CUDAGraph()
+            cg = torch.cuda.CUDAGraph()
             reset()
             side = torch.cuda.Stream()
             side.wait_stream(stream)
@@ -415,67 +425,115 @@ def main():
                 perop()  # warm the side stream
             torch.cuda.synchronize()
             reset()
-            with torch.cuda.graph(g):
+            with torch.cuda.graph(cg):
                 perop()
             torch.cuda.synchronize()
-            for _ in range(args.warmup):
-                g.replay()
+            for _ in range(warmup):
+                cg.replay()
             check()
-            baselines["perop_graph_us"] = 1000.0 * timed(g.replay, args.steps) / args.steps
-            del g
+            base["perop_graph_us"] = 1000.0 * timed(cg.replay, steps) / steps
+            del cg
         except Exception as e:  # capture refused: report why
-            baselines["perop_graph_error"] = str(e)[:200]
-        baselines["perop_launches_per_step"] = n_ops
+            base["perop_graph_error"] = str(e)[:200]
+        base["perop_launches_per_step"] = mk.info().n_ops
 
     # the same K steps as ONE launch (mk_decode_steps: tokens fed back on the
     # device); reported beside the one-launch-per-step loop above
-    multi_out = torch.zeros((args.steps, w.batch), dtype=torch.int32, device="cuda")
-    multi = lambda: run_steps(args.steps, multi_out)  # noqa: E731
+    multi_out = torch.zeros((steps, w.batch), dtype=torch.int32, device="cuda")
     reset()
-    run_steps(args.warmup, multi_out)
+    run_steps(warmup, multi_out)
     check()
-    multi_us = 1000.0 * timed(multi, 1) / args.steps
+    multi_us = 1000.0 * timed(lambda: run_steps(steps, multi_out), 1) / steps
 
     trace_summary = None
-    if args.trace:
+    if trace_path or event_trace:
         from persistent_runtime_b200 import trace as mktrace
-        g = mk.graph()
-        buf = torch.zeros(8 * g.n_tasks, dtype=torch.int64, device="cuda")
+        gr = mk.graph()
+        buf = torch.zeros(8 * gr.n_tasks, dtype=torch.int64, device="cuda")
         mk.set_trace(buf)
         reset()
         step()
         check()
         mk.set_trace(None)
         tr = buf.cpu().numpy().view(np.uint64)
-        trace_summary = mktrace.summarize(tr, g)
-        mktrace.to_chrome(tr, g, args.trace)
+        trace_summary = mktrace.summarize(tr, gr)
+        if trace_path:
+            mktrace.to_chrome(tr, gr, trace_path)
         trace_summary.pop("op_spans")
 
     peak, peak_kind = measured_peaks()
-    traffic = traffic_record(args.workload)
-    result = {
-        "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": us_step / 1000.0, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(w, lens, world),
-                       **({"kv_page_size": args.kv_page_size} if args.kv_page_size else {})),
+    traffic = traffic_record(w.name)
+    res = {
+        "value": us_step, "unit": UNIT, "steps": steps, "warmup": warmup,
+        "ms_per_step": us_step / 1000.0,
+        "config": dict(workload_config(w, lens, g.world), **({"kv_page_size": paged} if paged else {})),
         "tokens_per_s": tok_s, "hbm_gbs": gbs, "frac_of_8tbs": gbs / HBM_NOMINAL_GBS,
-        "bytes_per_step": bytes_k / args.steps,
+        "bytes_per_step": bytes_k / steps,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                      "frac": gbs / peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "kernel": "mk_worker_kernel (persistent, one launch per step)",
                      "traffic": None if traffic is None else traffic["dram_bytes_per_launch"]},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": 4 * w.batch,
                 "d2h_bytes_per_step": 4 * w.batch},
-        "multistep": {"value": multi_us, "unit": UNIT, "steps_per_launch": args.steps,
+        "multistep": {"value": multi_us, "unit": UNIT, "steps_per_launch": steps,
                       "note": "the same steps in one mk_decode_steps launch"},
-        "gpu_launches": args.steps,
+        "gpu_launches": steps,
         "clocks": clocks.summary(),
-        "baselines": baselines,
+        "baselines": base,
     }
     if trace_summary is not None:
-        result["trace"] = trace_summary
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["event_wait_frac"] = trace_summary["event_wait_frac"]
+        res["trace"] = trace_summary
+    mk.close()
+    host = (lens, tokens, k_host, v_host, cap) if keep_host else None
+    return res, host
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the per-operator arms")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="measure only --workload (by default the line also carries the other "
+                         "configurations of the model family)")
+    ap.add_argument("--tuning", default="", help="k=v,... passed to mk_tuning")
+    ap.add_argument("--kv-page-size", type=int, default=0,
+                    help="run on paged K/V pools with this many positions per page")
+    ap.add_argument("--trace", default="", help="write a Chrome trace of one step to this path")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    g = Gpu()
+    w = synth.WORKLOADS[args.workload]
+    tuning = {}
+    for kv in filter(None, args.tuning.split(",")):
+        key, val = kv.split("=")
+        tuning[key] = int(val)
+    if args.kv_page_size:
+        tuning["kv_page_size"] = args.kv_page_size
+    keep_host = g.rank == 0 and g.world == 1 and not args.no_cpu_baseline
+    weights, dw = device_weights(g, w, args.seed)
+    if not keep_host:
+        weights = None
+    res, host = measure(g, w, args, args.steps, args.warmup, dw, tuning,
+                        baselines=not args.no_baselines, trace_path=args.trace, event_trace=True,
+                        keep_host=keep_host)
+    result = {"metric": METRIC, "value": res.pop("value"), "unit": UNIT, "n_gpus": g.world,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"),
+              "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+              "data": "synthetic", "config": res.pop("config")}
+    res.pop("steps"), res.pop("warmup"), res.pop("unit")
+    result.update(res)
+    if keep_host:
+        lens, tokens, k_host, v_host, cap = host
         if w.batch == 1:
             t = oracle_time_step(w, weights, lens, tokens, k_host, v_host, cap)
             sample = "one full decode step of the same workload, single-threaded fp32 oracle"
@@ -489,12 +547,42 @@ def main():
                                            seq_mask=mask)
             sample = (f"sequence 0's full decode step (kv {int(lens[0])}), single-threaded fp32 "
                       f"oracle, times {w.batch} sequences")
-        result["cpu_baseline"] = {"value": 1e6 * t, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                  "sample": sample}
-    mk.close()
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
+        result["cpu_baseline"] = dict({"value": 1e6 * t, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                       "sample": sample}, **host_cpu())
+        host = k_host = v_host = None
+    weights = None
+
+    if not args.no_other_workloads and not args.kv_page_size:
+        # the other configurations: same model family; the 8B configurations
+        # share the headline's weights (same seed and shapes)
+        others = {}
+        def same_shape(a, b):
+            return (a.n_layers, a.hidden, a.n_q_heads, a.n_kv_heads, a.ffn, a.vocab,
+                    a.tied_embeddings) == (b.n_layers, b.hidden, b.n_q_heads, b.n_kv_heads,
+                                           b.ffn, b.vocab, b.tied_embeddings)
+        # workloads that share the loaded weights first
+        order = sorted(OTHER_WORKLOADS, key=lambda e: not same_shape(synth.WORKLOADS[e[0]], w))
+        cur = w
+        for name, steps in order:
+            ow = synth.WORKLOADS[name]
+            if ow.name == w.name:
+                continue
+            if not same_shape(ow, cur):
+                dw = None
+                g.torch.cuda.empty_cache()
+                _, dw = device_weights(g, ow, args.seed)
+                cur = ow
+            r, _ = measure(g, ow, args, steps, args.warmup, dw, {}, baselines=not args.no_baselines,
+                           event_trace=True)
+            others[r["config"]["workload"]] = {
+                k: r[k] for k in ("value", "unit", "steps", "tokens_per_s", "hbm_gbs",
+                                  "bytes_per_step", "e2e", "multistep", "baselines", "clocks",
+                                  "event_wait_frac")}
+            others[r["config"]["workload"]]["roofline_frac"] = r["roofline"]["frac"]
+        result["other_workloads"] = others
+    dw = None
+    g.close()
+    if g.rank == 0:
         print(json.dumps(result))
     return 0
 
