@@ -15,11 +15,12 @@ def _golden_decode(name):
     w = synth.Workload("golden", cfg["layers"], cfg["hidden"], cfg["q_heads"], cfg["kv_heads"],
                        cfg["head_dim"], cfg["ffn"], cfg["vocab"], 0, cfg["batch"], 1)
     g = oracle.tgraph_decode(w, cfg["kv_capacity"], cfg["workers"], cfg["col_align"],
-                             cfg["apw"], cfg["min_chunk"])
+                             cfg["apw"], cfg["min_chunk"], attn_jit=cfg.get("jit", 0))
     return g, tasks, events
 
 
-@pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt"])
+@pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt",
+                                  "tgraph_tiny1_w2_b2_jit.txt"])
 def test_decode_graph_matches_hand_derived_tables(name):
     g, tasks, events = _golden_decode(name)
     gc.assert_tables_equal(g, tasks, events)

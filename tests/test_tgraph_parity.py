@@ -60,14 +60,18 @@ def test_tuning_variants_bit_exact(col_align, apw, min_chunk):
         gc.assert_graphs_equal(mine, ref)
 
 
-@pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt"])
+@pytest.mark.parametrize("name", ["tgraph_tiny1_w2_s1.txt", "tgraph_tiny1_w2_s4.txt",
+                                  "tgraph_tiny1_w2_b2_jit.txt"])
 def test_decode_goldens(name):
     cfg, _, _, tasks, events = gc.load_golden(name)
     w = synth.Workload("golden", cfg["layers"], cfg["hidden"], cfg["q_heads"], cfg["kv_heads"],
                        cfg["head_dim"], cfg["ffn"], cfg["vocab"], 0, cfg["batch"], 1)
     g = prb.plan_graph(w, cfg["kv_capacity"], cfg["workers"], col_align=cfg["col_align"],
-                       attn_tasks_per_worker=cfg["apw"], attn_min_chunk=cfg["min_chunk"])
+                       attn_tasks_per_worker=cfg["apw"], attn_min_chunk=cfg["min_chunk"],
+                       attn_jit=cfg.get("jit", 0))
     gc.assert_tables_equal(g, tasks, events)
+    if cfg.get("jit", 0):
+        assert g.tiling[5] == 3 and g.tiling[6] == 0  # S slots per pair, chunk set per step
 
 
 @pytest.mark.parametrize("name", ["tgraph_norm_dep.txt", "tgraph_norm_trig.txt"])
