@@ -852,6 +852,12 @@ __device__ void producer_loop(const Params &p, const Smem &sm, const Queue &q) {
   // stream of a step waits until the previous step has completed.  Weight
   // streams are never gated, so they run ahead across the step boundary.
   bool kv_open = s == 0;
+  // the prefetch cursor walks this step's queue from its first task
+  pf_n = 0;
+  pf_st = 0;
+  pfs.nst = -1;
+  pf_k = k;
+  ahead = 0;
   for (int n = 0; n < q.count; ++n) {
     const int tid_n = queue_task<kExt>(p, sm, q, n);
     if (tid_n < 0) break;
