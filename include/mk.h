@@ -97,7 +97,7 @@ typedef struct {
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while
                                 the compute warps wait for an O projection's event (the
                                 step's attention window, when HBM is otherwise idle);
-                                default 524288 at batch 1, off at batch >= 2 (attention
+                                default 2097152 at batch 1, off at batch >= 2 (attention
                                 streams the caches there); negative = off */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
   int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the

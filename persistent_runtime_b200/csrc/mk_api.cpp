@@ -52,11 +52,14 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
   // batch 1: while the compute warps wait for an O projection's event (the
-  // attention window), the producer prefetches up to 512 KB of its following
-  // stages into L2 (Qwen3-8B bs1, one box: 3079 us per step against 3095 us
-  // for 256 KB); at batch >= 2 attention streams the caches in that window.
-  // Negative: off.
-  if (d.l2_prefetch_bytes == 0) d.l2_prefetch_bytes = batch > 1 ? 0 : 512 * 1024;
+  // attention window), the producer prefetches up to 2 MB of its following
+  // stages into L2.  Qwen3-8B bs1, one box, us per step: off 3146, 512 KB
+  // 3121, 1 MB 3083, 2 MB 3064, 4 MB 3064 (the window ends first: about 370 KB
+  // per worker and layer are prefetched at 2 MB); opening the window also
+  // while a worker waits for its attention task's event, or at every event
+  // wait, prefetches more and runs slower (3090, 3126).  At batch >= 2
+  // attention streams the caches in that window.  Negative: off.
+  if (d.l2_prefetch_bytes == 0) d.l2_prefetch_bytes = batch > 1 ? 0 : 2 * 1024 * 1024;
   if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
   return d;
 }

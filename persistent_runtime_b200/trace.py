@@ -72,7 +72,39 @@ def summarize(trace: np.ndarray, graph) -> dict:
     return {"span_us": span, "workers": n_workers, "l2_prefetch_bytes_total": pf_total,
             "event_wait_frac": float(wait.sum() / (n_workers * span)),
             "busy_frac": float(body.sum() / (n_workers * span)),
-            "per_type": per_type, "op_spans": op_spans}
+            "per_type": per_type, "op_spans": op_spans,
+            "layer_phases": layer_phases(trace, graph)}
+
+
+def layer_phases(trace: np.ndarray, graph) -> dict | None:
+    """Mean over decoder layers of where a layer's time goes on the critical
+    path (microseconds): each projection from its first task becoming ready to
+    its last task ending, and the attention window from the last QKV task's
+    end to the first O task's start, in which only K/V rows, attention
+    partials and L2 prefetches move.  `layer_us` runs from one layer's first
+    QKV start to the next one's."""
+    wait0, ready, end, *_ = _fields(trace)
+    ran = end > 0
+    types, layers = np.asarray(graph.task_type), np.asarray(graph.task_layer)
+    spans = {}
+    for ty in (2, 3, 5, 6, 7):
+        for ly in np.unique(layers[ran & (types == ty)]):
+            sel = ran & (types == ty) & (layers == ly)
+            spans[(ty, int(ly))] = (int(ready[sel].min()), int(end[sel].max()))
+    lys = sorted(ly for ty, ly in spans if ty == 2)
+    rows = []
+    for ly in lys:
+        if not all((ty, ly) in spans for ty in (2, 3, 5, 6, 7)):
+            return None
+        q, a, o, g, d = (spans[(ty, ly)] for ty in (2, 3, 5, 6, 7))
+        nxt = spans.get((2, ly + 1))
+        rows.append([q[1] - q[0], o[0] - q[1], a[1] - a[0], o[1] - o[0], g[1] - g[0], d[1] - d[0],
+                     (nxt[0] - q[0]) if nxt else np.nan])
+    if not rows:
+        return None
+    m = np.nanmean(np.asarray(rows, dtype=np.float64), axis=0) / 1e3
+    keys = ("qkv_us", "attn_window_us", "attn_tasks_us", "o_us", "gateup_us", "down_us", "layer_us")
+    return {"layers": len(rows), **{k: float(v) for k, v in zip(keys, m)}}
 
 
 def to_chrome(trace: np.ndarray, graph, path: str) -> None:
