@@ -97,8 +97,11 @@ typedef struct {
   int l2_prefetch_bytes;     /* per-worker L2 prefetch distance ahead of the ring, used while
                                 the compute warps wait for an O projection's event (the
                                 step's attention window, when HBM is otherwise idle);
-                                default 2097152 at batch 1, off at batch >= 2 (attention
-                                streams the caches there); negative = off */
+                                default at batch 1: 2097152 when one layer's weights
+                                exceed 1 MB per worker, else off (the prefetches of small
+                                layers run layers ahead and leave L2 before use); off at
+                                batch >= 2 (attention streams the caches there);
+                                negative = off */
   unsigned wait_timeout_us;  /* device-side bound on one event wait (2,000,000) */
   int kv_page_size;          /* 0: contiguous K/V caches; else positions per page of the
                                 paged pools (a multiple of 64), see mk_decode_steps_paged */
@@ -345,7 +348,8 @@ mk_status mk_debug_set_event_count(mk_handle *h, int event, int count, void *str
 
 /* mk_set_trace - record, for every task of later steps, eight uint64 words
  * {wait begin, ready, end, (smid << 32) | worker, prologue done, streaming
- * done, 0, 0} (%globaltimer ns; the two marks are 0 for tasks without those
+ * done, bytes the worker has prefetched into L2 so far, first ring stage
+ * available} (%globaltimer ns; the phase marks are 0 for tasks without those
  * phases) into the caller's device buffer d_buf of `bytes` >= 64 * n_tasks
  * bytes (task id order).  d_buf = NULL turns tracing off.  The buffer must outlive the steps
  * that use it.  This is the "--profiling" trace of the MPK page, section 7.2. */

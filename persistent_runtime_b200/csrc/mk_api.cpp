@@ -51,17 +51,37 @@ mk_tuning fill_defaults(const mk_tuning *t, int batch = 1) {
   if (d.ring_stages <= 0) d.ring_stages = 4;
   if (d.ring_stage_bytes <= 0) d.ring_stage_bytes = 48 * 1024;
   if (d.wait_timeout_us == 0) d.wait_timeout_us = 2000000u;
-  // batch 1: while the compute warps wait for an O projection's event (the
-  // attention window), the producer prefetches up to 2 MB of its following
-  // stages into L2.  Qwen3-8B bs1, one box, us per step: off 3146, 512 KB
-  // 3121, 1 MB 3083, 2 MB 3064, 4 MB 3064 (the window ends first: about 370 KB
-  // per worker and layer are prefetched at 2 MB); opening the window also
-  // while a worker waits for its attention task's event, or at every event
-  // wait, prefetches more and runs slower (3090, 3126).  At batch >= 2
-  // attention streams the caches in that window.  Negative: off.
-  if (d.l2_prefetch_bytes == 0) d.l2_prefetch_bytes = batch > 1 ? 0 : 2 * 1024 * 1024;
-  if (d.l2_prefetch_bytes < 0) d.l2_prefetch_bytes = 0;
+  // l2_prefetch_bytes: 0 (default) is resolved by default_l2_prefetch once
+  // the worker count is known; negative stays "off" until then
   return d;
+}
+
+// Default distance of the attention-window L2 prefetch.  At batch 1, while the
+// compute warps wait for an O projection's event (the attention window), the
+// producer prefetches up to this many bytes of its following stages into L2.
+// Qwen3-8B bs1, one box, us per step: off 3146, 512 KB 3121, 1 MB 3083, 2 MB
+// 3064, 4 MB 3064 (the window ends first: about 370 KB per worker and layer
+// are prefetched at 2 MB); opening the window also while a worker waits for
+// its attention task's event, or at every event wait, prefetches more and
+// runs slower (3090, 3126).  It pays only where a layer's weights are large
+// per worker: Qwen3-0.6B (0.21 MB per worker and layer against 2.4 MB for 8B)
+// runs 892 us off against 909 us with 2 MB (its prefetches run layers ahead
+// and leave L2 before use: DRAM reads 1.68x the algorithmic bytes) and
+// 894-902 us at 128 KB - 1 MB.  At batch >= 2 attention streams the caches in
+// that window.
+int default_l2_prefetch(const mk_model_config &c, int workers) {
+  if (c.batch > 1) return 0;
+  const double rep = (double)c.n_q_heads / c.n_kv_heads;
+  const double layer_bytes =
+      2.0 * ((double)c.n_kv_heads * (rep + 2.0) * c.head_dim * c.hidden +
+             (double)c.hidden * c.n_q_heads * c.head_dim + 3.0 * (double)c.ffn * c.hidden);
+  return layer_bytes / workers >= 1024.0 * 1024.0 ? 2 * 1024 * 1024 : 0;
+}
+
+// Resolve the defaults that depend on the worker count.
+void resolve_worker_defaults(mk_tuning &t, const mk_model_config &c, int workers) {
+  if (t.l2_prefetch_bytes == 0) t.l2_prefetch_bytes = default_l2_prefetch(c, workers);
+  if (t.l2_prefetch_bytes < 0) t.l2_prefetch_bytes = 0;
 }
 
 std::string check_shape(const mk_model_config &c) {
@@ -154,6 +174,7 @@ mk_status mk_plan_graph(const mk_model_config *cfg, const mk_tuning *tuning, int
   h->cfg = *cfg;
   h->tune = fill_defaults(tuning, cfg->batch);
   h->tune.num_workers = num_workers;
+  resolve_worker_defaults(h->tune, *cfg, num_workers);
   mk_status s = plan(cfg, h->tune, num_workers, h);
   if (s != MK_OK) {
     g_last_error = h->err;
@@ -264,6 +285,7 @@ mk_status mk_build_graph(const mk_model_config *cfg, const mk_tuning *tuning, in
     return fail(nullptr, MK_ERR_ARG, "more workers than co-resident CTAs");
   }
   t.num_workers = W;
+  resolve_worker_defaults(t, c, W);
   mk_status s = plan(cfg, t, W, h);
   if (s != MK_OK) {
     g_last_error = h->err;

@@ -34,14 +34,18 @@ def _run_single(c, n):
             c.d_k.cpu().numpy(), c.d_v.cpu().numpy())
 
 
-@pytest.mark.parametrize("w", [synth.TINY.with_(kv_len=40, steps=6),
-                               synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None,
-                                                kv_len_range=(0, 300), steps=6),
-                               synth.Q06B.with_(steps=4)],
-                         ids=["tiny", "tiny-batch5-split", "qwen3-0.6b"])
-def test_multistep_equals_single_steps_bitwise(w):
+@pytest.mark.parametrize("w,tuning", [(synth.TINY.with_(kv_len=40, steps=6), {}),
+                                      (synth.TINY.with_(name="tiny-b5", batch=5, kv_len=None,
+                                                        kv_len_range=(0, 300), steps=6), {}),
+                                      (synth.Q06B.with_(steps=4), {}),
+                                      # the attention-window L2 prefetch, off by default
+                                      # for layers this small: its cursor restarts
+                                      # with every step of the launch
+                                      (synth.Q06B.with_(steps=4), {"l2_prefetch_bytes": 1 << 20})],
+                         ids=["tiny", "tiny-batch5-split", "qwen3-0.6b", "qwen3-0.6b-prefetch"])
+def test_multistep_equals_single_steps_bitwise(w, tuning):
     n = w.steps
-    c = Case(w, seed=41)
+    c = Case(w, seed=41, **tuning)
     a = _run_steps(c, n)
     b = _run_single(c, n)
     for x, y in zip(a, b):
